@@ -1,0 +1,254 @@
+/*
+ * moe_b200.h -- C ABI of a single-GPU Mixture-of-Experts expert layer for NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes follows "Olmo-core 3" as the three news pages describe it:
+ *   - each token activates k of E experts (noticiarioia.com, "Mudanca de arquitetura e ganhos de
+ *     desempenho"; unite.ai, intro);
+ *   - routing metadata stays on the GPU so the host enqueues work without waiting for copies back
+ *     (bytechap.com, "Como funciona"; unite.ai, "Parallelismo, precisione e tecniche di memoria");
+ *   - routed rows are written straight into each expert's contiguous input buffer ("row-wise"
+ *     expert parallelism; same two sections);
+ *   - one device-scheduled grouped GEMM runs all experts without host synchronisation (unite.ai,
+ *     same section);
+ *   - MXFP8 operands are supported (unite.ai, same section; noticiarioia.com, "Otimizacoes e
+ *     testes em escala de trilhoes").
+ * The formulas the pages leave open are fixed as follows (per token t):
+ *   l_t = W_r x_t (+ bias); S_t = top-k experts of l_t, equal scores to the lower expert id, slots in
+ *   descending score order; g_t,j = softmax(l_t)[S_j] renormalised over S_t;
+ *   out_t = sum_j g_t,j W2_e (silu(W1_e x_t) * W3_e x_t), e = S_t,j, W13_e = [W1_e ; W3_e].
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers unless the argument says "host". The caller allocates and
+ *     owns every buffer; the library never allocates, frees, synchronises the host or copies device
+ *     to host (moe_get_error is the one explicit, caller-requested exception).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). All work is
+ *     enqueued asynchronously on it; results are valid once that stream reaches this point.
+ *   - Tensors are dense row-major. Weights use the [out, in] convention: W_r [E,d], W13 [E,2F,d]
+ *     (rows 0..F-1 gate W1, rows F..2F-1 up W3), W2 [E,d,F].
+ *   - "act" dtype is fp32 when cfg->dtype == MOE_DTYPE_FP32 and bf16 otherwise. Router scores,
+ *     gates and gate gradients are always fp32; index arrays are int32.
+ *   - Routed-row buffers have moe_max_rows(cfg) = T*k + 31*E rows: each expert's group starts on a
+ *     32-row boundary (poff) and its pad rows are kept at zero by the kernels that write the buffer.
+ *   - Every function returns MOE_OK (0) or a negative MOE_ERR_* code. Arguments are validated on the
+ *     host before anything is enqueued; on an error nothing is enqueued.
+ *   - Device-side problems (an expert id outside [0,E), counts that do not add up to T*k, a
+ *     non-finite router score, a bounded wait that ran out) set bits of a sticky int32 flag that
+ *     lives in the first bytes of the workspace; kernels that detect them skip the offending
+ *     accesses and return instead of trapping or spinning. Read it with moe_get_error.
+ *   - Calls are stateless and re-entrant; two calls may share a workspace only if they are ordered
+ *     on the same stream.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---------------------------------------------------------------------------- */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1) /* null pointer, bad size, bad enum value */
+#define MOE_ERR_UNSUPPORTED (-2) /* valid request outside what this build implements */
+#define MOE_ERR_WORKSPACE (-3)   /* workspace missing or smaller than moe_workspace_size() */
+#define MOE_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed (launch, tensor map) */
+
+/* ---- device error flag bits (moe_get_error) --------------------------------------------------- */
+#define MOE_DEVERR_ROUTING 1u  /* expert id out of range or sum(counts) != T*k */
+#define MOE_DEVERR_TIMEOUT 2u  /* a bounded pipeline wait ran out; the kernel returned early */
+#define MOE_DEVERR_NONFINITE 4u/* a router score was NaN or infinite */
+
+/* ---- configuration ----------------------------------------------------------------------------- */
+enum moe_dtype {
+  MOE_DTYPE_FP32 = 0,  /* fp32 storage, GEMMs on tf32 tensor cores, fp32 accumulate */
+  MOE_DTYPE_BF16 = 1,  /* bf16 storage, fp32 accumulate */
+  MOE_DTYPE_MXFP8 = 2  /* bf16 storage, GEMM operands E4M3 + one UE8M0 scale per 32 along K */
+};
+
+typedef struct {
+  int T;      /* tokens, >= 1 */
+  int d;      /* model width, multiple of 64 */
+  int F;      /* expert hidden width, multiple of 128 */
+  int E;      /* experts, 1..256 */
+  int k;      /* experts per token, 1..min(E, 8) */
+  int dtype;  /* enum moe_dtype */
+  int renorm; /* 1: gates renormalised over the chosen k (required by the backward pass) */
+} moe_config_t;
+
+/* Rows of every routed-row buffer: T*k + 31*E. Returns 0 for an invalid config. */
+MOE_API int64_t moe_max_rows(const moe_config_t* cfg);
+
+/* Bytes of scratch the layer-level calls need (routing histograms, router-gradient scratch and the
+ * sticky error flag). The first call on a fresh workspace must be preceded by moe_clear_error (or a
+ * zero fill of the buffer) so that the flag starts at 0. Returns MOE_ERR_INVALID_ARG on a bad cfg. */
+MOE_API int moe_workspace_size(const moe_config_t* cfg, size_t* bytes /* host */);
+
+/* Copy the sticky device error flag to *flags (host) -- synchronises with `stream`. */
+MOE_API int moe_get_error(const void* ws, uint32_t* flags /* host */, void* stream);
+/* Reset the sticky device error flag to 0 (asynchronous on `stream`). */
+MOE_API int moe_clear_error(void* ws, void* stream);
+
+/* ---- routing ------------------------------------------------------------------------------------ */
+
+/* Router scores l = x W_r^T (+ bias), fp32 [T,E]. x: act [T,d]; W_r: act [E,d]; bias: fp32 [E] or
+ * NULL (a constant input with no gradient). Tensor-core GEMM with fp32 accumulation. */
+MOE_API int moe_router_logits(const moe_config_t* cfg, const void* x, const void* W_r, const float* bias,
+                      float* logits, void* ws, size_t ws_bytes, void* stream);
+
+/* Top-k selection and gates (bytechap.com, "Detalles clave": routing scores pick the experts).
+ * logits: fp32 [T,E]; bias: fp32 [E] added before selection and softmax, or NULL.
+ * idx: int32 [T,k] out -- the k largest scores, equal scores to the lower id, descending order.
+ * gates: fp32 [T,k] out -- softmax probabilities of the chosen experts, renormalised over the k
+ * chosen when cfg->renorm. A non-finite score sets MOE_DEVERR_NONFINITE. */
+MOE_API int moe_route_topk(const moe_config_t* cfg, const float* logits, const float* bias, int32_t* idx,
+                   float* gates, void* ws, size_t ws_bytes, void* stream);
+
+/* GPU-resident routing metadata from idx (int32 [T,k]); no host synchronisation (bytechap.com,
+ * "Como funciona"). Outputs (all int32):
+ *   counts[E]      rows routed to each expert;
+ *   offsets[E+1]   exclusive prefix sum of counts, offsets[E] = T*k;
+ *   poff[E+1]      exclusive prefix sum of counts rounded up to 32: expert e owns padded rows
+ *                  [poff[e], poff[e+1]) of every routed-row buffer;
+ *   perm[T*k]      position of entry t*k+j in the expert-sorted order, ascending token id within an
+ *                  expert (a stable counting sort; deterministic, no atomics in the ordering);
+ *   prow[T*k]      padded row of entry t*k+j: poff[e] + perm - offsets[e];
+ *   row_token[max_rows]  entry t*k+j held by each padded row, -1 for pad rows and unused rows.
+ * An expert id outside [0,E) sets MOE_DEVERR_ROUTING; such entries are skipped. */
+MOE_API int moe_route_metadata(const moe_config_t* cfg, const int32_t* idx, int32_t* counts,
+                       int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
+                       int32_t* row_token, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- row-wise dispatch and combine --------------------------------------------------------------- */
+
+/* Row-wise dispatch (unite.ai, "Parallelismo, precisione e tecniche di memoria": each routed token is
+ * written directly into its expert's input buffer): x_perm[prow[t*k+j]] = x[t] for all j, and every
+ * pad row [poff[e]+counts[e], poff[e+1]) is zeroed. x: act [T,d]; x_perm: act [max_rows,d]. */
+MOE_API int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* prow, const int32_t* counts,
+                 const int32_t* poff, void* x_perm, void* stream);
+
+/* Gate-weighted combine: out[t] = sum_j gates[t,j] * y[prow[t*k+j]] (fp32 accumulation, a gather:
+ * deterministic, no atomics). y: act [max_rows,d]; out: act [T,d]. */
+MOE_API int moe_combine(const moe_config_t* cfg, const void* y, const float* gates, const int32_t* prow,
+                void* out, void* stream);
+
+/* Backward of the combine: dy[prow[t*k+j]] = gates[t,j] * dout[t]; dgates[t,j] = <dout[t], y[row]>.
+ * Pad rows of dy are zeroed. When dlsel is non-NULL (learned router, renormalised gates) it also
+ * writes dlsel[t,j] = g_j (dg_j - sum_i g_i dg_i), the score gradient of the chosen experts, and,
+ * when dlogits is non-NULL, the dense score gradient dlogits[t,e] (act [T,E], zero for experts
+ * not chosen). dout: act [T,d]; y: act [max_rows,d]; dy: act [max_rows,d]; dgates, dlsel: fp32 [T,k]. */
+MOE_API int moe_combine_bwd(const moe_config_t* cfg, const void* dout, const void* y, const float* gates,
+                    const int32_t* prow, const int32_t* idx, const int32_t* counts,
+                    const int32_t* poff, void* dy, float* dgates, float* dlsel, void* dlogits,
+                    void* stream);
+
+/* Scatter-add of routed-row gradients back to tokens, done as a deterministic gather-sum:
+ * dx[t] = sum_j dx_perm[prow[t*k+j]] (+ sum_j dlsel[t,j] * W_r[idx[t,j]] when dlsel, idx and W_r
+ * are all non-NULL: the router's input gradient). dx_perm: act [max_rows,d]; dx: act [T,d]. */
+MOE_API int moe_token_reduce(const moe_config_t* cfg, const void* dx_perm, const int32_t* prow,
+                     const float* dlsel, const int32_t* idx, const void* W_r, void* dx, void* stream);
+
+/* ---- device-scheduled grouped GEMM (tcgen05 tensor cores, TMA, TMEM) ------------------------------ */
+
+enum moe_gemm_op {
+  /* h13 = X_e W13_e^T and a = silu(h13[:, :F]) * h13[:, F:] for every expert's rows.
+   * A = x_perm act [max_rows,d]; B = W13 [E,2F,d]; C = h13 act [max_rows,2F]; C2 = a act [max_rows,F]. */
+  MOE_GEMM_FWD1_SWIGLU = 0,
+  /* y = a_e W2_e^T.  A = a [max_rows,F]; B = W2 [E,d,F]; C = y [max_rows,d]. */
+  MOE_GEMM_FWD2 = 1,
+  /* da = dy_e W2_e, then the SwiGLU backward with the saved h13 (aux):
+   * dh13[:, :F] = da * up * silu'(gate), dh13[:, F:] = da * silu(gate).
+   * A = dy [max_rows,d]; B = W2 [E,d,F]; aux = h13 [max_rows,2F]; C = dh13 [max_rows,2F]. */
+  MOE_GEMM_DGRAD2_SWIGLU = 2,
+  /* dx_perm = dh13_e W13_e.  A = dh13 [max_rows,2F]; B = W13 [E,2F,d]; C = dx_perm [max_rows,d]. */
+  MOE_GEMM_DGRAD1 = 3,
+  /* dW2_e = dy_e^T a_e over the expert's rows (zero for an expert with no rows).
+   * A = dy [max_rows,d]; B = a [max_rows,F]; C = dW2 act [E,d,F]. */
+  MOE_GEMM_WGRAD2 = 4,
+  /* dW13_e = dh13_e^T x_perm_e.  A = dh13 [max_rows,2F]; B = x_perm [max_rows,d]; C = dW13 [E,2F,d]. */
+  MOE_GEMM_WGRAD1 = 5
+};
+
+/* One launch runs every expert. The tile schedule is built on the device from counts/poff (as
+ * produced by moe_route_metadata): a persistent grid of one CTA per SM walks the ragged tiles, so the
+ * host never learns the group sizes. Row tiles past an expert's padded end are masked. Rows of the
+ * routed buffers must keep the zero pad rows that dispatch / combine_bwd / this GEMM write. */
+MOE_API int moe_grouped_gemm(const moe_config_t* cfg, int op, const void* A, const void* B, void* C, void* C2,
+                     const void* aux, const int32_t* counts, const int32_t* poff, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/* Router weight gradient dW_r = dlogits^T x (act [E,d]) from the dense score gradient written by
+ * moe_combine_bwd (act [T,E]); a single-group tensor-core GEMM contracting over tokens. */
+MOE_API int moe_router_wgrad(const moe_config_t* cfg, const void* dlogits, const void* x, void* dW_r,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* ---- whole layer ------------------------------------------------------------------------------------ */
+
+typedef struct {
+  const void* W_r; /* act [E,d]; NULL when routing is given as input (saved->idx / saved->gates) */
+  const void* W13; /* act [E,2F,d] */
+  const void* W2;  /* act [E,d,F] */
+} moe_weights_t;
+
+/* Forward results kept for the backward pass. Caller-owned device buffers. */
+typedef struct {
+  float* logits;      /* fp32 [T,E] (learned router only, else may be NULL) */
+  int32_t* idx;       /* [T,k]  output, or INPUT when W_r == NULL */
+  float* gates;       /* [T,k]  output, or INPUT when W_r == NULL */
+  int32_t* counts;    /* [E] */
+  int32_t* offsets;   /* [E+1] */
+  int32_t* poff;      /* [E+1] */
+  int32_t* perm;      /* [T*k] */
+  int32_t* prow;      /* [T*k] */
+  int32_t* row_token; /* [max_rows] */
+  void* x_perm;       /* act [max_rows,d] */
+  void* h13;          /* act [max_rows,2F] */
+  void* a;            /* act [max_rows,F] */
+  void* y;            /* act [max_rows,d] */
+} moe_saved_t;
+
+/* Gradients (outputs) and backward scratch (caller-owned device buffers). */
+typedef struct {
+  void* dW_r;    /* act [E,d] (learned router only, else may be NULL) */
+  void* dW13;    /* act [E,2F,d] */
+  void* dW2;     /* act [E,d,F] */
+  float* dgates; /* fp32 [T,k] */
+  void* dy;      /* act [max_rows,d]   scratch */
+  void* dh13;    /* act [max_rows,2F]  scratch */
+  void* dx_perm; /* act [max_rows,d]   scratch */
+} moe_grads_t;
+
+/* Whole forward: [router scores -> top-k] -> metadata -> dispatch -> grouped GEMM1 + SwiGLU ->
+ * grouped GEMM2 -> combine. x: act [T,d]; bias: fp32 [E] or NULL; out: act [T,d]. */
+MOE_API int moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* w, const void* x, const float* bias,
+                  void* out, moe_saved_t* saved, void* ws, size_t ws_bytes, void* stream);
+
+/* Whole backward given dout (act [T,d]): combine_bwd -> GEMM2 dgrad + SwiGLU bwd -> GEMM2 wgrad ->
+ * GEMM1 dgrad -> GEMM1 wgrad -> token reduce (+ router terms). x is the forward input. The
+ * selection is held fixed (no gradient through the top-k choice). Requires cfg->renorm == 1 when
+ * the router is learned. */
+MOE_API int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_saved_t* saved,
+                  const void* x, const void* dout, void* dx, moe_grads_t* g, void* ws,
+                  size_t ws_bytes, void* stream);
+
+/* ---- test support ------------------------------------------------------------------------------------- */
+
+/* Launch one block whose thread waits on a pipeline barrier that nothing ever completes, with the
+ * library's bounded wait and the given limit (ns). It must give up, set MOE_DEVERR_TIMEOUT in the
+ * workspace flag and return; used to check the timeout path without hanging a GPU. */
+MOE_API int moe_test_bounded_wait(void* ws, uint64_t limit_ns, void* stream);
+
+/* Library version string (host). */
+MOE_API const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

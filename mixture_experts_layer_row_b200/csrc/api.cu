@@ -1,0 +1,358 @@
+// C ABI of the MoE expert layer library: argument validation, workspace layout, and the forward /
+// backward composition of the kernels. Every entry point validates on the host and enqueues nothing
+// on an error; all work is asynchronous on the caller's stream; nothing here allocates.
+#include <cstring>
+
+#include "internal.h"
+
+using namespace moe;
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s per pipeline wait
+
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round256(size_t b) { return (b + 255) & ~size_t(255); }
+
+int check_cfg(const moe_config_t* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 1 || c->d < 1 || c->F < 1 || c->E < 1 || c->k < 1) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_DTYPE_FP32 && c->dtype != MOE_DTYPE_BF16 && c->dtype != MOE_DTYPE_MXFP8)
+    return MOE_ERR_INVALID_ARG;
+  if (c->renorm != 0 && c->renorm != 1) return MOE_ERR_INVALID_ARG;
+  if (c->k > c->E) return MOE_ERR_INVALID_ARG;
+  if (c->E > 256 || c->k > 8) return MOE_ERR_UNSUPPORTED;
+  if (c->d % 64 != 0 || c->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  const int64_t rows = (int64_t)c->T * c->k + 31ll * c->E;
+  if (rows >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+inline int es_of(const moe_config_t* c) { return c->dtype == MOE_DTYPE_FP32 ? 4 : 2; }
+inline int64_t max_rows_of(const moe_config_t* c) { return (int64_t)c->T * c->k + 31ll * c->E; }
+
+struct WsLayout {
+  size_t head, hist, dlsel, dlogits, total;
+};
+
+WsLayout ws_layout(const moe_config_t* c) {
+  WsLayout w;
+  w.head = 0;
+  w.hist = kWsHeadBytes;
+  w.dlsel = w.hist + round256(metadata_ws_bytes(c->T, c->E));
+  w.dlogits = w.dlsel + round256((size_t)c->T * c->k * sizeof(float));
+  w.total = w.dlogits + round256((size_t)c->T * c->E * es_of(c));
+  return w;
+}
+
+int check_ws(const moe_config_t* c, void* ws, size_t ws_bytes) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < ws_layout(c).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+inline uint32_t* err_of(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
+
+#define MOE_TRY(expr)            \
+  do {                           \
+    const int _r = (expr);       \
+    if (_r != MOE_OK) return _r; \
+  } while (0)
+
+#define MOE_REQUIRE(cond, code) \
+  do {                          \
+    if (!(cond)) return (code); \
+  } while (0)
+
+GemmParams base_params(const moe_config_t* c, void* ws) {
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.E = c->E;
+  p.F = c->F;
+  p.vec_ok = 1;
+  p.err = ws ? err_of(ws) : nullptr;
+  p.wait_limit_ns = kWaitLimitNs;
+  return p;
+}
+
+int gemm_op(const moe_config_t* c, int op, const void* A, const void* B, void* Cout, void* C2,
+            const void* aux, const int32_t* counts, const int32_t* poff, void* ws, cudaStream_t s) {
+  const int es = es_of(c);
+  const int64_t R = max_rows_of(c);
+  const int d = c->d, F = c->F, E = c->E;
+  GemmParams p = base_params(c, ws);
+  p.counts = counts;
+  p.poff = poff;
+  p.C = Cout;
+  GemmOperand a{A, 0, 0, 0}, b{B, 0, 0, 0};
+  switch (op) {
+    case MOE_GEMM_FWD1_SWIGLU:
+      MOE_REQUIRE(C2, MOE_ERR_INVALID_ARG);
+      a = {A, R, d, d};
+      b = {B, (int64_t)E * 2 * F, d, d};
+      p.K = d; p.N = F; p.b_rows_per_group = 2 * F; p.ldc = 2 * F; p.C2 = C2; p.ldc2 = F;
+      return launch_gemm(GK_FWD1_SWIGLU, es, 256, a, b, p, s);
+    case MOE_GEMM_FWD2:
+      a = {A, R, F, F};
+      b = {B, (int64_t)E * d, F, F};
+      p.K = F; p.N = d; p.b_rows_per_group = d; p.ldc = d;
+      return launch_gemm(GK_FWD2, es, d >= 256 ? 256 : 128, a, b, p, s);
+    case MOE_GEMM_DGRAD2_SWIGLU:
+      MOE_REQUIRE(aux, MOE_ERR_INVALID_ARG);
+      MOE_REQUIRE(aligned16(aux), MOE_ERR_INVALID_ARG);
+      a = {A, R, d, d};
+      b = {B, (int64_t)E * d, F, F};
+      p.K = d; p.N = F; p.b_rows_per_group = d; p.aux = aux; p.ldaux = 2 * F; p.ldc = 2 * F;
+      return launch_gemm(GK_DGRAD2_SWIGLU, es, F >= 256 ? 256 : 128, a, b, p, s);
+    case MOE_GEMM_DGRAD1:
+      a = {A, R, 2 * F, 2 * F};
+      b = {B, (int64_t)E * 2 * F, d, d};
+      p.K = 2 * F; p.N = d; p.b_rows_per_group = 2 * F; p.ldc = d;
+      return launch_gemm(GK_DGRAD1, es, d >= 256 ? 256 : 128, a, b, p, s);
+    case MOE_GEMM_WGRAD2:
+      a = {A, R, d, d};
+      b = {B, R, F, F};
+      p.M = d; p.N = F; p.ldc = F; p.c_group_stride = (int64_t)d * F;
+      return launch_gemm(GK_WGRAD, es, F >= 256 ? 256 : 128, a, b, p, s);
+    case MOE_GEMM_WGRAD1:
+      a = {A, R, 2 * F, 2 * F};
+      b = {B, R, d, d};
+      p.M = 2 * F; p.N = d; p.ldc = d; p.c_group_stride = (int64_t)2 * F * d;
+      return launch_gemm(GK_WGRAD, es, d >= 256 ? 256 : 128, a, b, p, s);
+    default:
+      return MOE_ERR_INVALID_ARG;
+  }
+}
+
+int router_logits_impl(const moe_config_t* c, const void* x, const void* Wr, const float* bias,
+                       float* logits, void* ws, cudaStream_t s) {
+  GemmParams p = base_params(c, ws);
+  p.counts = nullptr;
+  p.M = c->T; p.K = c->d; p.N = c->E; p.b_rows_per_group = 0;
+  p.C = logits; p.ldc = c->E; p.bias = bias;
+  p.vec_ok = (c->E % 4 == 0);
+  GemmOperand a{x, c->T, c->d, c->d}, b{Wr, c->E, c->d, c->d};
+  return launch_gemm(GK_ROUTER, es_of(c), c->E <= 128 ? 128 : 256, a, b, p, s);
+}
+
+int router_wgrad_impl(const moe_config_t* c, const void* dlogits, const void* x, void* dWr, void* ws,
+                      cudaStream_t s) {
+  GemmParams p = base_params(c, ws);
+  p.counts = nullptr;
+  p.M = c->E; p.N = c->d; p.K = c->T;
+  p.C = dWr; p.ldc = c->d; p.c_group_stride = 0;
+  GemmOperand a{dlogits, c->T, c->E, c->E}, b{x, c->T, c->d, c->d};
+  return launch_gemm(GK_WGRAD, es_of(c), c->d >= 256 ? 256 : 128, a, b, p, s);
+}
+
+bool router_shape_ok(const moe_config_t* c) {
+  // the dense score-gradient [T,E] is a TMA operand: its rows must be 16-byte multiples
+  return ((size_t)c->E * es_of(c)) % 16 == 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_version(void) { return "moe_b200 0.1 (sm_100a)"; }
+
+int64_t moe_max_rows(const moe_config_t* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return max_rows_of(cfg);
+}
+
+int moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(bytes, MOE_ERR_INVALID_ARG);
+  *bytes = ws_layout(cfg).total;
+  return MOE_OK;
+}
+
+int moe_get_error(const void* ws, uint32_t* flags, void* stream) {
+  MOE_REQUIRE(ws && flags, MOE_ERR_INVALID_ARG);
+  if (cudaMemcpyAsync(flags, ws, sizeof(uint32_t), cudaMemcpyDeviceToHost, S(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cudaStreamSynchronize(S(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_clear_error(void* ws, void* stream) {
+  MOE_REQUIRE(ws, MOE_ERR_INVALID_ARG);
+  return cudaMemsetAsync(ws, 0, sizeof(uint32_t), S(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_router_logits(const moe_config_t* cfg, const void* x, const void* W_r, const float* bias,
+                      float* logits, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(cfg->dtype != MOE_DTYPE_MXFP8, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(x && W_r && logits, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(x) && aligned16(W_r) && aligned16(logits), MOE_ERR_INVALID_ARG);
+  return router_logits_impl(cfg, x, W_r, bias, logits, ws, S(stream));
+}
+
+int moe_route_topk(const moe_config_t* cfg, const float* logits, const float* bias, int32_t* idx,
+                   float* gates, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(logits && idx && gates, MOE_ERR_INVALID_ARG);
+  return launch_topk(logits, bias, cfg->T, cfg->E, cfg->k, cfg->renorm, idx, gates, err_of(ws),
+                     S(stream));
+}
+
+int moe_route_metadata(const moe_config_t* cfg, const int32_t* idx, int32_t* counts,
+                       int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
+                       int32_t* row_token, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(idx && counts && offsets && poff && perm && prow && row_token, MOE_ERR_INVALID_ARG);
+  const WsLayout L = ws_layout(cfg);
+  int32_t* hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.hist);
+  return launch_metadata(idx, cfg->T, cfg->E, cfg->k, max_rows_of(cfg), counts, offsets, poff, perm,
+                         prow, row_token, hist, err_of(ws), S(stream));
+}
+
+int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* prow, const int32_t* counts,
+                 const int32_t* poff, void* x_perm, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(cfg->dtype != MOE_DTYPE_MXFP8, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(x && prow && counts && poff && x_perm, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(x) && aligned16(x_perm), MOE_ERR_INVALID_ARG);
+  return launch_dispatch(x, prow, counts, poff, x_perm, cfg->T, cfg->k, cfg->E, cfg->d * es_of(cfg),
+                         S(stream));
+}
+
+int moe_combine(const moe_config_t* cfg, const void* y, const float* gates, const int32_t* prow,
+                void* out, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(y && gates && prow && out, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(y) && aligned16(out), MOE_ERR_INVALID_ARG);
+  return launch_combine(y, gates, prow, out, cfg->T, cfg->k, cfg->d * es_of(cfg), es_of(cfg) == 2,
+                        S(stream));
+}
+
+int moe_combine_bwd(const moe_config_t* cfg, const void* dout, const void* y, const float* gates,
+                    const int32_t* prow, const int32_t* idx, const int32_t* counts,
+                    const int32_t* poff, void* dy, float* dgates, float* dlsel, void* dlogits,
+                    void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(dout && y && gates && prow && counts && poff && dy && dgates, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(dout) && aligned16(y) && aligned16(dy), MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(!dlogits || (dlsel && idx), MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(!dlsel || cfg->renorm == 1, MOE_ERR_UNSUPPORTED);
+  return launch_combine_bwd(dout, y, gates, prow, idx, counts, poff, dy, dgates, dlsel, dlogits,
+                            cfg->T, cfg->k, cfg->E, cfg->d * es_of(cfg), es_of(cfg) == 2, S(stream));
+}
+
+int moe_token_reduce(const moe_config_t* cfg, const void* dx_perm, const int32_t* prow,
+                     const float* dlsel, const int32_t* idx, const void* W_r, void* dx, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(dx_perm && prow && dx, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(dx_perm) && aligned16(dx) && (!W_r || aligned16(W_r)), MOE_ERR_INVALID_ARG);
+  return launch_token_reduce(dx_perm, prow, dlsel, idx, W_r, dx, cfg->T, cfg->k, cfg->E,
+                             cfg->d * es_of(cfg), es_of(cfg) == 2, S(stream));
+}
+
+int moe_grouped_gemm(const moe_config_t* cfg, int op, const void* A, const void* B, void* C, void* C2,
+                     const void* aux, const int32_t* counts, const int32_t* poff, void* ws,
+                     size_t ws_bytes, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(cfg->dtype != MOE_DTYPE_MXFP8, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(A && B && C && counts && poff, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(A) && aligned16(B) && aligned16(C) && (!C2 || aligned16(C2)),
+              MOE_ERR_INVALID_ARG);
+  return gemm_op(cfg, op, A, B, C, C2, aux, counts, poff, ws, S(stream));
+}
+
+int moe_router_wgrad(const moe_config_t* cfg, const void* dlogits, const void* x, void* dW_r, void* ws,
+                     size_t ws_bytes, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(cfg->dtype != MOE_DTYPE_MXFP8, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(dlogits && x && dW_r, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(dlogits) && aligned16(x) && aligned16(dW_r), MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(router_shape_ok(cfg), MOE_ERR_UNSUPPORTED);
+  return router_wgrad_impl(cfg, dlogits, x, dW_r, ws, S(stream));
+}
+
+int moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* w, const void* x, const float* bias,
+                  void* out, moe_saved_t* sv, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(cfg->dtype != MOE_DTYPE_MXFP8, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(w && sv && x && out && w->W13 && w->W2, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(sv->idx && sv->gates && sv->counts && sv->offsets && sv->poff && sv->perm && sv->prow &&
+                  sv->row_token && sv->x_perm && sv->h13 && sv->a && sv->y,
+              MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(x) && aligned16(out) && aligned16(w->W13) && aligned16(w->W2) &&
+                  aligned16(sv->x_perm) && aligned16(sv->h13) && aligned16(sv->a) &&
+                  aligned16(sv->y),
+              MOE_ERR_INVALID_ARG);
+  cudaStream_t s = S(stream);
+  if (w->W_r) {
+    MOE_REQUIRE(sv->logits && aligned16(w->W_r) && aligned16(sv->logits), MOE_ERR_INVALID_ARG);
+    MOE_TRY(router_logits_impl(cfg, x, w->W_r, bias, sv->logits, ws, s));
+    MOE_TRY(launch_topk(sv->logits, nullptr, cfg->T, cfg->E, cfg->k, cfg->renorm, sv->idx, sv->gates,
+                        err_of(ws), s));
+  }
+  const WsLayout L = ws_layout(cfg);
+  int32_t* hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.hist);
+  MOE_TRY(launch_metadata(sv->idx, cfg->T, cfg->E, cfg->k, max_rows_of(cfg), sv->counts, sv->offsets,
+                          sv->poff, sv->perm, sv->prow, sv->row_token, hist, err_of(ws), s));
+  MOE_TRY(launch_dispatch(x, sv->prow, sv->counts, sv->poff, sv->x_perm, cfg->T, cfg->k, cfg->E,
+                          cfg->d * es_of(cfg), s));
+  MOE_TRY(gemm_op(cfg, MOE_GEMM_FWD1_SWIGLU, sv->x_perm, w->W13, sv->h13, sv->a, nullptr, sv->counts,
+                  sv->poff, ws, s));
+  MOE_TRY(gemm_op(cfg, MOE_GEMM_FWD2, sv->a, w->W2, sv->y, nullptr, nullptr, sv->counts, sv->poff, ws,
+                  s));
+  return launch_combine(sv->y, sv->gates, sv->prow, out, cfg->T, cfg->k, cfg->d * es_of(cfg),
+                        es_of(cfg) == 2, s);
+}
+
+int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_saved_t* sv,
+                  const void* x, const void* dout, void* dx, moe_grads_t* g, void* ws,
+                  size_t ws_bytes, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(cfg->dtype != MOE_DTYPE_MXFP8, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(w && sv && g && x && dout && dx && w->W13 && w->W2, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(g->dW13 && g->dW2 && g->dgates && g->dy && g->dh13 && g->dx_perm, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(dout) && aligned16(dx) && aligned16(g->dW13) && aligned16(g->dW2) &&
+                  aligned16(g->dy) && aligned16(g->dh13) && aligned16(g->dx_perm),
+              MOE_ERR_INVALID_ARG);
+  const bool router = w->W_r != nullptr;
+  if (router) {
+    MOE_REQUIRE(cfg->renorm == 1, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(router_shape_ok(cfg), MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(g->dW_r && aligned16(g->dW_r), MOE_ERR_INVALID_ARG);
+  }
+  cudaStream_t s = S(stream);
+  const WsLayout L = ws_layout(cfg);
+  float* dlsel = router ? reinterpret_cast<float*>(static_cast<char*>(ws) + L.dlsel) : nullptr;
+  void* dlog = router ? static_cast<void*>(static_cast<char*>(ws) + L.dlogits) : nullptr;
+  const int rb = cfg->d * es_of(cfg);
+  const bool bf = es_of(cfg) == 2;
+  MOE_TRY(launch_combine_bwd(dout, sv->y, sv->gates, sv->prow, sv->idx, sv->counts, sv->poff, g->dy,
+                             g->dgates, dlsel, dlog, cfg->T, cfg->k, cfg->E, rb, bf, s));
+  MOE_TRY(gemm_op(cfg, MOE_GEMM_DGRAD2_SWIGLU, g->dy, w->W2, g->dh13, nullptr, sv->h13, sv->counts,
+                  sv->poff, ws, s));
+  MOE_TRY(gemm_op(cfg, MOE_GEMM_WGRAD2, g->dy, sv->a, g->dW2, nullptr, nullptr, sv->counts, sv->poff,
+                  ws, s));
+  MOE_TRY(gemm_op(cfg, MOE_GEMM_DGRAD1, g->dh13, w->W13, g->dx_perm, nullptr, nullptr, sv->counts,
+                  sv->poff, ws, s));
+  MOE_TRY(gemm_op(cfg, MOE_GEMM_WGRAD1, g->dh13, sv->x_perm, g->dW13, nullptr, nullptr, sv->counts,
+                  sv->poff, ws, s));
+  MOE_TRY(launch_token_reduce(g->dx_perm, sv->prow, dlsel, router ? sv->idx : nullptr, w->W_r, dx,
+                              cfg->T, cfg->k, cfg->E, rb, bf, s));
+  if (router) MOE_TRY(router_wgrad_impl(cfg, dlog, x, g->dW_r, ws, s));
+  return MOE_OK;
+}
+
+int moe_test_bounded_wait(void* ws, uint64_t limit_ns, void* stream) {
+  MOE_REQUIRE(ws, MOE_ERR_INVALID_ARG);
+  return launch_bounded_wait_probe(err_of(ws), limit_ns, S(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,622 @@
+// Device-scheduled grouped GEMM on the 5th-generation tensor cores (tcgen05), the one dense
+// contraction of the MoE layer ("grouped GEMM combines many small expert computations",
+// bytechap.com "Como funciona"; "device-scheduled grouped matrix multiplications that make expert
+// parallelism completely synchronisation-free", unite.ai "Parallelismo, precisione e tecniche di
+// memoria").
+//
+// Structure (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: one elected thread streams A/B tiles into a STAGES-deep shared-memory
+//               ring (128-byte swizzle), completion counted on a "full" mbarrier per stage;
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, fp32 accumulate) into
+//               one of two TMEM accumulators and frees each ring stage with tcgen05.commit;
+//   warps 2..5  epilogue: tcgen05.ld the finished accumulator (one row per thread), apply the fused
+//               op (store, SwiGLU forward, SwiGLU backward, fp32 + bias) and store to global memory,
+//               while the MMA thread already fills the other accumulator.
+// The tile schedule is built on the device from the routing metadata (counts, padded offsets): the
+// host never learns the group sizes. Two grouping modes:
+//   GROUP_M  ragged rows per expert (forward and dgrad): tiles (expert, n-block, m-block), m fastest
+//            so CTAs running at the same time share the expert's weight block through L2;
+//   GROUP_K  ragged contraction per expert (wgrad): tiles (expert, m-block, n-block), the K loop runs
+//            over the expert's 32-aligned row range in 32-row chunks (zero pad rows make the tail
+//            exact); an expert with no rows writes a zero gradient.
+// Every mbarrier wait is bounded; on a timeout the CTA raises MOE_DEVERR_TIMEOUT, drains what it has
+// in flight (bounded), frees TMEM and returns.
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+
+template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
+struct Cfg {
+  static constexpr int EPR = 128 / ES;       // elements per 128-byte smem row
+  static constexpr int BK = EPR;             // K elements per pipeline stage
+  static constexpr int UK = 32 / ES;         // K per tcgen05.mma (32 bytes)
+  static constexpr int KSTEPS = BK / UK;     // MMAs per full stage (4)
+  static constexpr int CHUNKS = BK / 32;     // 32-row K chunks per stage (MN-major operands)
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;   // two accumulators
+  static constexpr int BN_OUT = (EPI == EPI_SWIGLU_FWD) ? BN / 2 : BN;  // output columns per tile
+  static constexpr uint32_t IDESC = instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, BM, BN);
+  static constexpr size_t SMEM_BYTES =
+      1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + 1024 /*barriers etc*/ + 257 * 4;
+};
+
+struct TileInfo {
+  int e;        // group
+  int m0;       // GROUP_M: first row (relative to the group start); GROUP_K: first output row
+  int n0;       // first output column
+  int rows;     // GROUP_M: valid rows of the group (padded count); GROUP_K: M
+  int kstart;   // GROUP_M: unused; GROUP_K: first contraction row in the routed buffer
+  int nchunks;  // number of 32-row K chunks (GROUP_K) or K/BK stages (GROUP_M)
+  int row_base; // GROUP_M: poff[e]
+};
+
+template <class C, int MODE>
+__device__ __forceinline__ int num_kstages(const TileInfo& ti) {
+  if constexpr (MODE == GROUP_M) return ti.nchunks;
+  else return (ti.nchunks + C::CHUNKS - 1) / C::CHUNKS;
+}
+
+template <class C, int EPI, int MODE>
+__device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const int* prefix,
+                                          int n_tiles, int m_tiles_fixed, TileInfo& ti) {
+  if constexpr (MODE == GROUP_M) {
+    int e = 0;
+    if (p.counts) {
+      int lo = 0, hi = p.E - 1;  // largest e with prefix[e] <= tile
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+      }
+      e = lo;
+    }
+    const int local = tile - prefix[e];
+    const int rows = p.counts ? (p.poff[e + 1] - p.poff[e]) : p.M;
+    const int mt = (rows + BM - 1) / BM;
+    ti.e = e;
+    ti.n0 = (local / mt) * C::BN_OUT;
+    ti.m0 = (local % mt) * BM;
+    ti.rows = rows;
+    ti.row_base = p.counts ? p.poff[e] : 0;
+    ti.kstart = 0;
+    ti.nchunks = p.K / C::BK;
+  } else {
+    const int per = m_tiles_fixed * n_tiles;
+    const int e = tile / per;
+    const int local = tile - e * per;
+    ti.e = e;
+    ti.m0 = (local / n_tiles) * BM;
+    ti.n0 = (local % n_tiles) * (C::B_BYTES / 128);
+    ti.rows = p.M;
+    ti.row_base = 0;
+    if (p.counts) {
+      ti.kstart = p.poff[e];
+      ti.nchunks = (p.poff[e + 1] - p.poff[e]) / 32;
+    } else {
+      ti.kstart = 0;
+      ti.nchunks = (p.K + 31) / 32;
+    }
+  }
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.f + expf(-g)); }
+
+// Store 32 consecutive fp32 values as bf16 (64 bytes) or fp32 (128 bytes).
+template <int ES>
+__device__ __forceinline__ void store32(void* dst, const float* v) {
+  if constexpr (ES == 2) {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      d[q] = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                        pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+  } else {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      d[q] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                        __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+  }
+}
+
+template <int ES>
+__device__ __forceinline__ void store_masked(void* base, int col0, int ncols, const float* v) {
+  for (int c = 0; c < 32; ++c) {
+    if (col0 + c < ncols) {
+      if constexpr (ES == 2)
+        reinterpret_cast<__nv_bfloat16*>(base)[c] = __float2bfloat16_rn(v[c]);
+      else
+        reinterpret_cast<float*>(base)[c] = v[c];
+    }
+  }
+}
+
+template <int ES>
+__device__ __forceinline__ void load32(const void* src, float* v) {
+  if constexpr (ES == 2) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 w = s[q];
+      v[8 * q + 0] = bf16lo(w.x); v[8 * q + 1] = bf16hi(w.x);
+      v[8 * q + 2] = bf16lo(w.y); v[8 * q + 3] = bf16hi(w.y);
+      v[8 * q + 4] = bf16lo(w.z); v[8 * q + 5] = bf16hi(w.z);
+      v[8 * q + 6] = bf16lo(w.w); v[8 * q + 7] = bf16hi(w.w);
+    }
+  } else {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint4 w = s[q];
+      v[4 * q] = __uint_as_float(w.x); v[4 * q + 1] = __uint_as_float(w.y);
+      v[4 * q + 2] = __uint_as_float(w.z); v[4 * q + 3] = __uint_as_float(w.w);
+    }
+  }
+}
+
+template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+  using C = Cfg<ES, A_MN, B_MN, BN, EPI, MODE>;
+  static_assert(MODE == GROUP_M || (A_MN && B_MN), "wgrad mode needs MN-major operands");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* smA = smem;
+  uint8_t* smB = smem + (size_t)C::STAGES * C::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smB + (size_t)C::STAGES * C::B_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* tfull = bars + 2 * C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_word = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* prefix = reinterpret_cast<int*>(tmem_slot + 2);  // [E+1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- device-side tile schedule ----
+  int n_tiles, m_tiles_fixed = 0, total;
+  if constexpr (MODE == GROUP_M) {
+    n_tiles = (p.N + C::BN_OUT - 1) / C::BN_OUT;
+    const int G = p.counts ? p.E : 1;
+    for (int e = threadIdx.x; e < G; e += blockDim.x) {
+      const int rows = p.counts ? (p.poff[e + 1] - p.poff[e]) : p.M;
+      prefix[e + 1] = ((rows + BM - 1) / BM) * n_tiles;
+    }
+    __syncthreads();
+    if (warp == 0) {  // inclusive scan of per-group tile counts, 8 groups per lane
+      int loc[8], s = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane * 8 + i;
+        loc[i] = e < G ? prefix[e + 1] : 0;
+        s += loc[i];
+      }
+      int inc = s;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += o;
+      }
+      int run = inc - s;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = lane * 8 + i;
+        run += loc[i];
+        if (e < G) prefix[e + 1] = run;
+      }
+      if (lane == 0) prefix[0] = 0;
+    }
+    __syncthreads();
+    total = prefix[p.counts ? p.E : 1];
+  } else {
+    n_tiles = (p.N + BN - 1) / BN;
+    m_tiles_fixed = (p.M + BM - 1) / BM;
+    total = (p.counts ? p.E : 1) * m_tiles_fixed * n_tiles;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kEpiThreads);
+    }
+    mbar_init(done, 1);
+    *abort_word = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ===================== TMA producer =====================
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        TileInfo ti;
+        tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
+        const int nst = num_kstages<C, MODE>(ti);
+        for (int ks = 0; ks < nst; ++ks, ++it) {
+          const int s = it % C::STAGES;
+          if (!mbar_wait_bounded(&empty[s], ((it / C::STAGES) & 1) ^ 1, p.wait_limit_ns, abort_word,
+                                 p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a_dst = smA + (size_t)s * C::A_BYTES;
+          uint8_t* b_dst = smB + (size_t)s * C::B_BYTES;
+          if constexpr (MODE == GROUP_M) {
+            const int k0 = ks * C::BK;
+            mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+            // A: K-major rows of the routed buffer (or the token matrix)
+            tma_load_2d(a_dst, &tmA, &full[s], k0, ti.row_base + ti.m0);
+            if constexpr (!B_MN) {
+              const int brow = ti.e * p.b_rows_per_group;
+              if constexpr (EPI == EPI_SWIGLU_FWD) {
+                tma_load_2d(b_dst, &tmB, &full[s], k0, brow + ti.n0);                       // gate
+                tma_load_2d(b_dst + (BN / 2) * 128, &tmB, &full[s], k0, brow + p.F + ti.n0);  // up
+              } else {
+                tma_load_2d(b_dst, &tmB, &full[s], k0, brow + ti.n0);
+              }
+            } else {
+              // MN-major weight [E*K rows, N cols]: BN/EPR column blocks x BK rows, 32-row boxes
+              const int krow = ti.e * p.b_rows_per_group + k0;
+#pragma unroll
+              for (int blk = 0; blk < BN / C::EPR; ++blk)
+#pragma unroll
+                for (int ch = 0; ch < C::CHUNKS; ++ch)
+                  tma_load_2d(b_dst + blk * (C::BK * 128) + ch * 4096, &tmB, &full[s],
+                              ti.n0 + blk * C::EPR, krow + ch * 32);
+            }
+          } else {
+            // GROUP_K: both operands MN-major, contraction rows kstart + 32*chunk
+            const int c0 = ks * C::CHUNKS;
+            const int nch = min(C::CHUNKS, ti.nchunks - c0);
+            mbar_arrive_expect_tx(&full[s], nch * 32 * 128 * ((BM + BN) / C::EPR));
+            for (int ch = 0; ch < nch; ++ch) {
+              const int krow = ti.kstart + (c0 + ch) * 32;
+#pragma unroll
+              for (int blk = 0; blk < BM / C::EPR; ++blk)
+                tma_load_2d(a_dst + blk * (C::BK * 128) + ch * 4096, &tmA, &full[s],
+                            ti.m0 + blk * C::EPR, krow);
+#pragma unroll
+              for (int blk = 0; blk < BN / C::EPR; ++blk)
+                tma_load_2d(b_dst + blk * (C::BK * 128) + ch * 4096, &tmB, &full[s],
+                            ti.n0 + blk * C::EPR, krow);
+            }
+          }
+        }
+      }
+      // drain: every load this thread issued must have landed before the CTA exits
+      for (int j = max(0, it - C::STAGES); j < it; ++j)
+        mbar_wait_bounded(&full[j % C::STAGES], (j / C::STAGES) & 1, p.wait_limit_ns, nullptr, p.err);
+    }
+  } else if (warp == 1) {
+    // ===================== MMA issuer =====================
+    if (lane == 0) {
+      int it = 0, local = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+        TileInfo ti;
+        tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
+        const int nst = num_kstages<C, MODE>(ti);
+        const int buf = local & 1;
+        if (!mbar_wait_bounded(&tempty[buf], ((local >> 1) & 1) ^ 1, p.wait_limit_ns, abort_word,
+                               p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int ks = 0; ks < nst; ++ks, ++it) {
+          const int s = it % C::STAGES;
+          if (!mbar_wait_bounded(&full[s], (it / C::STAGES) & 1, p.wait_limit_ns, abort_word, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smA + (size_t)s * C::A_BYTES);
+          const uint32_t b_addr = smem_u32(smB + (size_t)s * C::B_BYTES);
+          int nk = C::KSTEPS;
+          if constexpr (MODE == GROUP_K) nk = min(C::CHUNKS, ti.nchunks - ks * C::CHUNKS) * (32 / C::UK);
+          for (int kk = 0; kk < nk; ++kk) {
+            uint64_t ad, bd;
+            if constexpr (A_MN) ad = smem_desc_sw128(a_addr + kk * C::UK * 128, C::BK * 128, 1024);
+            else ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+            if constexpr (B_MN) bd = smem_desc_sw128(b_addr + kk * C::UK * 128, C::BK * 128, 1024);
+            else bd = smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+            umma<ES == 2 ? 0 : 1>(d_tmem, ad, bd, C::IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
+            issued = true;
+          }
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        if (nst > 0) umma_commit(&tfull[buf]);
+        else mbar_arrive(&tfull[buf]);
+      }
+      // all MMAs issued by this thread must be complete before TMEM is released
+      if (issued) {
+        umma_commit(done);
+        mbar_wait_bounded(done, 0, p.wait_limit_ns, nullptr, p.err);
+      }
+    }
+  } else {
+    // ===================== epilogue (warps 2..5) =====================
+    const int q = warp & 3;               // TMEM lane quadrant this warp may access
+    const int r = q * 32 + lane;          // accumulator row owned by this thread
+    int local = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+      TileInfo ti;
+      tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
+      const int nst = num_kstages<C, MODE>(ti);
+      const int buf = local & 1;
+      int ok = 1;
+      if (lane == 0)
+        ok = mbar_wait_bounded(&tfull[buf], (local >> 1) & 1, p.wait_limit_ns, abort_word, p.err);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+      const bool row_ok = (ti.m0 + r) < ti.rows;
+      if constexpr (MODE == GROUP_K) {
+        // weight gradient of group e: C[e][m0 + r][n0 + c]
+        char* crow = reinterpret_cast<char*>(p.C) +
+                     ((size_t)ti.e * p.c_group_stride + (size_t)(ti.m0 + r) * p.ldc + ti.n0) * ES;
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          if (nst > 0) {
+            uint32_t raw[32];
+            tmem_ld_32x32b_x32(t_row + c, raw);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+          if (row_ok) {
+            if (p.vec_ok && ti.n0 + c + 32 <= p.N) store32<ES>(crow + (size_t)c * ES, v);
+            else if (ti.n0 + c < p.N) store_masked<ES>(crow + (size_t)c * ES, ti.n0 + c, p.N, v);
+          }
+        }
+      } else {
+        const size_t grow = (size_t)ti.row_base + ti.m0 + r;  // row in the routed buffer
+        if constexpr (EPI == EPI_SWIGLU_FWD) {
+          char* hrow = reinterpret_cast<char*>(p.C) + grow * p.ldc * ES;
+          char* arow = reinterpret_cast<char*>(p.C2) + grow * p.ldc2 * ES;
+          for (int c = 0; c < BN / 2; c += 32) {
+            uint32_t rg[32], ru[32];
+            tmem_ld_32x32b_x32(t_row + c, rg);
+            tmem_ld_32x32b_x32(t_row + BN / 2 + c, ru);
+            tmem_ld_wait();
+            float g[32], u[32], a[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              g[i] = __uint_as_float(rg[i]);
+              u[i] = __uint_as_float(ru[i]);
+              a[i] = silu_f(g[i]) * u[i];
+            }
+            if (row_ok) {
+              store32<ES>(hrow + (size_t)(ti.n0 + c) * ES, g);
+              store32<ES>(hrow + (size_t)(p.F + ti.n0 + c) * ES, u);
+              store32<ES>(arow + (size_t)(ti.n0 + c) * ES, a);
+            }
+          }
+        } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+          const char* hrow = reinterpret_cast<const char*>(p.aux) + grow * p.ldaux * ES;
+          char* drow = reinterpret_cast<char*>(p.C) + grow * p.ldc * ES;
+          for (int c = 0; c < BN; c += 32) {
+            uint32_t rd[32];
+            tmem_ld_32x32b_x32(t_row + c, rd);
+            tmem_ld_wait();
+            if (row_ok && ti.n0 + c < p.N) {
+              float g[32], u[32], dg[32], du[32];
+              load32<ES>(hrow + (size_t)(ti.n0 + c) * ES, g);
+              load32<ES>(hrow + (size_t)(p.F + ti.n0 + c) * ES, u);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float da = __uint_as_float(rd[i]);
+                const float sg = 1.f / (1.f + expf(-g[i]));
+                du[i] = da * g[i] * sg;
+                dg[i] = da * u[i] * sg * (1.f + g[i] * (1.f - sg));
+              }
+              store32<ES>(drow + (size_t)(ti.n0 + c) * ES, dg);
+              store32<ES>(drow + (size_t)(p.F + ti.n0 + c) * ES, du);
+            }
+          }
+        } else {
+          // plain store (EPI_STORE: act dtype) or fp32 + bias (EPI_STORE_F32_BIAS)
+          constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : ES;
+          char* crow = reinterpret_cast<char*>(p.C) + (grow * p.ldc + ti.n0) * OES;
+          for (int c = 0; c < BN; c += 32) {
+            uint32_t raw[32];
+            tmem_ld_32x32b_x32(t_row + c, raw);
+            tmem_ld_wait();
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+            if constexpr (EPI == EPI_STORE_F32_BIAS) {
+              if (p.bias)
+                for (int i = 0; i < 32; ++i)
+                  if (ti.n0 + c + i < p.N) v[i] += p.bias[ti.n0 + c + i];
+            }
+            if (row_ok) {
+              if (p.vec_ok && ti.n0 + c + 32 <= p.N) store32<OES>(crow + (size_t)c * OES, v);
+              else if (ti.n0 + c < p.N) store_masked<OES>(crow + (size_t)c * OES, ti.n0 + c, p.N, v);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ------------------------------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `es`-byte elements, box [box_rows, box_cols], 128B swizzle.
+bool make_tmap(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t cols, int64_t ld,
+               int box_cols, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        2, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!n[dev]) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
+  return n[dev] > 0 ? n[dev] : 148;
+}
+
+template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
+int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p, int grid_cap,
+                cudaStream_t s) {
+  using C = Cfg<ES, A_MN, B_MN, BN, EPI, MODE>;
+  auto kern = grouped_gemm_kernel<ES, A_MN, B_MN, BN, EPI, MODE>;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)C::SMEM_BYTES) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  CUtensorMap ta, tb;
+  // A box: K-major -> [BM rows, EPR cols]; MN-major -> [32 rows, EPR cols]
+  if (!make_tmap(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, A_MN ? 32 : BM)) return MOE_ERR_CUDA;
+  int b_box_rows = B_MN ? 32 : (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN);
+  if (!make_tmap(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, b_box_rows)) return MOE_ERR_CUDA;
+  int grid = sm_count();
+  if (grid_cap > 0 && grid_cap < grid) grid = grid_cap;
+  if (grid < 1) grid = 1;
+  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+// Dispatch a GEMM request to its compiled variant. The caller (api.cu) has validated shapes.
+int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
+                const GemmParams& p, cudaStream_t s) {
+  // GROUP_K launches know their tile count on the host; cap the grid there.
+  int cap = 0;
+  if (kind == GK_WGRAD) {
+    const int mt = (p.M + BM - 1) / BM, nt = (p.N + bn - 1) / bn;
+    const int64_t total = (int64_t)(p.counts ? p.E : 1) * mt * nt;
+    cap = total < 1 ? 1 : (int)(total < (1 << 30) ? total : (1 << 30));
+  }
+#define MOE_GEMM_CASES(ES_)                                                                          \
+  switch (kind) {                                                                                    \
+    case GK_FWD1_SWIGLU:                                                                             \
+      return launch_impl<ES_, false, false, 256, EPI_SWIGLU_FWD, GROUP_M>(A, B, p, cap, s);          \
+    case GK_FWD2:                                                                                    \
+      if (bn == 256) return launch_impl<ES_, false, false, 256, EPI_STORE, GROUP_M>(A, B, p, cap, s); \
+      return launch_impl<ES_, false, false, 128, EPI_STORE, GROUP_M>(A, B, p, cap, s);               \
+    case GK_DGRAD2_SWIGLU:                                                                           \
+      if (bn == 256)                                                                                 \
+        return launch_impl<ES_, false, true, 256, EPI_SWIGLU_BWD, GROUP_M>(A, B, p, cap, s);         \
+      return launch_impl<ES_, false, true, 128, EPI_SWIGLU_BWD, GROUP_M>(A, B, p, cap, s);           \
+    case GK_DGRAD1:                                                                                  \
+      if (bn == 256) return launch_impl<ES_, false, true, 256, EPI_STORE, GROUP_M>(A, B, p, cap, s);  \
+      return launch_impl<ES_, false, true, 128, EPI_STORE, GROUP_M>(A, B, p, cap, s);                \
+    case GK_WGRAD:                                                                                   \
+      if (bn == 256) return launch_impl<ES_, true, true, 256, EPI_STORE, GROUP_K>(A, B, p, cap, s);   \
+      return launch_impl<ES_, true, true, 128, EPI_STORE, GROUP_K>(A, B, p, cap, s);                 \
+    case GK_ROUTER:                                                                                  \
+      if (bn == 256)                                                                                 \
+        return launch_impl<ES_, false, false, 256, EPI_STORE_F32_BIAS, GROUP_M>(A, B, p, cap, s);    \
+      return launch_impl<ES_, false, false, 128, EPI_STORE_F32_BIAS, GROUP_M>(A, B, p, cap, s);      \
+  }
+  if (es == 2) {
+    MOE_GEMM_CASES(2)
+  } else {
+    MOE_GEMM_CASES(4)
+  }
+#undef MOE_GEMM_CASES
+  return MOE_ERR_UNSUPPORTED;
+}
+
+// Bounded-wait self-test: wait on a barrier nobody arrives at.
+__global__ void bounded_wait_probe_kernel(uint32_t* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_word = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, limit_ns, &abort_word, err);
+}
+
+int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s) {
+  bounded_wait_probe_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

@@ -1,0 +1,65 @@
+// Internal declarations shared by the translation units of libmoe_b200 (not part of the C ABI).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// Grouped GEMM epilogues and grouping modes.
+enum { EPI_STORE = 0, EPI_SWIGLU_FWD = 1, EPI_SWIGLU_BWD = 2, EPI_STORE_F32_BIAS = 3 };
+enum { GROUP_M = 0, GROUP_K = 1 };
+
+enum GemmKind { GK_FWD1_SWIGLU, GK_FWD2, GK_DGRAD2_SWIGLU, GK_DGRAD1, GK_WGRAD, GK_ROUTER };
+
+// A row-major 2-D operand as the TMA unit sees it.
+struct GemmOperand {
+  const void* ptr;
+  int64_t rows, cols, ld;  // ld in elements
+};
+
+struct GemmParams {
+  const int32_t* counts;  // [E] rows per group, or nullptr for one group
+  const int32_t* poff;    // [E+1] 32-aligned group starts
+  int E;
+  int M;  // GROUP_K: output rows per group; single-group GROUP_M: rows
+  int N;  // output columns (GROUP_M SwiGLU forward: F)
+  int K;  // GROUP_M: contraction length; single-group GROUP_K: contraction rows
+  int b_rows_per_group;  // rows of the weight operand's 2-D view per group
+  void* C;
+  int64_t ldc;
+  void* C2;
+  int64_t ldc2;
+  const void* aux;
+  int64_t ldaux;
+  const float* bias;
+  int F;
+  int64_t c_group_stride;  // GROUP_K: elements between two groups' outputs
+  int vec_ok;              // output rows allow 16-byte vector stores
+  uint32_t* err;
+  uint64_t wait_limit_ns;
+};
+
+int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
+                const GemmParams& p, cudaStream_t s);
+int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s);
+
+int launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm, int32_t* idx,
+                float* gates, uint32_t* err, cudaStream_t s);
+size_t metadata_ws_bytes(int T, int E);
+int launch_metadata(const int32_t* idx, int T, int E, int k, int64_t max_rows, int32_t* counts,
+                    int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
+                    int32_t* row_token, int32_t* hist_ws, uint32_t* err, cudaStream_t s);
+
+int launch_dispatch(const void* x, const int32_t* prow, const int32_t* counts, const int32_t* poff,
+                    void* xp, int T, int k, int E, int row_bytes, cudaStream_t s);
+int launch_combine(const void* y, const float* gates, const int32_t* prow, void* out, int T, int k,
+                   int row_bytes, bool bf16, cudaStream_t s);
+int launch_combine_bwd(const void* dout, const void* y, const float* gates, const int32_t* prow,
+                       const int32_t* idx, const int32_t* counts, const int32_t* poff, void* dy,
+                       float* dgates, float* dlsel, void* dlogits, int T, int k, int E, int row_bytes,
+                       bool bf16, cudaStream_t s);
+int launch_token_reduce(const void* dxp, const int32_t* prow, const float* dlsel, const int32_t* idx,
+                        const void* Wr, void* dx, int T, int k, int E, int row_bytes, bool bf16,
+                        cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,319 @@
+// Row movement between token order and expert-grouped order, all HBM-bound and written as
+// coalesced 16-byte vector loops (one warp per token, every lane moving 16-byte chunks of the row):
+//   dispatch      x[t] -> x_perm[prow[t,j]] for j < k, read once and written k times ("row-wise"
+//                 placement straight into each expert's contiguous input buffer: bytechap.com, "Como
+//                 funciona"; unite.ai, "Parallelismo, precisione e tecniche di memoria"); pad rows 0.
+//   combine       out[t] = sum_j g[t,j] y[prow[t,j]]  (a gather: deterministic, no atomics)
+//   combine_bwd   dy[prow[t,j]] = g[t,j] dout[t];  dg[t,j] = <dout[t], y[prow[t,j]]> (+ score grads)
+//   token_reduce  dx[t] = sum_j dx_perm[prow[t,j]] (+ sum_j dl[t,j] W_r[idx[t,j]])
+// Every routed-row pad row (the tail of each expert's 32-aligned group) is written as zero by
+// dispatch and combine_bwd so the grouped GEMMs can run whole 32-row blocks.
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kWarps = 8;  // warps per block = tokens per block
+
+// 16-byte vector <-> floats. BF16: 8 values per vector; FP32: 4.
+template <bool BF16>
+struct Vec;
+template <>
+struct Vec<true> {
+  static constexpr int N = 8;
+  __device__ static void unpack(const uint4& v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      f[2 * i] = bf16lo(w[i]);
+      f[2 * i + 1] = bf16hi(w[i]);
+    }
+  }
+  __device__ static uint4 pack(const float (&f)[8]) {
+    return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                      pack_bf16(f[6], f[7]));
+  }
+};
+template <>
+struct Vec<false> {
+  static constexpr int N = 4;
+  __device__ static void unpack(const uint4& v, float (&f)[4]) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
+  __device__ static uint4 pack(const float (&f)[4]) {
+    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                      __float_as_uint(f[3]));
+  }
+};
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Zero the pad rows [poff[e]+counts[e], poff[e+1]) of one expert; called by whole blocks.
+__device__ __forceinline__ void zero_pad_rows(uint4* buf, int e, const int32_t* counts,
+                                              const int32_t* poff, int vpr) {
+  const int r0 = poff[e] + counts[e], r1 = poff[e + 1];
+  const int64_t n = (int64_t)(r1 - r0) * vpr;
+  uint4* base = buf + (size_t)r0 * vpr;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) base[i] = make_uint4(0, 0, 0, 0);
+}
+
+__global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ prow, const int32_t* __restrict__ counts,
+    const int32_t* __restrict__ poff, uint4* __restrict__ xp, int T, int k, int vpr, int tok_blocks) {
+  if ((int)blockIdx.x >= tok_blocks) {
+    zero_pad_rows(xp, blockIdx.x - tok_blocks, counts, poff, vpr);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int myrow = lane < k ? prow[(size_t)t * k + lane] : 0;
+  int rows[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xffffffffu, myrow, j);
+  const uint4* src = x + (size_t)t * vpr;
+#pragma unroll 4
+  for (int v = lane; v < vpr; v += 32) {
+    const uint4 val = ldg_stream(src + v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < k) xp[(size_t)rows[j] * vpr + v] = val;
+  }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kWarps * 32) combine_kernel(const uint4* __restrict__ y,
+                                                              const float* __restrict__ gates,
+                                                              const int32_t* __restrict__ prow,
+                                                              uint4* __restrict__ out, int T, int k,
+                                                              int vpr) {
+  using V = Vec<BF16>;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int myrow = lane < k ? prow[(size_t)t * k + lane] : 0;
+  const float myg = lane < k ? gates[(size_t)t * k + lane] : 0.f;
+  int rows[8];
+  float g[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    rows[j] = __shfl_sync(0xffffffffu, myrow, j);
+    g[j] = __shfl_sync(0xffffffffu, myg, j);
+  }
+#pragma unroll 2
+  for (int v = lane; v < vpr; v += 32) {
+    float acc[V::N];
+#pragma unroll
+    for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j < k) {
+        float f[V::N];
+        V::unpack(ldg_stream(y + (size_t)rows[j] * vpr + v), f);
+#pragma unroll
+        for (int i = 0; i < V::N; ++i) acc[i] = fmaf(g[j], f[i], acc[i]);
+      }
+    }
+    out[(size_t)t * vpr + v] = V::pack(acc);
+  }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kWarps * 32) combine_bwd_kernel(
+    const uint4* __restrict__ dout, const uint4* __restrict__ y, const float* __restrict__ gates,
+    const int32_t* __restrict__ prow, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ counts, const int32_t* __restrict__ poff, uint4* __restrict__ dy,
+    float* __restrict__ dgates, float* __restrict__ dlsel, void* __restrict__ dlogits, int T, int k,
+    int E, int vpr, int tok_blocks) {
+  using V = Vec<BF16>;
+  if ((int)blockIdx.x >= tok_blocks) {
+    zero_pad_rows(dy, blockIdx.x - tok_blocks, counts, poff, vpr);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int myrow = lane < k ? prow[(size_t)t * k + lane] : 0;
+  const float myg = lane < k ? gates[(size_t)t * k + lane] : 0.f;
+  int rows[8];
+  float g[8], dot[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    rows[j] = __shfl_sync(0xffffffffu, myrow, j);
+    g[j] = __shfl_sync(0xffffffffu, myg, j);
+    dot[j] = 0.f;
+  }
+#pragma unroll 2
+  for (int v = lane; v < vpr; v += 32) {
+    float fd[V::N];
+    V::unpack(ldg_stream(dout + (size_t)t * vpr + v), fd);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j < k) {
+        float fy[V::N], o[V::N];
+        V::unpack(ldg_stream(y + (size_t)rows[j] * vpr + v), fy);
+#pragma unroll
+        for (int i = 0; i < V::N; ++i) {
+          dot[j] = fmaf(fd[i], fy[i], dot[j]);
+          o[i] = g[j] * fd[i];
+        }
+        dy[(size_t)rows[j] * vpr + v] = V::pack(o);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], off);
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < k) s = fmaf(g[j], dot[j], s);
+  float mydl = 0.f;
+  int mye = -1;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < k && lane == j) {
+      dgates[(size_t)t * k + j] = dot[j];
+      mydl = g[j] * (dot[j] - s);
+      if (dlsel) dlsel[(size_t)t * k + j] = mydl;
+      mye = idx ? idx[(size_t)t * k + j] : -1;
+    }
+  }
+  if (dlogits) {
+    // dense score-gradient row: zero except the k chosen experts
+    int ej[8];
+    float dj[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      ej[j] = __shfl_sync(0xffffffffu, mye, j);
+      dj[j] = __shfl_sync(0xffffffffu, mydl, j);
+    }
+    for (int e = lane; e < E; e += 32) {
+      float val = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < k && ej[j] == e) val = dj[j];
+      if (BF16)
+        reinterpret_cast<__nv_bfloat16*>(dlogits)[(size_t)t * E + e] = __float2bfloat16_rn(val);
+      else
+        reinterpret_cast<float*>(dlogits)[(size_t)t * E + e] = val;
+    }
+  }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kWarps * 32) token_reduce_kernel(
+    const uint4* __restrict__ dxp, const int32_t* __restrict__ prow, const float* __restrict__ dlsel,
+    const int32_t* __restrict__ idx, const uint4* __restrict__ Wr, uint4* __restrict__ dx, int T,
+    int k, int E, int vpr) {
+  using V = Vec<BF16>;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const bool router = dlsel && idx && Wr;
+  const int myrow = lane < k ? prow[(size_t)t * k + lane] : 0;
+  const float mydl = (router && lane < k) ? dlsel[(size_t)t * k + lane] : 0.f;
+  int mye = (router && lane < k) ? idx[(size_t)t * k + lane] : 0;
+  if (mye < 0 || mye >= E) mye = 0;
+  int rows[8], es[8];
+  float dl[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    rows[j] = __shfl_sync(0xffffffffu, myrow, j);
+    dl[j] = __shfl_sync(0xffffffffu, mydl, j);
+    es[j] = __shfl_sync(0xffffffffu, mye, j);
+  }
+#pragma unroll 2
+  for (int v = lane; v < vpr; v += 32) {
+    float acc[V::N];
+#pragma unroll
+    for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (j < k) {
+        float f[V::N];
+        V::unpack(ldg_stream(dxp + (size_t)rows[j] * vpr + v), f);
+#pragma unroll
+        for (int i = 0; i < V::N; ++i) acc[i] += f[i];
+        if (router) {
+          V::unpack(Wr[(size_t)es[j] * vpr + v], f);
+#pragma unroll
+          for (int i = 0; i < V::N; ++i) acc[i] = fmaf(dl[j], f[i], acc[i]);
+        }
+      }
+    }
+    dx[(size_t)t * vpr + v] = V::pack(acc);
+  }
+}
+
+}  // namespace
+
+int launch_dispatch(const void* x, const int32_t* prow, const int32_t* counts, const int32_t* poff,
+                    void* xp, int T, int k, int E, int row_bytes, cudaStream_t s) {
+  const int vpr = row_bytes / 16;
+  const int tok_blocks = (T + kWarps - 1) / kWarps;
+  dispatch_kernel<<<tok_blocks + E, kWarps * 32, 0, s>>>(
+      static_cast<const uint4*>(x), prow, counts, poff, static_cast<uint4*>(xp), T, k, vpr,
+      tok_blocks);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_combine(const void* y, const float* gates, const int32_t* prow, void* out, int T, int k,
+                   int row_bytes, bool bf16, cudaStream_t s) {
+  const int vpr = row_bytes / 16;
+  const int blocks = (T + kWarps - 1) / kWarps;
+  if (bf16)
+    combine_kernel<true><<<blocks, kWarps * 32, 0, s>>>(static_cast<const uint4*>(y), gates, prow,
+                                                        static_cast<uint4*>(out), T, k, vpr);
+  else
+    combine_kernel<false><<<blocks, kWarps * 32, 0, s>>>(static_cast<const uint4*>(y), gates, prow,
+                                                         static_cast<uint4*>(out), T, k, vpr);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_combine_bwd(const void* dout, const void* y, const float* gates, const int32_t* prow,
+                       const int32_t* idx, const int32_t* counts, const int32_t* poff, void* dy,
+                       float* dgates, float* dlsel, void* dlogits, int T, int k, int E, int row_bytes,
+                       bool bf16, cudaStream_t s) {
+  const int vpr = row_bytes / 16;
+  const int tok_blocks = (T + kWarps - 1) / kWarps;
+  if (bf16)
+    combine_bwd_kernel<true><<<tok_blocks + E, kWarps * 32, 0, s>>>(
+        static_cast<const uint4*>(dout), static_cast<const uint4*>(y), gates, prow, idx, counts,
+        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks);
+  else
+    combine_bwd_kernel<false><<<tok_blocks + E, kWarps * 32, 0, s>>>(
+        static_cast<const uint4*>(dout), static_cast<const uint4*>(y), gates, prow, idx, counts,
+        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_token_reduce(const void* dxp, const int32_t* prow, const float* dlsel, const int32_t* idx,
+                        const void* Wr, void* dx, int T, int k, int E, int row_bytes, bool bf16,
+                        cudaStream_t s) {
+  const int vpr = row_bytes / 16;
+  const int blocks = (T + kWarps - 1) / kWarps;
+  if (bf16)
+    token_reduce_kernel<true><<<blocks, kWarps * 32, 0, s>>>(
+        static_cast<const uint4*>(dxp), prow, dlsel, idx, static_cast<const uint4*>(Wr),
+        static_cast<uint4*>(dx), T, k, E, vpr);
+  else
+    token_reduce_kernel<false><<<blocks, kWarps * 32, 0, s>>>(
+        static_cast<const uint4*>(dxp), prow, dlsel, idx, static_cast<const uint4*>(Wr),
+        static_cast<uint4*>(dx), T, k, E, vpr);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

@@ -140,6 +140,32 @@ def combine(y: np.ndarray, gates: np.ndarray, meta: dict) -> np.ndarray:
     return out
 
 
+def combine_bwd(dout: np.ndarray, y: np.ndarray, gates: np.ndarray, meta: dict):
+    """Exact derivative of the combine: dy[prow[t*k+j]] = g[t,j] dout[t] (pad rows 0) and
+    dgates[t,j] = <dout[t], y[prow[t*k+j]]>."""
+    T, k = gates.shape
+    dy = np.zeros((y.shape[0],) + dout.shape[1:])
+    dgates = np.zeros((T, k))
+    for t in range(T):
+        for j in range(k):
+            r = meta["prow"][t * k + j]
+            dy[r] = gates[t, j] * dout[t]
+            dgates[t, j] = float(np.dot(dout[t], y[r]))
+    return dy, dgates
+
+
+def token_reduce(dx_perm: np.ndarray, meta: dict, T: int, k: int, dlogits=None, W_r=None):
+    """Gradient back to tokens: dx[t] = sum_j dx_perm[prow[t*k+j]] (+ dlogits[t] W_r, the router's
+    input gradient, when given)."""
+    dx = np.zeros((T,) + dx_perm.shape[1:])
+    for t in range(T):
+        for j in range(k):
+            dx[t] += dx_perm[meta["prow"][t * k + j]]
+    if dlogits is not None:
+        dx = dx + dlogits @ W_r
+    return dx
+
+
 # ----------------------------------------------------------------------------------------------
 # Expert MLP (SwiGLU)
 # ----------------------------------------------------------------------------------------------
@@ -177,15 +203,43 @@ def _mx_col(a):
     return mxfp8.fake_quant_cols(ap)[:n]
 
 
+def gemm_fwd1_swiglu(X, W13_e, qr=_ident):
+    """First expert GEMM and SwiGLU: h13 = X W13_e^T = [gate | up]; a = silu(gate) * up."""
+    F = W13_e.shape[0] // 2
+    h13 = qr(X) @ qr(W13_e).T
+    return h13, silu(h13[:, :F]) * h13[:, F:]
+
+
+def gemm_fwd2(A, W2_e, qr=_ident):
+    """Second expert GEMM: y = a W2_e^T."""
+    return qr(A) @ qr(W2_e).T
+
+
+def gemm_dgrad2_swiglu(dY, W2_e, h13, qr=_ident, qc=_ident):
+    """dA = dY W2_e (contraction over d), then the SwiGLU backward with the saved h13:
+    dgate = dA * up * silu'(gate), dup = dA * silu(gate); returns dH13 = [dgate | dup]."""
+    F = h13.shape[1] // 2
+    gate, up = h13[:, :F], h13[:, F:]
+    dA = qr(dY) @ qc(W2_e)
+    return np.concatenate([dA * up * silu_grad(gate), dA * silu(gate)], axis=1)
+
+
+def gemm_dgrad1(dH13, W13_e, qr=_ident, qc=_ident):
+    """dX = dH13 W13_e (contraction over 2F)."""
+    return qr(dH13) @ qc(W13_e)
+
+
+def gemm_wgrad(G, X, qc=_ident):
+    """Weight gradient over one expert's rows: G^T X (contraction over the rows)."""
+    return qc(G).T @ qc(X)
+
+
 def expert_fwd(X: np.ndarray, W13_e: np.ndarray, W2_e: np.ndarray, mx: bool = False):
     """One expert on its rows X [n,d]: h13 = X W13_e^T = [gate | up], a = silu(gate)*up, y = a W2_e^T.
     With `mx`, every GEMM operand is MXFP8-quantised along that GEMM's contraction axis first."""
     qr = _mx_row if mx else _ident
-    F = W13_e.shape[0] // 2
-    h13 = qr(X) @ qr(W13_e).T
-    a = silu(h13[:, :F]) * h13[:, F:]
-    y = qr(a) @ qr(W2_e).T
-    return h13, a, y
+    h13, a = gemm_fwd1_swiglu(X, W13_e, qr)
+    return h13, a, gemm_fwd2(a, W2_e, qr)
 
 
 def expert_bwd(X, W13_e, W2_e, h13, a, dY, mx: bool = False):
@@ -194,15 +248,10 @@ def expert_bwd(X, W13_e, W2_e, h13, a, dY, mx: bool = False):
     operand of a dgrad GEMM and for both operands of a wgrad GEMM)."""
     qr = _mx_row if mx else _ident
     qc = _mx_col if mx else _ident
-    F = W13_e.shape[0] // 2
-    gate, up = h13[:, :F], h13[:, F:]
-    dA = qr(dY) @ qc(W2_e)              # [n,F]   contraction over d
-    dW2 = qc(dY).T @ qc(a)              # [d,F]   contraction over the expert's rows
-    dgate = dA * up * silu_grad(gate)
-    dup = dA * silu(gate)
-    dH13 = np.concatenate([dgate, dup], axis=1)   # [n,2F]
-    dW13 = qc(dH13).T @ qc(X)           # [2F,d]  contraction over the expert's rows
-    dX = qr(dH13) @ qc(W13_e)           # [n,d]   contraction over 2F
+    dH13 = gemm_dgrad2_swiglu(dY, W2_e, h13, qr, qc)   # [n,2F]
+    dW2 = gemm_wgrad(dY, a, qc)                        # [d,F]
+    dW13 = gemm_wgrad(dH13, X, qc)                     # [2F,d]
+    dX = gemm_dgrad1(dH13, W13_e, qr, qc)              # [n,d]
     return dX, dW13, dW2, dH13
 
 
@@ -269,14 +318,7 @@ def layer_bwd(dout, x, W13, W2, idx, gates, saved, W_r=None, renorm=True, logits
     T, k = idx.shape
     E, F2, d = W13.shape
     rows = saved["x_perm"].shape[0]
-    y = saved["y"]
-    dy = np.zeros((rows, d))
-    dgates = np.zeros((T, k))
-    for t in range(T):
-        for j in range(k):
-            r = meta["prow"][t * k + j]
-            dy[r] = gates[t, j] * dout[t]
-            dgates[t, j] = float(np.dot(dout[t], y[r]))
+    dy, dgates = combine_bwd(dout, saved["y"], gates, meta)
     dW13 = np.zeros_like(W13, dtype=np.float64)
     dW2 = np.zeros_like(W2, dtype=np.float64)
     dxp = np.zeros((rows, d))
@@ -289,15 +331,11 @@ def layer_bwd(dout, x, W13, W2, idx, gates, saved, W_r=None, renorm=True, logits
         dX, dW13[e], dW2[e], dh13[sl] = expert_bwd(saved["x_perm"][sl], W13[e], W2[e],
                                                    saved["h13"][sl], saved["a"][sl], dy[sl], mx)
         dxp[sl] = dX
-    dx = np.zeros((T, d))
-    for t in range(T):
-        for j in range(k):
-            dx[t] += dxp[meta["prow"][t * k + j]]
     dlogits = dW_r = None
     if W_r is not None:
         dlogits = router_bwd(dgates, gates, idx, E, renorm, logits)
         dW_r = dlogits.T @ x
-        dx = dx + dlogits @ W_r
+    dx = token_reduce(dxp, meta, T, k, dlogits, W_r)
     return dict(dx=dx, dW13=dW13, dW2=dW2, dgates=dgates, dlogits=dlogits, dW_r=dW_r,
                 dy=dy, dh13=dh13, dx_perm=dxp)
 
