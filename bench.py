@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""MoE expert layer, forward + backward, tokens/s on B200 (one GPU per process; N independent replicas).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is the whole hot path over one batch: routing metadata, row-wise dispatch, grouped GEMM1 +
+SwiGLU, grouped GEMM2, combine, combine backward, GEMM2 dgrad + SwiGLU backward, GEMM2 wgrad, GEMM1
+dgrad, GEMM1 wgrad, token reduce (plus router scores / top-k / router backward for learned-router
+workloads). Inputs are resident in HBM when the timed region starts; the e2e figure repeats the
+measurement through the public layer API with host-resident inputs and outputs copied each step.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd+bwd tokens/s at E=128 top-4; grouped GEMM % tensor-core peak"
+DEFAULT_WORKLOAD = "e128_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "source": "fallback"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS)
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic work per op (bytes moved once, flops of the definition); R = routed rows = T*k
+# ------------------------------------------------------------------------------------------------
+
+def op_work(w, es=2):
+    T, d, F, E, k = w.T, w.d, w.F, w.E, w.k
+    R = T * k
+    Rp = R + 31 * E  # upper bound of padded rows written (pad rows are written as zeros)
+    ops = {}
+    if w.routing == "learned":
+        ops["router_logits"] = (T * d * es + E * d * es + T * E * 4, 2 * T * d * E)
+        ops["route_topk"] = (T * E * 4 + T * k * 8, 0)
+    ops["route_metadata"] = (T * k * 4 * 3 + Rp * 4, 0)
+    ops["dispatch"] = ((T + R) * d * es, 0)
+    ops["gemm_fwd1_swiglu"] = ((R * d + E * 2 * F * d + R * 2 * F + R * F) * es, 2 * R * d * 2 * F)
+    ops["gemm_fwd2"] = ((R * F + E * d * F + R * d) * es, 2 * R * F * d)
+    ops["combine"] = ((R * d + T * d) * es + T * k * 8, 0)
+    ops["combine_bwd"] = ((T * d + 2 * R * d) * es + T * k * 12, 0)
+    ops["gemm_dgrad2_swiglu"] = ((R * d + E * d * F + 2 * R * 2 * F) * es, 2 * R * d * F)
+    ops["gemm_wgrad2"] = ((R * d + R * F + E * d * F) * es, 2 * R * d * F)
+    ops["gemm_dgrad1"] = ((R * 2 * F + E * 2 * F * d + R * d) * es, 2 * R * 2 * F * d)
+    ops["gemm_wgrad1"] = ((R * 2 * F + R * d + E * 2 * F * d) * es, 2 * R * 2 * F * d)
+    ops["token_reduce"] = ((R * d + T * d) * es + (T * k * 8 if w.routing == "learned" else 0), 0)
+    if w.routing == "learned":
+        ops["router_wgrad"] = ((T * E + T * d + E * d) * es, 2 * T * E * d)
+    return ops
+
+
+class Step:
+    """The layer's kernels issued op by op through the C ABI (the same sequence moe_layer_fwd /
+    moe_layer_bwd enqueue), with CUDA events between ops for a per-kernel breakdown."""
+
+    def __init__(self, layer, w, inp):
+        import torch
+        from mixture_experts_layer_row_b200 import _lib as L
+        self.L, self.layer, self.w, self.inp = L, layer, w, inp
+        self.learned = w.routing == "learned"
+        lay = layer
+        if self.learned:
+            self.dlsel = torch.zeros((w.T, w.k), dtype=torch.float32, device=lay.device)
+            self.dlogits = torch.zeros((w.T, w.E), dtype=lay.act, device=lay.device)
+        else:
+            lay.idx.copy_(inp["idx"])
+            lay.gates.copy_(inp["gates"])
+        self.names = list(op_work(w).keys())
+        self.ev = None
+
+    def events(self, n_steps):
+        import torch
+        self.ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(self.names) + 1)]
+                   for _ in range(n_steps)]
+
+    def run(self, i=None):
+        L, lay, w, inp = self.L, self.layer, self.w, self.inp
+        ev = self.ev[i] if (i is not None and self.ev is not None) else None
+        c = lay.cfg
+        n = 0
+
+        def mark():
+            nonlocal n
+            if ev is not None:
+                ev[n].record()
+            n += 1
+
+        if self.learned:
+            mark(); L.router_logits(c, inp["x"], inp["W_r"], inp["bias"], lay.logits, lay.ws)
+            mark(); L.route_topk(c, lay.logits, None, lay.idx, lay.gates, lay.ws)
+        mark(); L.route_metadata(c, lay.idx, lay.counts, lay.offsets, lay.poff, lay.perm, lay.prow,
+                                 lay.row_token, lay.ws)
+        mark(); L.dispatch(c, inp["x"], lay.prow, lay.counts, lay.poff, lay.x_perm)
+        mark(); L.grouped_gemm(c, L.GEMM_FWD1_SWIGLU, lay.x_perm, inp["W13"], lay.h13, lay.a, None,
+                               lay.counts, lay.poff, lay.ws)
+        mark(); L.grouped_gemm(c, L.GEMM_FWD2, lay.a, inp["W2"], lay.y, None, None, lay.counts, lay.poff,
+                               lay.ws)
+        mark(); L.combine(c, lay.y, lay.gates, lay.prow, lay.out)
+        dls = self.dlsel if self.learned else None
+        dlg = self.dlogits if self.learned else None
+        mark(); L.combine_bwd(c, inp["dout"], lay.y, lay.gates, lay.prow, lay.idx, lay.counts, lay.poff,
+                              lay.dy, lay.dgates, dls, dlg)
+        mark(); L.grouped_gemm(c, L.GEMM_DGRAD2_SWIGLU, lay.dy, inp["W2"], lay.dh13, None, lay.h13,
+                               lay.counts, lay.poff, lay.ws)
+        mark(); L.grouped_gemm(c, L.GEMM_WGRAD2, lay.dy, lay.a, lay.dW2, None, None, lay.counts,
+                               lay.poff, lay.ws)
+        mark(); L.grouped_gemm(c, L.GEMM_DGRAD1, lay.dh13, inp["W13"], lay.dx_perm, None, None,
+                               lay.counts, lay.poff, lay.ws)
+        mark(); L.grouped_gemm(c, L.GEMM_WGRAD1, lay.dh13, lay.x_perm, lay.dW13, None, None,
+                               lay.counts, lay.poff, lay.ws)
+        mark(); L.token_reduce(c, lay.dx_perm, lay.prow, lay.dx, dls,
+                               lay.idx if self.learned else None, inp["W_r"] if self.learned else None)
+        if self.learned:
+            mark(); L.router_wgrad(c, self.dlogits, inp["x"], lay.dW_r, lay.ws)
+        mark()
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        reasons = set()
+        for r in rows:
+            for name, col in (("hw_slowdown", 5), ("hw_thermal_slowdown", 6),
+                              ("sw_thermal_slowdown", 7), ("sw_power_cap", 8)):
+                if r[col].lower().startswith("active"):
+                    reasons.add(name)
+        loaded = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+def cpu_baseline(w, inp, n_tokens, label):
+    """The fp64 oracle, as it stands, on the first n_tokens tokens of the workload (their routing,
+    the full expert weights), forward + backward; returns tokens/s and what was run."""
+    import numpy as np
+    import torch
+    from oracle import moe as O
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    x = f64(inp["x"][:n_tokens])
+    dout = f64(inp["dout"][:n_tokens])
+    W13, W2 = f64(inp["W13"]), f64(inp["W2"])
+    learned = w.routing == "learned"
+    Wr = f64(inp["W_r"]) if learned else None
+    bias = f64(inp["bias"]) if inp["bias"] is not None else None
+    if not learned:
+        idx = inp["idx"][:n_tokens].cpu().numpy().astype(np.int64)
+        gates = f64(inp["gates"][:n_tokens])
+    t0 = time.perf_counter()
+    if learned:
+        lg = O.router_logits(x, Wr, bias)
+        idx, gates = O.route(lg, w.k)
+    out, saved = O.layer_fwd(x, W13, W2, idx, gates)
+    O.layer_bwd(dout, x, W13, W2, idx, gates, saved, W_r=Wr)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{label}: first {n_tokens} tokens ({n_tokens * w.k} routed rows), full expert "
+                      f"weights, fp64 forward + backward, {dt:.1f} s"}
+
+
+def run_reference(args, w):
+    """The oracle timed as it stands on the host cores (rank 0 only), on bounded samples."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from moe_workloads import make_inputs
+    inp = make_inputs(w, seed=0, device="cpu")
+    ntok = args.ref_tokens
+    times = []
+    info = None
+    for i in range(args.warmup + args.steps):
+        info = cpu_baseline(w, inp, ntok, w.name)
+        if i >= args.warmup:
+            times.append(ntok / info["value"])
+    per = statistics.mean(times)
+    val = ntok / per
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w),
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": info["cores"],
+                             "kind": "oracle", "sample": info["sample"]},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {"workload": f"{w.name}: T={w.T} d={w.d} F={w.F} E={w.E} k={w.k} {w.dtype}, "
+                        f"{w.routing} routing" + (f", skew bias {w.skew}*ln(1/rank)" if w.skew else ""),
+            "T": w.T, "d_model": w.d, "ffn": w.F, "experts": w.E, "top_k": w.k,
+            "routing": w.routing, "seed": 0,
+            "l2": "no flush: every step streams inputs larger than the 126 MB L2 "
+                  "(expert weights alone are read twice and their gradients written once per step)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=512, help="oracle sample for cpu_baseline")
+    ap.add_argument("--ref-tokens", type=int, default=64, help="oracle sample per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    from moe_workloads import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if w.dtype not in ("bf16", "fp32"):
+        print(json.dumps({"error": f"workload {w.name} ({w.dtype}) is not built yet"}))
+        return 2
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    from moe_workloads import make_inputs
+    from mixture_experts_layer_row_b200 import MoELayer
+    from mixture_experts_layer_row_b200 import _lib as L
+
+    inp = make_inputs(w, seed=0, device="cuda")
+    learned = w.routing == "learned"
+    layer = MoELayer(w.T, w.d, w.F, w.E, w.k, dtype=w.dtype, learned_router=learned)
+    layer.set_weights(inp["W13"], inp["W2"], inp["W_r"] if learned else None)
+    step = Step(layer, w, inp)
+
+    # the op-by-op sequence computes exactly what the public layer API computes
+    step.run()
+    torch.cuda.synchronize()
+    ref = (layer.out.clone(), layer.dx.clone(), layer.dW13.clone(), layer.dW2.clone())
+    layer.forward(inp["x"], bias=inp["bias"], idx=inp["idx"], gates=inp["gates"])
+    layer.backward(inp["dout"])
+    torch.cuda.synchronize()
+    same = all(torch.equal(a, b) for a, b in zip(ref, (layer.out, layer.dx, layer.dW13, layer.dW2)))
+    assert same, "op-by-op sequence differs from moe_layer_fwd/bwd"
+    assert layer.error_flags() == 0, "device error flag set"
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step.run()
+    step.events(args.steps)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    n0 = L.launch_count()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(args.steps):
+        step.run(i)
+    t_end.record()
+    torch.cuda.synchronize()
+    launches = L.launch_count() - n0
+    clk = clocks.stop()
+    barrier()
+    ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_per_step = ms / args.steps
+    value = world * w.T / (ms_per_step / 1e3)
+
+    # per-op durations over the timed region
+    per_op = {n: 0.0 for n in step.names}
+    for i in range(args.steps):
+        ev = step.ev[i]
+        for j, n in enumerate(step.names):
+            per_op[n] += ev[j].elapsed_time(ev[j + 1])
+    per_op = {n: v / args.steps for n, v in per_op.items()}
+
+    peaks = load_peaks()
+    work = op_work(w, 4 if w.dtype == "fp32" else 2)
+    bw = peaks["hbm_gbs"]
+    tc = peaks["bf16_tflops"] * (0.5 if w.dtype == "fp32" else 1.0)  # tf32 dense = half of bf16
+    roof_time = 0.0
+    for n, (b, f) in work.items():
+        roof_time += max(b / (bw * 1e9), f / (tc * 1e12))
+    gemm_ops = [n for n in work if n.startswith("gemm_")]
+    gemm_flops = sum(work[n][1] for n in gemm_ops)
+    gemm_ms = sum(per_op[n] for n in gemm_ops)
+    dom = max(per_op, key=lambda n: per_op[n])
+    b, f = work[dom]
+    t_dom = per_op[dom] / 1e3
+    if b / (bw * 1e9) >= f / (tc * 1e12) or f == 0:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": b / t_dom / 1e9, "peak": bw, "unit": "GB/s",
+                "frac": (b / t_dom / 1e9) / bw, "traffic": None,
+                "algorithmic_bytes": b, "flops": f, "ms": per_op[dom],
+                "peak_source": f"{peaks['source']} hbm_gbs"}
+    else:
+        roof = {"kernel": dom, "bound": "tensor", "achieved": f / t_dom / 1e12, "peak": tc,
+                "unit": "TFLOP/s", "frac": (f / t_dom / 1e12) / tc, "traffic": None,
+                "algorithmic_bytes": b, "flops": f, "ms": per_op[dom],
+                "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
+
+    # end to end through the public layer API: host inputs in, host results out, every step
+    e2e = None
+    if not args.no_e2e:
+        hx = inp["x"].cpu().pin_memory()
+        hd = inp["dout"].cpu().pin_memory()
+        hi = inp["idx"].cpu().pin_memory() if not learned else None
+        hg = inp["gates"].cpu().pin_memory() if not learned else None
+        dx_in = torch.empty_like(inp["x"])
+        dd_in = torch.empty_like(inp["dout"])
+        di = torch.empty_like(inp["idx"]) if not learned else None
+        dgt = torch.empty_like(inp["gates"]) if not learned else None
+        ho = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+        hdx = torch.empty(layer.dx.shape, dtype=layer.dx.dtype).pin_memory()
+        h2d = hx.numel() * hx.element_size() + hd.numel() * hd.element_size()
+        if not learned:
+            h2d += hi.numel() * 4 + hg.numel() * 4
+        d2h = ho.numel() * ho.element_size() + hdx.numel() * hdx.element_size()
+
+        def e2e_step():
+            dx_in.copy_(hx, non_blocking=True)
+            dd_in.copy_(hd, non_blocking=True)
+            if not learned:
+                di.copy_(hi, non_blocking=True)
+                dgt.copy_(hg, non_blocking=True)
+            layer.forward(dx_in, bias=inp["bias"], idx=di, gates=dgt)
+            layer.backward(dd_in)
+            ho.copy_(layer.out, non_blocking=True)
+            hdx.copy_(layer.dx, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([ems], device="cuda")
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": world * w.T / (ems / args.steps / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": ems / args.steps, "api": "MoELayer.forward/backward -> moe_layer_fwd/bwd"}
+        assert torch.equal(ho.cuda(), ref[0]) and torch.equal(hdx.cuda(), ref[1])
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp, args.cpu_tokens, w.name)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded; shapes and distributions of the workload)",
+            "config": dict(workload_config(w), parallelism=f"replicas x{world}"),
+            "tflops": 18 * w.d * w.F * w.T * w.k * world / (ms_per_step / 1e3) / 1e12,
+            "grouped_gemm_tensor_frac": (gemm_flops / (gemm_ms / 1e3) / 1e12) / tc,
+            "layer_roofline": {"roofline_ms": roof_time * 1e3, "frac": roof_time * 1e3 / ms_per_step,
+                               "peaks": peaks},
+            "roofline": roof,
+            "per_op_ms": {n: round(v, 4) for n, v in per_op.items()},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -248,6 +248,10 @@ MOE_API int moe_test_bounded_wait(void* ws, uint64_t limit_ns, void* stream);
 /* Library version string (host). */
 MOE_API const char* moe_version(void);
 
+/* Number of kernels this library has enqueued in this process so far (host counter, diagnostics;
+ * benchmarks read it before and after a timed region). */
+MOE_API uint64_t moe_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

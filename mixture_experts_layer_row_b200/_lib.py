@@ -25,7 +25,7 @@ EXPORTS = [
     "moe_max_rows", "moe_workspace_size", "moe_get_error", "moe_clear_error", "moe_router_logits",
     "moe_route_topk", "moe_route_metadata", "moe_dispatch", "moe_combine", "moe_combine_bwd",
     "moe_token_reduce", "moe_grouped_gemm", "moe_router_wgrad", "moe_layer_fwd", "moe_layer_bwd",
-    "moe_test_bounded_wait", "moe_version",
+    "moe_test_bounded_wait", "moe_version", "moe_launch_count",
 ]
 
 
@@ -80,6 +80,7 @@ def _load():
                            ctypes.POINTER(Grads), vp, sz, vp], i),
         "moe_test_bounded_wait": ([vp, u64, vp], i),
         "moe_version": ([], ctypes.c_char_p),
+        "moe_launch_count": ([], ctypes.c_uint64),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -212,3 +213,8 @@ def layer_bwd(cfg, weights: Weights, saved: Saved, x, dout, dx, grads: Grads, ws
 
 def version() -> str:
     return lib.moe_version().decode()
+
+
+def launch_count() -> int:
+    """Kernels this library has enqueued in this process so far."""
+    return int(lib.moe_launch_count())

@@ -1,9 +1,15 @@
 // C ABI of the MoE expert layer library: argument validation, workspace layout, and the forward /
 // backward composition of the kernels. Every entry point validates on the host and enqueues nothing
 // on an error; all work is asynchronous on the caller's stream; nothing here allocates.
+#include <atomic>
 #include <cstring>
 
 #include "internal.h"
+
+namespace moe {
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace moe
 
 using namespace moe;
 
@@ -157,6 +163,8 @@ bool router_shape_ok(const moe_config_t* c) {
 extern "C" {
 
 const char* moe_version(void) { return "moe_b200 0.1 (sm_100a)"; }
+
+uint64_t moe_launch_count(void) { return moe::g_launches.load(std::memory_order_relaxed); }
 
 int64_t moe_max_rows(const moe_config_t* cfg) {
   if (check_cfg(cfg) != MOE_OK) return 0;

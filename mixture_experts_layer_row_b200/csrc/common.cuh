@@ -168,15 +168,20 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Shared-memory matrix descriptor for tcgen05 (128-byte swizzle, version 1 for sm_100).
-//   start: byte address in shared memory; lbo/sbo: leading / stride byte offsets.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t start, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor for tcgen05 (version 1 for sm_100).
+//   start: byte address in shared memory; lbo/sbo: leading / stride byte offsets;
+//   layout: 2 = 128-byte swizzle (16-byte chunks, 8-row atoms), 1 = 128-byte swizzle with 32-byte
+//   chunks and 4-row atoms (the layout MN-major 32-bit operands need).
+constexpr uint32_t kLayoutSW128 = 2;
+constexpr uint32_t kLayoutSW128Atom32 = 1;
+__device__ __forceinline__ uint64_t smem_desc(uint32_t start, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((start >> 4) & 0x3FFF);
   d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
   d |= (uint64_t)1 << 46;  // descriptor version for sm_100
-  d |= (uint64_t)2 << 61;  // layout: 128-byte swizzle
+  d |= (uint64_t)(layout & 7u) << 61;
   return d;
 }
 

@@ -45,6 +45,10 @@ struct Cfg {
   static constexpr int TMEM_COLS = 2 * BN;   // two accumulators
   static constexpr int BN_OUT = (EPI == EPI_SWIGLU_FWD) ? BN / 2 : BN;  // output columns per tile
   static constexpr uint32_t IDESC = instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, BM, BN);
+  // MN-major operands: 16-bit types use the plain 128B swizzle (8-row atoms of 1 KB); 32-bit (tf32)
+  // operands need the 128B swizzle with 32-byte chunks (4-row atoms of 512 B).
+  static constexpr uint32_t MN_LAYOUT = ES == 4 ? kLayoutSW128Atom32 : kLayoutSW128;
+  static constexpr uint32_t MN_SBO = ES == 4 ? 512 : 1024;
   static constexpr size_t SMEM_BYTES =
       1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + 1024 /*barriers etc*/ + 257 * 4;
 };
@@ -347,10 +351,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (MODE == GROUP_K) nk = min(C::CHUNKS, ti.nchunks - ks * C::CHUNKS) * (32 / C::UK);
           for (int kk = 0; kk < nk; ++kk) {
             uint64_t ad, bd;
-            if constexpr (A_MN) ad = smem_desc_sw128(a_addr + kk * C::UK * 128, C::BK * 128, 1024);
-            else ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-            if constexpr (B_MN) bd = smem_desc_sw128(b_addr + kk * C::UK * 128, C::BK * 128, 1024);
-            else bd = smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+            if constexpr (A_MN) ad = smem_desc(a_addr + kk * C::UK * 128, C::BK * 128, C::MN_SBO, C::MN_LAYOUT);
+            else ad = smem_desc(a_addr + kk * 32, 16, 1024, kLayoutSW128);
+            if constexpr (B_MN) bd = smem_desc(b_addr + kk * C::UK * 128, C::BK * 128, C::MN_SBO, C::MN_LAYOUT);
+            else bd = smem_desc(b_addr + kk * 32, 16, 1024, kLayoutSW128);
             umma<ES == 2 ? 0 : 1>(d_tmem, ad, bd, C::IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
             issued = true;
           }
@@ -506,9 +510,10 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 2-D row-major tensor [rows, cols] of `es`-byte elements, box [box_rows, box_cols], 128B swizzle.
+// 2-D row-major tensor [rows, cols] of `es`-byte elements, box [box_rows, box_cols], 128B swizzle
+// (with 32-byte swizzle atoms when `atom32`).
 bool make_tmap(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t cols, int64_t ld,
-               int box_cols, int box_rows) {
+               int box_cols, int box_rows, bool atom32 = false) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
@@ -517,7 +522,8 @@ bool make_tmap(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t co
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                         2, const_cast<void*>(ptr), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -548,13 +554,16 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   }
   CUtensorMap ta, tb;
   // A box: K-major -> [BM rows, EPR cols]; MN-major -> [32 rows, EPR cols]
-  if (!make_tmap(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, A_MN ? 32 : BM)) return MOE_ERR_CUDA;
+  if (!make_tmap(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, A_MN ? 32 : BM, A_MN && ES == 4))
+    return MOE_ERR_CUDA;
   int b_box_rows = B_MN ? 32 : (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN);
-  if (!make_tmap(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, b_box_rows)) return MOE_ERR_CUDA;
+  if (!make_tmap(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, b_box_rows, B_MN && ES == 4))
+    return MOE_ERR_CUDA;
   int grid = sm_count();
   if (grid_cap > 0 && grid_cap < grid) grid = grid_cap;
   if (grid < 1) grid = 1;
   kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, p);
+  count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -616,6 +625,7 @@ __global__ void bounded_wait_probe_kernel(uint32_t* err, uint64_t limit_ns) {
 
 int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s) {
   bounded_wait_probe_kernel<<<1, 32, 0, s>>>(err, limit_ns);
+  count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

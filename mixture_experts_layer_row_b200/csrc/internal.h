@@ -39,6 +39,9 @@ struct GemmParams {
   uint64_t wait_limit_ns;
 };
 
+// Host-side count of kernels enqueued (every launcher adds the kernels it launched).
+void count_launches(int n);
+
 int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
                 const GemmParams& p, cudaStream_t s);
 int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s);

@@ -267,6 +267,7 @@ int launch_dispatch(const void* x, const int32_t* prow, const int32_t* counts, c
   dispatch_kernel<<<tok_blocks + E, kWarps * 32, 0, s>>>(
       static_cast<const uint4*>(x), prow, counts, poff, static_cast<uint4*>(xp), T, k, vpr,
       tok_blocks);
+  count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -280,6 +281,7 @@ int launch_combine(const void* y, const float* gates, const int32_t* prow, void*
   else
     combine_kernel<false><<<blocks, kWarps * 32, 0, s>>>(static_cast<const uint4*>(y), gates, prow,
                                                          static_cast<uint4*>(out), T, k, vpr);
+  count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -297,6 +299,7 @@ int launch_combine_bwd(const void* dout, const void* y, const float* gates, cons
     combine_bwd_kernel<false><<<tok_blocks + E, kWarps * 32, 0, s>>>(
         static_cast<const uint4*>(dout), static_cast<const uint4*>(y), gates, prow, idx, counts,
         poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks);
+  count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -313,6 +316,7 @@ int launch_token_reduce(const void* dxp, const int32_t* prow, const float* dlsel
     token_reduce_kernel<false><<<blocks, kWarps * 32, 0, s>>>(
         static_cast<const uint4*>(dxp), prow, dlsel, idx, static_cast<const uint4*>(Wr),
         static_cast<uint4*>(dx), T, k, E, vpr);
+  count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -266,6 +266,7 @@ int launch_topk(const float* logits, const float* bias, int T, int E, int k, int
     default:
       return MOE_ERR_UNSUPPORTED;
   }
+  count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -282,6 +283,7 @@ int launch_metadata(const int32_t* idx, int T, int E, int k, int64_t max_rows, i
   scan_kernel<<<1, 256, 0, s>>>(hist_ws, nchunks, T, E, k, max_rows, counts, offsets, poff,
                                 row_token, err);
   rank_kernel<<<nchunks, kChunk, 0, s>>>(idx, T, E, k, hist_ws, offsets, poff, perm, prow, row_token);
+  count_launches(3);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
