@@ -271,8 +271,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-tokens", type=int, default=512, help="oracle sample for cpu_baseline")
-    ap.add_argument("--ref-tokens", type=int, default=64, help="oracle sample per reference step")
+    ap.add_argument("--cpu-tokens", type=int, default=8192, help="oracle sample for cpu_baseline (capped at T)")
+    ap.add_argument("--ref-tokens", type=int, default=256, help="oracle sample per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
@@ -431,7 +431,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, inp, args.cpu_tokens, w.name)
+        cpu = cpu_baseline(w, inp, min(args.cpu_tokens, w.T), w.name)
 
     if rank == 0:
         line = {
