@@ -126,6 +126,25 @@ MOE_API int moe_route_metadata(const moe_config_t* cfg, const int32_t* idx, int3
                        int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
                        int32_t* row_token, void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of moe_route_metadata (the pages have no counterpart; this is a service
+ * for callers). Some callers cannot allocate device memory: an engine plugin handed only its input and
+ * output tensors under a fixed memory plan, or a host runtime without a device allocator, cannot
+ * provide the workspace moe_route_metadata needs for its per-chunk histograms. This entry point takes
+ * the same inputs and outputs (same meaning, layout and results) and no workspace: its scratch is a
+ * static device array inside the library of 65536 int32 (256 KB), held on every GPU that loads the
+ * library until the process exits.
+ *   - Limit: ceil(T/256) * E <= 65536 (e.g. T = 131072 at E = 128); larger requests return
+ *     MOE_ERR_WORKSPACE and enqueue nothing.
+ *   - The first call on a device looks up the scratch's device address (cudaGetSymbolAddress, with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array: calls that overlap on the GPU (other streams, other
+ *     host threads) race and corrupt each other's results. Order them on one stream.
+ *   - Nothing in the scratch needs clearing (each call writes all it reads). Device-side routing
+ *     errors (expert ids outside [0,E)) are skipped but not reported: there is no error flag. */
+MOE_API int moe_route_metadata_noalloc(const moe_config_t* cfg, const int32_t* idx, int32_t* counts,
+                                       int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
+                                       int32_t* row_token, void* stream);
+
 /* ---- row-wise dispatch and combine --------------------------------------------------------------- */
 
 /* Row-wise dispatch (unite.ai, "Parallelismo, precisione e tecniche di memoria": each routed token is

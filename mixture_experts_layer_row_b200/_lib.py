@@ -25,7 +25,7 @@ EXPORTS = [
     "moe_max_rows", "moe_workspace_size", "moe_get_error", "moe_clear_error", "moe_router_logits",
     "moe_route_topk", "moe_route_metadata", "moe_dispatch", "moe_combine", "moe_combine_bwd",
     "moe_token_reduce", "moe_grouped_gemm", "moe_router_wgrad", "moe_layer_fwd", "moe_layer_bwd",
-    "moe_test_bounded_wait", "moe_version", "moe_launch_count",
+    "moe_test_bounded_wait", "moe_version", "moe_launch_count", "moe_route_metadata_noalloc",
 ]
 
 
@@ -81,6 +81,7 @@ def _load():
         "moe_test_bounded_wait": ([vp, u64, vp], i),
         "moe_version": ([], ctypes.c_char_p),
         "moe_launch_count": ([], ctypes.c_uint64),
+        "moe_route_metadata_noalloc": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp], i),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -156,6 +157,13 @@ def route_metadata(cfg, idx, counts, offsets, poff, perm, prow, row_token, ws, s
     check(lib.moe_route_metadata(ctypes.byref(cfg), ptr(idx), ptr(counts), ptr(offsets), ptr(poff),
                                  ptr(perm), ptr(prow), ptr(row_token), w, n, stream_handle(stream)),
           "moe_route_metadata")
+
+
+def route_metadata_noalloc(cfg, idx, counts, offsets, poff, perm, prow, row_token, stream=None):
+    """moe_route_metadata without a workspace (scratch in a static device array of the library)."""
+    check(lib.moe_route_metadata_noalloc(ctypes.byref(cfg), ptr(idx), ptr(counts), ptr(offsets),
+                                         ptr(poff), ptr(perm), ptr(prow), ptr(row_token),
+                                         stream_handle(stream)), "moe_route_metadata_noalloc")
 
 
 def dispatch(cfg, x, prow, counts, poff, x_perm, stream=None):
