@@ -84,7 +84,7 @@ GemmParams base_params(const moe_config_t* c, void* ws) {
 }
 
 int gemm_op(const moe_config_t* c, int op, const void* A, const void* B, void* Cout, void* C2,
-            const void* aux, const int32_t* counts, const int32_t* poff, void* ws, cudaStream_t s) {
+                 const void* aux, const int32_t* counts, const int32_t* poff, void* ws, cudaStream_t s) {
   const int es = es_of(c);
   const int64_t R = max_rows_of(c);
   const int d = c->d, F = c->F, E = c->E;

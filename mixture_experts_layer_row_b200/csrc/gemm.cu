@@ -31,6 +31,9 @@ constexpr int BM = 128;
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 
+constexpr int kSmemBudget = 232448;  // 227 KB of opt-in shared memory per CTA
+constexpr int kCtrlBytes = 2048;      // mbarriers, TMEM slot, abort word, tile prefix [<=257 ints]
+
 template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
 struct Cfg {
   static constexpr int EPR = 128 / ES;       // elements per 128-byte smem row
@@ -41,7 +44,14 @@ struct Cfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+  // output staging: each epilogue warp owns NBUF swizzled 32-row x 128-byte boxes
+  static constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : ES;  // output element size
+  static constexpr int OEPR = 128 / OES;     // output columns per staged box
+  static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3 : 2;
+  static constexpr int STAGING_BYTES = 4 * NBUF * 4096;
+  static constexpr int STAGES_FIT = (kSmemBudget - kCtrlBytes - 1024 - STAGING_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static_assert(STAGES >= 2, "pipeline too shallow");
   static constexpr int TMEM_COLS = 2 * BN;   // two accumulators
   static constexpr int BN_OUT = (EPI == EPI_SWIGLU_FWD) ? BN / 2 : BN;  // output columns per tile
   static constexpr uint32_t IDESC = instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, BM, BN);
@@ -50,7 +60,7 @@ struct Cfg {
   static constexpr uint32_t MN_LAYOUT = ES == 4 ? kLayoutSW128Atom32 : kLayoutSW128;
   static constexpr uint32_t MN_SBO = ES == 4 ? 512 : 1024;
   static constexpr size_t SMEM_BYTES =
-      1024 /*align slack*/ + (size_t)STAGES * STAGE_BYTES + 1024 /*barriers etc*/ + 257 * 4;
+      kCtrlBytes + 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + STAGING_BYTES;
 };
 
 struct TileInfo {
@@ -111,35 +121,39 @@ __device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const i
   }
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.f + expf(-g)); }
+// SwiGLU helpers with the fast exponential and division intrinsics (bf16 outputs need ~8 bits).
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.f + __expf(-g)); }
 
-// Store 32 consecutive fp32 values as bf16 (64 bytes) or fp32 (128 bytes).
-template <int ES>
-__device__ __forceinline__ void store32(void* dst, const float* v) {
-  if constexpr (ES == 2) {
-    uint4* d = reinterpret_cast<uint4*>(dst);
+// Write 32 fp32 values of this thread's row into a staged box (row `lane`, 128 bytes, 128B swizzle:
+// 16-byte chunk j of row r sits at chunk j ^ (r & 7)) as OES-byte elements, starting at chunk `ch0`.
+template <int OES>
+__device__ __forceinline__ void stage_row32(uint8_t* box, int lane, int ch0, const float* v) {
+  uint8_t* row = box + lane * 128;
+  if constexpr (OES == 2) {
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      d[q] = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                        pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+    for (int q = 0; q < 4; ++q) {
+      const uint4 w = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                                 pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+      st_shared_v4(row + (((ch0 + q) ^ (lane & 7)) << 4), w);
+    }
   } else {
-    uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-      d[q] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                        __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+    for (int q = 0; q < 8; ++q) {
+      const uint4 w = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                 __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+      st_shared_v4(row + (((ch0 + q) ^ (lane & 7)) << 4), w);
+    }
   }
 }
 
-template <int ES>
-__device__ __forceinline__ void store_masked(void* base, int col0, int ncols, const float* v) {
-  for (int c = 0; c < 32; ++c) {
-    if (col0 + c < ncols) {
-      if constexpr (ES == 2)
-        reinterpret_cast<__nv_bfloat16*>(base)[c] = __float2bfloat16_rn(v[c]);
-      else
-        reinterpret_cast<float*>(base)[c] = v[c];
-    }
+// Hand a fully written box to the TMA unit: every lane fences its writes, lane 0 stores the box.
+__device__ __forceinline__ void box_store(const CUtensorMap* map, const uint8_t* box, int lane, int c0,
+                                          int c1) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, box, c0, c1);
+    bulk_commit();
   }
 }
 
@@ -169,15 +183,18 @@ __device__ __forceinline__ void load32(const void* src, float* v) {
 template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmC,
+                        const __grid_constant__ CUtensorMap tmC2, const GemmParams p) {
   using C = Cfg<ES, A_MN, B_MN, BN, EPI, MODE>;
   static_assert(MODE == GROUP_M || (A_MN && B_MN), "wgrad mode needs MN-major operands");
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw);  // control area first
+  const uint32_t data_addr = smem_u32(smem_raw) + kCtrlBytes;
+  uint8_t* smem = smem_raw + kCtrlBytes + (((data_addr + 1023u) & ~1023u) - data_addr);
   uint8_t* smA = smem;
   uint8_t* smB = smem + (size_t)C::STAGES * C::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smB + (size_t)C::STAGES * C::B_BYTES);
+  uint8_t* stg = smB + (size_t)C::STAGES * C::B_BYTES;  // epilogue staging, 1 KB aligned
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* tfull = bars + 2 * C::STAGES;
@@ -246,6 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmC);
+    if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmC2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -372,8 +391,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ===================== epilogue (warps 2..5) =====================
+    // Each warp owns the 32 accumulator rows of its TMEM lane quadrant (one row per thread). It
+    // stages 32-row x 128-byte boxes in swizzled shared memory and stores them with TMA. A warp's
+    // slab of 32 rows is entirely inside or entirely outside its expert's 32-aligned group, so whole
+    // slabs are skipped instead of masking rows; columns past N are clipped by the tensor bounds.
     const int q = warp & 3;               // TMEM lane quadrant this warp may access
-    const int r = q * 32 + lane;          // accumulator row owned by this thread
+    uint8_t* wstg = stg + (size_t)q * C::NBUF * 4096;
+    int nb = 0;                           // next staging box (round robin)
     int local = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       TileInfo ti;
@@ -387,37 +411,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-      const bool row_ok = (ti.m0 + r) < ti.rows;
-      if constexpr (MODE == GROUP_K) {
-        // weight gradient of group e: C[e][m0 + r][n0 + c]
-        char* crow = reinterpret_cast<char*>(p.C) +
-                     ((size_t)ti.e * p.c_group_stride + (size_t)(ti.m0 + r) * p.ldc + ti.n0) * ES;
-        for (int c = 0; c < BN; c += 32) {
-          float v[32];
-          if (nst > 0) {
-            uint32_t raw[32];
-            tmem_ld_32x32b_x32(t_row + c, raw);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
-          }
-          if (row_ok) {
-            if (p.vec_ok && ti.n0 + c + 32 <= p.N) store32<ES>(crow + (size_t)c * ES, v);
-            else if (ti.n0 + c < p.N) store_masked<ES>(crow + (size_t)c * ES, ti.n0 + c, p.N, v);
-          }
-        }
-      } else {
-        const size_t grow = (size_t)ti.row_base + ti.m0 + r;  // row in the routed buffer
-        if constexpr (EPI == EPI_SWIGLU_FWD) {
-          char* hrow = reinterpret_cast<char*>(p.C) + grow * p.ldc * ES;
-          char* arow = reinterpret_cast<char*>(p.C2) + grow * p.ldc2 * ES;
-          for (int c = 0; c < BN / 2; c += 32) {
+      const bool active = (ti.m0 + q * 32) < ti.rows;       // warp-uniform
+      int c1;                                               // tensor row of this slab
+      if constexpr (MODE == GROUP_K) c1 = ti.e * p.M + ti.m0 + q * 32;
+      else c1 = ti.row_base + ti.m0 + q * 32;
+      if constexpr (EPI == EPI_SWIGLU_FWD) {
+        // accumulator columns [0, BN/2) gate, [BN/2, BN) up for output columns n0 + [0, BN/2)
+        for (int c = 0; c < BN / 2; c += C::OEPR) {
+          uint8_t* bg = wstg;
+          uint8_t* bu = wstg + 4096;
+          uint8_t* ba = wstg + 8192;
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
+#pragma unroll 1
+          for (int h = 0; h < C::OEPR; h += 32) {
             uint32_t rg[32], ru[32];
-            tmem_ld_32x32b_x32(t_row + c, rg);
-            tmem_ld_32x32b_x32(t_row + BN / 2 + c, ru);
+            tmem_ld_32x32b_x32(t_row + c + h, rg);
+            tmem_ld_32x32b_x32(t_row + BN / 2 + c + h, ru);
             tmem_ld_wait();
             float g[32], u[32], a[32];
 #pragma unroll
@@ -426,78 +436,120 @@ __global__ void __launch_bounds__(kThreads, 1)
               u[i] = __uint_as_float(ru[i]);
               a[i] = silu_f(g[i]) * u[i];
             }
-            if (row_ok) {
-              store32<ES>(hrow + (size_t)(ti.n0 + c) * ES, g);
-              store32<ES>(hrow + (size_t)(p.F + ti.n0 + c) * ES, u);
-              store32<ES>(arow + (size_t)(ti.n0 + c) * ES, a);
+            if (active) {
+              const int ch0 = (h * C::OES) >> 4;
+              stage_row32<C::OES>(bg, lane, ch0, g);
+              stage_row32<C::OES>(bu, lane, ch0, u);
+              stage_row32<C::OES>(ba, lane, ch0, a);
             }
           }
-        } else if constexpr (EPI == EPI_SWIGLU_BWD) {
-          const char* hrow = reinterpret_cast<const char*>(p.aux) + grow * p.ldaux * ES;
-          char* drow = reinterpret_cast<char*>(p.C) + grow * p.ldc * ES;
-          for (int c = 0; c < BN; c += 32) {
+          if (active) {
+            box_store(&tmC, bg, lane, ti.n0 + c, c1);
+            box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
+            box_store(&tmC2, ba, lane, ti.n0 + c, c1);
+          }
+        }
+      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+        const char* hrow = reinterpret_cast<const char*>(p.aux) +
+                           ((size_t)ti.row_base + ti.m0 + q * 32 + lane) * p.ldaux * ES;
+        for (int c = 0; c < BN; c += C::OEPR) {
+          uint8_t* bg = wstg;
+          uint8_t* bu = wstg + 4096;
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
+          const bool cols = active && (ti.n0 + c < p.N);
+#pragma unroll 1
+          for (int h = 0; h < C::OEPR; h += 32) {
             uint32_t rd[32];
-            tmem_ld_32x32b_x32(t_row + c, rd);
+            tmem_ld_32x32b_x32(t_row + c + h, rd);
             tmem_ld_wait();
-            if (row_ok && ti.n0 + c < p.N) {
+            if (cols) {
               float g[32], u[32], dg[32], du[32];
-              load32<ES>(hrow + (size_t)(ti.n0 + c) * ES, g);
-              load32<ES>(hrow + (size_t)(p.F + ti.n0 + c) * ES, u);
+              load32<ES>(hrow + (size_t)(ti.n0 + c + h) * ES, g);
+              load32<ES>(hrow + (size_t)(p.F + ti.n0 + c + h) * ES, u);
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const float da = __uint_as_float(rd[i]);
-                const float sg = 1.f / (1.f + expf(-g[i]));
+                const float sg = __fdividef(1.f, 1.f + __expf(-g[i]));
                 du[i] = da * g[i] * sg;
                 dg[i] = da * u[i] * sg * (1.f + g[i] * (1.f - sg));
               }
-              store32<ES>(drow + (size_t)(ti.n0 + c) * ES, dg);
-              store32<ES>(drow + (size_t)(p.F + ti.n0 + c) * ES, du);
+              const int ch0 = (h * C::OES) >> 4;
+              stage_row32<C::OES>(bg, lane, ch0, dg);
+              stage_row32<C::OES>(bu, lane, ch0, du);
             }
           }
-        } else {
-          // plain store (EPI_STORE: act dtype) or fp32 + bias (EPI_STORE_F32_BIAS)
-          constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : ES;
-          char* crow = reinterpret_cast<char*>(p.C) + (grow * p.ldc + ti.n0) * OES;
-          for (int c = 0; c < BN; c += 32) {
-            uint32_t raw[32];
-            tmem_ld_32x32b_x32(t_row + c, raw);
-            tmem_ld_wait();
+          if (cols) {
+            box_store(&tmC, bg, lane, ti.n0 + c, c1);
+            box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
+          }
+        }
+      } else {
+        // plain store (act dtype), fp32 + bias (router scores), or a weight gradient (GROUP_K)
+        for (int c = 0; c < BN; c += C::OEPR) {
+          uint8_t* bx = wstg + nb * 4096;
+          const bool cols = active && (ti.n0 + c < p.N);
+          if (cols) {
+            if (lane == 0) bulk_wait_read<C::NBUF - 1>();
+            __syncwarp();
+          }
+#pragma unroll 1
+          for (int h = 0; h < C::OEPR; h += 32) {
             float v[32];
+            if (nst > 0) {
+              uint32_t raw[32];
+              tmem_ld_32x32b_x32(t_row + c + h, raw);
+              tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+              for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            }
             if constexpr (EPI == EPI_STORE_F32_BIAS) {
-              if (p.bias)
-                for (int i = 0; i < 32; ++i)
-                  if (ti.n0 + c + i < p.N) v[i] += p.bias[ti.n0 + c + i];
+              if (p.bias) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  const int col = ti.n0 + c + h + i;
+                  if (col < p.N) v[i] += p.bias[col];
+                }
+              }
             }
-            if (row_ok) {
-              if (p.vec_ok && ti.n0 + c + 32 <= p.N) store32<OES>(crow + (size_t)c * OES, v);
-              else if (ti.n0 + c < p.N) store_masked<OES>(crow + (size_t)c * OES, ti.n0 + c, p.N, v);
-            }
+            if (cols) stage_row32<C::OES>(bx, lane, (h * C::OES) >> 4, v);
+          }
+          if (cols) {
+            box_store(&tmC, bx, lane, ti.n0 + c, c1);
+            nb = (nb + 1) % C::NBUF;
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
     }
+    if (lane == 0) bulk_wait_all();  // every staged box written out before the CTA ends
   }
 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
 }
 
 // ------------------------------------------------------------------------------------------------
 // host side: tensor maps and launch
 // ------------------------------------------------------------------------------------------------
 
+}  // namespace
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn get_encode_fn() {
+static EncodeTiledFn get_encode_fn() {
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void* ptr = nullptr;
@@ -510,22 +562,35 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 2-D row-major tensor [rows, cols] of `es`-byte elements, box [box_rows, box_cols], 128B swizzle
-// (with 32-byte swizzle atoms when `atom32`).
-bool make_tmap(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t cols, int64_t ld,
-               int box_cols, int box_rows, bool atom32 = false) {
+bool make_tmap_nd(CUtensorMap* m, const void* ptr, int es, int rank, const uint64_t* dims,
+                  const uint64_t* strides_bytes, const uint32_t* box, int swizzle) {
   EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
-  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
-  const cuuint32_t estr[2] = {1, 1};
+  if (!fn || rank < 1 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], es1[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    es1[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides_bytes[i];
+  const CUtensorMapSwizzle sw = swizzle == 2   ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle == 1 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                                               : CU_TENSOR_MAP_SWIZZLE_NONE;
   const CUresult r = fn(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                        2, const_cast<void*>(ptr), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        rank, const_cast<void*>(ptr), d, st, b, es1, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// 2-D row-major tensor [rows, cols] of `es`-byte elements, box [box_rows, box_cols]; swizzle as in
+// make_tmap_nd (2: 128B, 1: 128B with 32-byte atoms, 0: none).
+bool make_tmap(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t cols, int64_t ld,
+               int box_cols, int box_rows, int swizzle) {
+  const uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+  const uint64_t strides[1] = {(uint64_t)(ld * es)};
+  const uint32_t box[2] = {(uint32_t)box_cols, (uint32_t)box_rows};
+  return make_tmap_nd(m, ptr, es, 2, dims, strides, box, swizzle);
 }
 
 int sm_count() {
@@ -536,6 +601,8 @@ int sm_count() {
   if (!n[dev]) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
   return n[dev] > 0 ? n[dev] : 148;
 }
+
+namespace {
 
 template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
 int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p, int grid_cap,
@@ -554,15 +621,23 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   }
   CUtensorMap ta, tb;
   // A box: K-major -> [BM rows, EPR cols]; MN-major -> [32 rows, EPR cols]
-  if (!make_tmap(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, A_MN ? 32 : BM, A_MN && ES == 4))
+  if (!make_tmap(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, A_MN ? 32 : BM, (A_MN && ES == 4) ? 1 : 2))
     return MOE_ERR_CUDA;
   int b_box_rows = B_MN ? 32 : (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN);
-  if (!make_tmap(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, b_box_rows, B_MN && ES == 4))
+  if (!make_tmap(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, b_box_rows, (B_MN && ES == 4) ? 1 : 2))
+    return MOE_ERR_CUDA;
+  // outputs: 32-row x 128-byte boxes stored from the epilogue's swizzled staging
+  CUtensorMap tc, tc2;
+  const int64_t out_rows = (MODE == GROUP_K) ? (int64_t)(p.counts ? p.E : 1) * p.M : A.rows;
+  const int64_t out_cols = (EPI == EPI_SWIGLU_FWD || EPI == EPI_SWIGLU_BWD) ? 2 * (int64_t)p.F : p.N;
+  if (!make_tmap(&tc, p.C, C::OES, out_rows, out_cols, p.ldc, C::OEPR, 32, 2)) return MOE_ERR_CUDA;
+  tc2 = tc;
+  if (EPI == EPI_SWIGLU_FWD && !make_tmap(&tc2, p.C2, C::OES, out_rows, p.F, p.ldc2, C::OEPR, 32, 2))
     return MOE_ERR_CUDA;
   int grid = sm_count();
   if (grid_cap > 0 && grid_cap < grid) grid = grid_cap;
   if (grid < 1) grid = 1;
-  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, p);
+  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, tc, tc2, p);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

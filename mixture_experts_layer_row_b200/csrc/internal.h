@@ -42,6 +42,13 @@ struct GemmParams {
 // Host-side count of kernels enqueued (every launcher adds the kernels it launched).
 void count_launches(int n);
 
+// Host helpers for TMA descriptors (swizzle: 2 = 128B, 1 = 128B with 32-byte atoms, 0 = none).
+bool make_tmap_nd(CUtensorMap* m, const void* ptr, int es, int rank, const uint64_t* dims,
+                  const uint64_t* strides_bytes, const uint32_t* box, int swizzle);
+bool make_tmap(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t cols, int64_t ld,
+               int box_cols, int box_rows, int swizzle);
+int sm_count();
+
 int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
                 const GemmParams& p, cudaStream_t s);
 int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s);
