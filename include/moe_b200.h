@@ -208,6 +208,38 @@ MOE_API int moe_grouped_gemm(const moe_config_t* cfg, int op, const void* A, con
 MOE_API int moe_router_wgrad(const moe_config_t* cfg, const void* dlogits, const void* x, void* dW_r,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* ---- MXFP8 ----------------------------------------------------------------------------------------- */
+
+/* MXFP8 quantisation of a bf16 matrix src [rows, cols] (row-major), per the OCP Microscaling (MX) v1.0
+ * definitions (the pages only name the format: unite.ai, "Parallelismo, precisione e tecniche di
+ * memoria"): per block of 32 elements, scale byte e+127 with e = clamp(floor(log2 amax) - 8, -127,
+ * 127) (0 for an all-zero block) and E4M3 codes round-to-nearest-even(x / 2^e) saturated to +-448.
+ *   mode MOE_QUANT_ROW: blocks of 32 along a row; q [rows, cols], s [rows, cols/32]; cols % 32 == 0.
+ *   mode MOE_QUANT_COL: blocks of 32 down a column; q [rows, cols], s [cols, rows/32];
+ *                       rows % 32 == 0, cols % 8 == 0.
+ * src 16-byte aligned; q 16-byte (ROW) / 8-byte (COL) aligned. */
+#define MOE_QUANT_ROW 0
+#define MOE_QUANT_COL 1
+MOE_API int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode, uint8_t* q,
+                               uint8_t* s, void* stream);
+
+/* The grouped GEMM of moe_grouped_gemm with MXFP8 operands (tcgen05 kind::mxf8f6f4.block_scale, fp32
+ * accumulation, bf16 outputs). Each operand is E4M3 codes in the layout its bf16 counterpart has in
+ * moe_grouped_gemm plus UE8M0 scales along that GEMM's contraction axis:
+ *   FWD1_SWIGLU  A = x_perm  ROW [R32,d]          B = W13 ROW [E*2F,d]
+ *   FWD2         A = a       ROW [R32,F]          B = W2  ROW [E*d,F]
+ *   DGRAD2_SWIGLU A = dy     ROW [R32,d]          B = W2  COL [E*d,F] (scales [F, E*d/32])
+ *   DGRAD1       A = dh13    ROW [R32,2F]         B = W13 COL [E*2F,d] (scales [d, E*2F/32])
+ *   WGRAD2       A = dy      COL [R32,d]          B = a   COL [R32,F]
+ *   WGRAD1       A = dh13    COL [R32,2F]         B = x_perm COL [R32,d]
+ * where R32 = moe_max_rows(cfg) rounded up to 32 (rows past the last group are never read by the
+ * wgrads; COL scales of activations are [cols, R32/32]). aux (DGRAD2) is the bf16 h13. Requires
+ * cfg->dtype == MOE_DTYPE_MXFP8 and d % 128 == 0. */
+MOE_API int moe_grouped_gemm_mxfp8(const moe_config_t* cfg, int op, const uint8_t* Aq, const uint8_t* As,
+                                   const uint8_t* Bq, const uint8_t* Bs, void* C, void* C2,
+                                   const void* aux, const int32_t* counts, const int32_t* poff,
+                                   void* ws, size_t ws_bytes, void* stream);
+
 /* ---- whole layer ------------------------------------------------------------------------------------ */
 
 typedef struct {

@@ -26,6 +26,7 @@ EXPORTS = [
     "moe_route_topk", "moe_route_metadata", "moe_dispatch", "moe_combine", "moe_combine_bwd",
     "moe_token_reduce", "moe_grouped_gemm", "moe_router_wgrad", "moe_layer_fwd", "moe_layer_bwd",
     "moe_test_bounded_wait", "moe_version", "moe_launch_count", "moe_route_metadata_noalloc",
+    "moe_quantize_mxfp8", "moe_grouped_gemm_mxfp8",
 ]
 
 
@@ -82,6 +83,8 @@ def _load():
         "moe_version": ([], ctypes.c_char_p),
         "moe_launch_count": ([], ctypes.c_uint64),
         "moe_route_metadata_noalloc": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp], i),
+        "moe_quantize_mxfp8": ([vp, ctypes.c_int64, i, i, vp, vp, vp], i),
+        "moe_grouped_gemm_mxfp8": ([cfgp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -217,6 +220,23 @@ def layer_bwd(cfg, weights: Weights, saved: Saved, x, dout, dx, grads: Grads, ws
     check(lib.moe_layer_bwd(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(saved), ptr(x),
                             ptr(dout), ptr(dx), ctypes.byref(grads), w, n, stream_handle(stream)),
           "moe_layer_bwd")
+
+
+QUANT_ROW, QUANT_COL = 0, 1
+
+
+def quantize_mxfp8(src, q, s, mode, stream=None):
+    """MXFP8 quantisation of a bf16 matrix src [rows, cols] into codes q and scales s."""
+    rows, cols = src.shape
+    check(lib.moe_quantize_mxfp8(ptr(src), rows, cols, mode, ptr(q), ptr(s), stream_handle(stream)),
+          "moe_quantize_mxfp8")
+
+
+def grouped_gemm_mxfp8(cfg, op, Aq, As, Bq, Bs, C, C2, aux, counts, poff, ws, stream=None):
+    w, n = _ws(ws)
+    check(lib.moe_grouped_gemm_mxfp8(ctypes.byref(cfg), int(op), ptr(Aq), ptr(As), ptr(Bq), ptr(Bs),
+                                     ptr(C), ptr(C2), ptr(aux), ptr(counts), ptr(poff), w, n,
+                                     stream_handle(stream)), "moe_grouped_gemm_mxfp8")
 
 
 def version() -> str:

@@ -132,6 +132,64 @@ int gemm_op(const moe_config_t* c, int op, const void* A, const void* B, void* C
   }
 }
 
+int64_t r32_of(const moe_config_t* c) { return (max_rows_of(c) + 31) / 32 * 32; }
+
+int gemm_op_mx(const moe_config_t* c, int op, const uint8_t* Aq, const uint8_t* As, const uint8_t* Bq,
+               const uint8_t* Bs, void* Cout, void* C2, const void* aux, const int32_t* counts,
+               const int32_t* poff, void* ws, cudaStream_t s) {
+  const int64_t R = r32_of(c);
+  const int d = c->d, F = c->F, E = c->E;
+  GemmParams p = base_params(c, ws);
+  p.counts = counts;
+  p.poff = poff;
+  p.C = Cout;
+  p.sA = As;
+  p.sB = Bs;
+  GemmOperand a{Aq, 0, 0, 0}, b{Bq, 0, 0, 0};
+  switch (op) {
+    case MOE_GEMM_FWD1_SWIGLU:
+      MOE_REQUIRE(C2, MOE_ERR_INVALID_ARG);
+      a = {Aq, R, d, d};
+      b = {Bq, (int64_t)E * 2 * F, d, d};
+      p.K = d; p.N = F; p.b_rows_per_group = 2 * F; p.ldc = 2 * F; p.C2 = C2; p.ldc2 = F;
+      p.sA_ld = d / 32; p.a_mn_limit = R; p.sB_ld = d / 32; p.b_mn_limit = (int64_t)E * 2 * F;
+      return launch_gemm(GK_FWD1_SWIGLU, 1, 128, a, b, p, s);
+    case MOE_GEMM_FWD2:
+      a = {Aq, R, F, F};
+      b = {Bq, (int64_t)E * d, F, F};
+      p.K = F; p.N = d; p.b_rows_per_group = d; p.ldc = d;
+      p.sA_ld = F / 32; p.a_mn_limit = R; p.sB_ld = F / 32; p.b_mn_limit = (int64_t)E * d;
+      return launch_gemm(GK_FWD2, 1, 128, a, b, p, s);
+    case MOE_GEMM_DGRAD2_SWIGLU:
+      MOE_REQUIRE(aux && aligned16(aux), MOE_ERR_INVALID_ARG);
+      a = {Aq, R, d, d};
+      b = {Bq, (int64_t)E * d, F, F};
+      p.K = d; p.N = F; p.b_rows_per_group = d; p.aux = aux; p.ldaux = 2 * F; p.ldc = 2 * F;
+      p.sA_ld = d / 32; p.a_mn_limit = R; p.sB_ld = (int64_t)E * d / 32; p.b_mn_limit = F;
+      return launch_gemm(GK_DGRAD2_SWIGLU, 1, 128, a, b, p, s);
+    case MOE_GEMM_DGRAD1:
+      a = {Aq, R, 2 * F, 2 * F};
+      b = {Bq, (int64_t)E * 2 * F, d, d};
+      p.K = 2 * F; p.N = d; p.b_rows_per_group = 2 * F; p.ldc = d;
+      p.sA_ld = 2 * F / 32; p.a_mn_limit = R; p.sB_ld = (int64_t)E * 2 * F / 32; p.b_mn_limit = d;
+      return launch_gemm(GK_DGRAD1, 1, 128, a, b, p, s);
+    case MOE_GEMM_WGRAD2:
+      a = {Aq, R, d, d};
+      b = {Bq, R, F, F};
+      p.M = d; p.N = F; p.ldc = F; p.c_group_stride = (int64_t)d * F;
+      p.sA_ld = R / 32; p.a_mn_limit = d; p.sB_ld = R / 32; p.b_mn_limit = F;
+      return launch_gemm(GK_WGRAD, 1, 128, a, b, p, s);
+    case MOE_GEMM_WGRAD1:
+      a = {Aq, R, 2 * F, 2 * F};
+      b = {Bq, R, d, d};
+      p.M = 2 * F; p.N = d; p.ldc = d; p.c_group_stride = (int64_t)2 * F * d;
+      p.sA_ld = R / 32; p.a_mn_limit = 2 * F; p.sB_ld = R / 32; p.b_mn_limit = d;
+      return launch_gemm(GK_WGRAD, 1, 128, a, b, p, s);
+    default:
+      return MOE_ERR_INVALID_ARG;
+  }
+}
+
 int router_logits_impl(const moe_config_t* c, const void* x, const void* Wr, const float* bias,
                        float* logits, void* ws, cudaStream_t s) {
   GemmParams p = base_params(c, ws);
@@ -272,6 +330,35 @@ int moe_grouped_gemm(const moe_config_t* cfg, int op, const void* A, const void*
   MOE_REQUIRE(aligned16(A) && aligned16(B) && aligned16(C) && (!C2 || aligned16(C2)),
               MOE_ERR_INVALID_ARG);
   return gemm_op(cfg, op, A, B, C, C2, aux, counts, poff, ws, S(stream));
+}
+
+int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode, uint8_t* q, uint8_t* s,
+                       void* stream) {
+  MOE_REQUIRE(src && q && s && rows >= 1 && cols >= 1, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(src), MOE_ERR_INVALID_ARG);
+  if (mode == MOE_QUANT_ROW) {
+    MOE_REQUIRE(cols % 32 == 0 && aligned16(q), MOE_ERR_INVALID_ARG);
+  } else if (mode == MOE_QUANT_COL) {
+    MOE_REQUIRE(rows % 32 == 0 && cols % 8 == 0 && (reinterpret_cast<uintptr_t>(q) & 7u) == 0,
+                MOE_ERR_INVALID_ARG);
+  } else {
+    return MOE_ERR_INVALID_ARG;
+  }
+  return launch_quantize(src, rows, cols, mode, q, s, S(stream));
+}
+
+int moe_grouped_gemm_mxfp8(const moe_config_t* cfg, int op, const uint8_t* Aq, const uint8_t* As,
+                           const uint8_t* Bq, const uint8_t* Bs, void* C, void* C2, const void* aux,
+                           const int32_t* counts, const int32_t* poff, void* ws, size_t ws_bytes,
+                           void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(cfg->dtype == MOE_DTYPE_MXFP8, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(cfg->d % 128 == 0, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(Aq && As && Bq && Bs && C && counts && poff, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(Aq) && aligned16(Bq) && aligned16(C) && (!C2 || aligned16(C2)),
+              MOE_ERR_INVALID_ARG);
+  return gemm_op_mx(cfg, op, Aq, As, Bq, Bs, C, C2, aux, counts, poff, ws, S(stream));
 }
 
 int moe_router_wgrad(const moe_config_t* cfg, const void* dlogits, const void* x, void* dW_r, void* ws,

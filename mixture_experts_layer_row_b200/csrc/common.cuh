@@ -178,6 +178,33 @@ __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t b
   }
 }
 
+// MXFP8 block-scaled MMA: E4M3 A/B from shared memory, one UE8M0 scale per 32 K-elements per row
+// of A and of B read from TMEM (scale columns at sfa/sfb; the byte of each 32-bit column that holds
+// this MMA's K-block is selected by the instruction descriptor's scale-factor ids).
+__device__ __forceinline__ void umma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p; }" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy 32 rows x 16 bytes from shared memory (described by a no-swizzle K-major descriptor) into 32
+// TMEM lanes x 4 columns, replicated to all four 32-lane quadrants.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Instruction descriptor for kind::mxf8f6f4.block_scale: E4M3 x E4M3, UE8M0 scales, fp32 accumulate.
+__host__ __device__ constexpr uint32_t instr_desc_mx(bool a_mn, bool b_mn, int M, int N) {
+  return (0u << 7) | (0u << 10)  // A, B: E4M3
+         | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         (1u << 23)  // scale format: UE8M0
+         | ((uint32_t)(M >> 4) << 24);
+}
+
 // Make the mbarrier track completion of all tcgen05 operations this thread issued before.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(

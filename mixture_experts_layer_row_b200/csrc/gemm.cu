@@ -45,22 +45,31 @@ struct Cfg {
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   // output staging: each epilogue warp owns NBUF swizzled 32-row x 128-byte boxes
-  static constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : ES;  // output element size
+  static constexpr bool MX = (ES == 1);      // MXFP8 block-scaled (E4M3 operands, UE8M0 scales)
+  static constexpr int THREADS = MX ? kThreads + 32 : kThreads;  // + scale-loader warp
+  static constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : (MX ? 2 : ES);  // output element size
   static constexpr int OEPR = 128 / OES;     // output columns per staged box
   static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3 : 2;
   static constexpr int STAGING_BYTES = 4 * NBUF * 4096;
-  static constexpr int STAGES_FIT = (kSmemBudget - kCtrlBytes - 1024 - STAGING_BYTES) / STAGE_BYTES;
+  // MXFP8: per stage, one 512-byte scale chunk per 128 rows of A and of B (TMEM: 4 columns each)
+  static constexpr int SF_BYTES = MX ? 512 + (BN / 128) * 512 : 0;
+  static constexpr int SF_COLS = MX ? 4 + 4 * (BN / 128) : 0;
+  static constexpr int STAGES_FIT =
+      (kSmemBudget - kCtrlBytes - 1024 - STAGING_BYTES) / (STAGE_BYTES + SF_BYTES);
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static_assert(STAGES >= 2, "pipeline too shallow");
-  static constexpr int TMEM_COLS = 2 * BN;   // two accumulators
+  static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;  // two accumulators (+ scale columns)
+  static_assert(!MX || 2 * BN + STAGES * SF_COLS <= 512, "TMEM overflow");
   static constexpr int BN_OUT = (EPI == EPI_SWIGLU_FWD) ? BN / 2 : BN;  // output columns per tile
-  static constexpr uint32_t IDESC = instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, BM, BN);
+  static constexpr uint32_t IDESC =
+      MX ? instr_desc_mx(A_MN, B_MN, BM, BN) : instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, BM, BN);
   // MN-major operands: 16-bit types use the plain 128B swizzle (8-row atoms of 1 KB); 32-bit (tf32)
   // operands need the 128B swizzle with 32-byte chunks (4-row atoms of 512 B).
   static constexpr uint32_t MN_LAYOUT = ES == 4 ? kLayoutSW128Atom32 : kLayoutSW128;
   static constexpr uint32_t MN_SBO = ES == 4 ? 512 : 1024;
   static constexpr size_t SMEM_BYTES =
-      kCtrlBytes + 1024 /*alignment slack*/ + (size_t)STAGES * STAGE_BYTES + STAGING_BYTES;
+      kCtrlBytes + 1024 /*alignment slack*/ + (size_t)STAGES * (STAGE_BYTES + SF_BYTES) +
+      STAGING_BYTES;
 };
 
 struct TileInfo {
@@ -181,7 +190,7 @@ __device__ __forceinline__ void load32(const void* src, float* v) {
 }
 
 template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmC,
@@ -195,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smA = smem;
   uint8_t* smB = smem + (size_t)C::STAGES * C::A_BYTES;
   uint8_t* stg = smB + (size_t)C::STAGES * C::B_BYTES;  // epilogue staging, 1 KB aligned
+  uint8_t* sfs = stg + C::STAGING_BYTES;                  // MXFP8 scale chunks, per stage
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* tfull = bars + 2 * C::STAGES;
@@ -249,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], C::MX ? 2 : 1);  // TMA bytes (+ the scale loader's arrival)
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -368,13 +378,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = smem_u32(smB + (size_t)s * C::B_BYTES);
           int nk = C::KSTEPS;
           if constexpr (MODE == GROUP_K) nk = min(C::CHUNKS, ti.nchunks - ks * C::CHUNKS) * (32 / C::UK);
+          uint32_t sf_col = 0;
+          if constexpr (C::MX) {
+            // this stage's scales: smem chunks -> TMEM columns after the two accumulators
+            sf_col = tmem_base + 2 * BN + s * C::SF_COLS;
+            const uint32_t sf_smem = smem_u32(sfs + (size_t)s * C::SF_BYTES);
+#pragma unroll
+            for (int c = 0; c < 1 + BN / 128; ++c)
+              tmem_cp_32x128b_x4(sf_col + 4 * c, smem_desc(sf_smem + 512 * c, 16, 128, 0));
+          }
           for (int kk = 0; kk < nk; ++kk) {
             uint64_t ad, bd;
             if constexpr (A_MN) ad = smem_desc(a_addr + kk * C::UK * 128, C::BK * 128, C::MN_SBO, C::MN_LAYOUT);
             else ad = smem_desc(a_addr + kk * 32, 16, 1024, kLayoutSW128);
             if constexpr (B_MN) bd = smem_desc(b_addr + kk * C::UK * 128, C::BK * 128, C::MN_SBO, C::MN_LAYOUT);
             else bd = smem_desc(b_addr + kk * 32, 16, 1024, kLayoutSW128);
-            umma<ES == 2 ? 0 : 1>(d_tmem, ad, bd, C::IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
+            if constexpr (C::MX) {
+              const uint32_t id = C::IDESC | ((uint32_t)kk << 29) | ((uint32_t)kk << 4);
+              umma_mx(d_tmem, ad, bd, id, sf_col | ((uint32_t)kk << 30),
+                      (sf_col + 4) | ((uint32_t)kk << 30), (ks > 0 || kk > 0) ? 1u : 0u);
+            } else {
+              umma<ES == 2 ? 0 : 1>(d_tmem, ad, bd, C::IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
+            }
             issued = true;
           }
           umma_commit(&empty[s]);
@@ -389,7 +414,90 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_bounded(done, 0, p.wait_limit_ns, nullptr, p.err);
       }
     }
-  } else {
+  } else if (C::MX && warp == 6) {
+    // ===================== MXFP8 scale loader (warp 6) =====================
+    // For every stage, lane L assembles smem row L of each 512-byte scale chunk: the 4 K-block
+    // scales of rows L, L+32, L+64, L+96 (4 bytes each), the layout tcgen05.cp spreads over TMEM.
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      TileInfo ti;
+      tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
+      const int nst = num_kstages<C, MODE>(ti);
+      bool ok = true;
+      for (int ks = 0; ks < nst; ++ks, ++it) {
+        const int s = it % C::STAGES;
+        int w = 1;
+        if (lane == 0)
+          w = mbar_wait_bounded(&empty[s], ((it / C::STAGES) & 1) ^ 1, p.wait_limit_ns, abort_word,
+                                p.err);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          ok = false;
+          break;
+        }
+        int64_t kb0;   // first K-block of this stage (global K-block index of the scale arrays)
+        int nkb = 4;   // valid K-blocks in this stage
+        if constexpr (MODE == GROUP_M) {
+          kb0 = ks * 4;
+        } else {
+          kb0 = ti.kstart / 32 + ks * 4;
+          nkb = min(4, ti.nchunks - ks * 4);
+        }
+        uint8_t* sfa = sfs + (size_t)s * C::SF_BYTES;
+        // A: rows of the accumulator
+        {
+          uint32_t wv[4];
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const int r = lane + 32 * qq;
+            int64_t mn, kb = kb0;
+            if constexpr (MODE == GROUP_M) mn = (int64_t)ti.row_base + ti.m0 + r;
+            else mn = (int64_t)ti.m0 + r;
+            uint32_t v = 0;
+            if (mn < p.a_mn_limit) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                if (j < nkb) v |= (uint32_t)p.sA[mn * p.sA_ld + kb + j] << (8 * j);
+            }
+            wv[qq] = v;
+          }
+          st_shared_v4(sfa + lane * 16, make_uint4(wv[0], wv[1], wv[2], wv[3]));
+        }
+        // B: columns of the accumulator, 128 per chunk
+#pragma unroll
+        for (int c = 0; c < BN / 128; ++c) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const int n = 128 * c + lane + 32 * qq;
+            int64_t mn, kb = kb0;
+            if constexpr (MODE == GROUP_K) {
+              mn = (int64_t)ti.n0 + n;
+            } else if constexpr (B_MN) {
+              mn = (int64_t)ti.n0 + n;
+              kb = (int64_t)ti.e * (p.b_rows_per_group / 32) + kb0;
+            } else if constexpr (EPI == EPI_SWIGLU_FWD) {
+              mn = (int64_t)ti.e * p.b_rows_per_group + (n < BN / 2 ? ti.n0 + n : p.F + ti.n0 + n - BN / 2);
+            } else {
+              mn = (int64_t)ti.e * p.b_rows_per_group + ti.n0 + n;
+            }
+            uint32_t v = 0;
+            if (mn < p.b_mn_limit) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                if (j < nkb) v |= (uint32_t)p.sB[mn * p.sB_ld + kb + j] << (8 * j);
+            }
+            wv[qq] = v;
+          }
+          st_shared_v4(sfa + 512 * (1 + c) + lane * 16, make_uint4(wv[0], wv[1], wv[2], wv[3]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[s]);
+      }
+      if (!ok) break;
+    }
+  } else if (warp >= 2 && warp < 6) {
     // ===================== epilogue (warps 2..5) =====================
     // Each warp owns the 32 accumulator rows of its TMEM lane quadrant (one row per thread). It
     // stages 32-row x 128-byte boxes in swizzled shared memory and stores them with TMA. A warp's
@@ -451,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
         const char* hrow = reinterpret_cast<const char*>(p.aux) +
-                           ((size_t)ti.row_base + ti.m0 + q * 32 + lane) * p.ldaux * ES;
+                           ((size_t)ti.row_base + ti.m0 + q * 32 + lane) * p.ldaux * C::OES;
         for (int c = 0; c < BN; c += C::OEPR) {
           uint8_t* bg = wstg;
           uint8_t* bu = wstg + 4096;
@@ -465,8 +573,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_wait();
             if (cols) {
               float g[32], u[32], dg[32], du[32];
-              load32<ES>(hrow + (size_t)(ti.n0 + c + h) * ES, g);
-              load32<ES>(hrow + (size_t)(p.F + ti.n0 + c + h) * ES, u);
+              load32<C::OES>(hrow + (size_t)(ti.n0 + c + h) * C::OES, g);
+              load32<C::OES>(hrow + (size_t)(p.F + ti.n0 + c + h) * C::OES, u);
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const float da = __uint_as_float(rd[i]);
@@ -577,7 +685,10 @@ bool make_tmap_nd(CUtensorMap* m, const void* ptr, int es, int rank, const uint6
   const CUtensorMapSwizzle sw = swizzle == 2   ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : swizzle == 1 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
                                                : CU_TENSOR_MAP_SWIZZLE_NONE;
-  const CUresult r = fn(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+  const CUtensorMapDataType dt = es == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const CUresult r = fn(m, dt,
                         rank, const_cast<void*>(ptr), d, st, b, es1, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -637,7 +748,7 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   int grid = sm_count();
   if (grid_cap > 0 && grid_cap < grid) grid = grid_cap;
   if (grid < 1) grid = 1;
-  kern<<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, tc, tc2, p);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, tc, tc2, p);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -678,8 +789,17 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
   }
   if (es == 2) {
     MOE_GEMM_CASES(2)
-  } else {
+  } else if (es == 4) {
     MOE_GEMM_CASES(4)
+  } else if (es == 1) {  // MXFP8: BN = 128 (TMEM holds two accumulators plus per-stage scales)
+    switch (kind) {
+      case GK_FWD1_SWIGLU: return launch_impl<1, false, false, 128, EPI_SWIGLU_FWD, GROUP_M>(A, B, p, cap, s);
+      case GK_FWD2: return launch_impl<1, false, false, 128, EPI_STORE, GROUP_M>(A, B, p, cap, s);
+      case GK_DGRAD2_SWIGLU: return launch_impl<1, false, true, 128, EPI_SWIGLU_BWD, GROUP_M>(A, B, p, cap, s);
+      case GK_DGRAD1: return launch_impl<1, false, true, 128, EPI_STORE, GROUP_M>(A, B, p, cap, s);
+      case GK_WGRAD: return launch_impl<1, true, true, 128, EPI_STORE, GROUP_K>(A, B, p, cap, s);
+      default: return MOE_ERR_UNSUPPORTED;
+    }
   }
 #undef MOE_GEMM_CASES
   return MOE_ERR_UNSUPPORTED;

@@ -35,6 +35,11 @@ struct GemmParams {
   int F;
   int64_t c_group_stride;  // GROUP_K: elements between two groups' outputs
   int vec_ok;              // output rows allow 16-byte vector stores
+  // MXFP8 operands: UE8M0 scale of (MN index i, 32-element K-block b) at s[i * s_ld + b]
+  const uint8_t* sA;
+  const uint8_t* sB;
+  int64_t sA_ld, sB_ld;
+  int64_t a_mn_limit, b_mn_limit;  // valid MN indices of each operand's scales
   uint32_t* err;
   uint64_t wait_limit_ns;
 };
@@ -51,6 +56,8 @@ int sm_count();
 
 int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
                 const GemmParams& p, cudaStream_t s);
+int launch_quantize(const void* src, int64_t rows, int cols, int mode, uint8_t* q, uint8_t* s,
+                    cudaStream_t st);
 int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s);
 
 int launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm, int32_t* idx,

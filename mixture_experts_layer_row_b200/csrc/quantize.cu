@@ -1,0 +1,156 @@
+// MXFP8 quantisation: bf16 -> E4M3 codes + one UE8M0 scale per 32 elements along the contraction
+// axis of the GEMM that consumes the operand (MXFP8 is the reduced-precision format of unite.ai,
+// "Parallelismo, precisione e tecniche di memoria"; element and scale encodings per the OCP
+// Microscaling Formats v1.0 specification):
+//   block exponent e = floor(log2(amax)) - 8 (8 = E4M3's largest exponent), clamped to [-127, 127];
+//   scale byte = e + 127; code = round-to-nearest-even(x * 2^-e) saturated to +-448;
+//   an all-zero block gets scale byte 0 and zero codes.
+// floor(log2) is read from the fp32 exponent bits (exact, subnormals included); the scaling by a power
+// of two is exact in fp32, and the conversion is the hardware's cvt.rn.satfinite.e4m3x2.f32.
+//
+// Two layouts, both HBM-bound streaming kernels with 16-byte loads:
+//   ROW  blocks of 32 consecutive elements of a row: codes [rows, cols], scales [rows, cols/32]
+//   COL  blocks of 32 consecutive rows of a column:  codes [rows, cols], scales [cols, rows/32]
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+// floor(log2(a)) for a finite a > 0 given as fp32 bits.
+__device__ __forceinline__ int floor_log2_bits(uint32_t bits) {
+  const int ex = (int)((bits >> 23) & 0xFFu);
+  if (ex != 0) return ex - 127;
+  const uint32_t man = bits & 0x7FFFFFu;  // subnormal: man * 2^-149
+  return -149 + (31 - __clz(man));
+}
+
+// 2^k as an fp32 value for k in [-127, 127] (2^-127 is subnormal, still exact).
+__device__ __forceinline__ float exp2_exact(int k) {
+  return k >= -126 ? __int_as_float((k + 127) << 23) : __int_as_float(1 << (k + 149));
+}
+
+// Block exponent and scale byte for a block with maximum magnitude amax (>= 0).
+__device__ __forceinline__ int block_exponent(float amax, uint8_t* scale_byte) {
+  if (!(amax > 0.f)) {
+    *scale_byte = 0;
+    return 127;  // unused: all codes are zero
+  }
+  int e = floor_log2_bits(__float_as_uint(amax)) - 8;
+  e = e < -127 ? -127 : (e > 127 ? 127 : e);
+  *scale_byte = (uint8_t)(e + 127);
+  return e;
+}
+
+// Two floats -> two E4M3 codes (round to nearest even, saturate to finite), packed lo | hi << 8.
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__global__ void __launch_bounds__(256) quant_row_kernel(const uint4* __restrict__ src, int64_t nblocks,
+                                                        int blocks_per_row, uint4* __restrict__ q,
+                                                        uint8_t* __restrict__ s) {
+  const int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= nblocks) return;
+  uint4 w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = src[b * 4 + i];
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t u[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[8 * i + 2 * j] = bf16lo(u[j]);
+      v[8 * i + 2 * j + 1] = bf16hi(u[j]);
+    }
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  uint8_t sb;
+  const int e = block_exponent(amax, &sb);
+  const float inv = exp2_exact(-e);
+  uint32_t c[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t lo = cvt_e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv);
+    const uint32_t hi = cvt_e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv);
+    c[i] = amax > 0.f ? (lo | (hi << 16)) : 0u;
+  }
+  q[b * 2] = make_uint4(c[0], c[1], c[2], c[3]);
+  q[b * 2 + 1] = make_uint4(c[4], c[5], c[6], c[7]);
+  s[b] = sb;
+  (void)blocks_per_row;
+}
+
+// One thread per (32-row block, 8 consecutive columns).
+__global__ void __launch_bounds__(256) quant_col_kernel(const uint4* __restrict__ src, int64_t rows,
+                                                        int cols, uint2* __restrict__ q,
+                                                        uint8_t* __restrict__ s) {
+  const int groups = cols / 8;
+  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t rblocks = rows / 32;
+  if (t >= rblocks * groups) return;
+  const int64_t rb = t / groups;
+  const int cg = (int)(t % groups);
+  float amax[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) amax[j] = 0.f;
+  const uint4* base = src + (rb * 32) * groups + cg;  // row stride = groups uint4
+#pragma unroll 4
+  for (int r = 0; r < 32; ++r) {
+    const uint4 w = base[(int64_t)r * groups];
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      amax[2 * j] = fmaxf(amax[2 * j], fabsf(bf16lo(u[j])));
+      amax[2 * j + 1] = fmaxf(amax[2 * j + 1], fabsf(bf16hi(u[j])));
+    }
+  }
+  float inv[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint8_t sb;
+    const int e = block_exponent(amax[j], &sb);
+    inv[j] = amax[j] > 0.f ? exp2_exact(-e) : 0.f;
+    s[(int64_t)(cg * 8 + j) * rblocks + rb] = sb;
+  }
+  uint2* qb = q + (rb * 32) * groups + cg;
+#pragma unroll 4
+  for (int r = 0; r < 32; ++r) {
+    const uint4 w = base[(int64_t)r * groups];
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    uint32_t c[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t lo = cvt_e4m3x2(bf16lo(u[2 * h]) * inv[4 * h], bf16hi(u[2 * h]) * inv[4 * h + 1]);
+      const uint32_t hi =
+          cvt_e4m3x2(bf16lo(u[2 * h + 1]) * inv[4 * h + 2], bf16hi(u[2 * h + 1]) * inv[4 * h + 3]);
+      c[h] = lo | (hi << 16);
+    }
+    qb[(int64_t)r * groups] = make_uint2(c[0], c[1]);
+  }
+}
+
+}  // namespace
+
+int launch_quantize(const void* src, int64_t rows, int cols, int mode, uint8_t* q, uint8_t* s,
+                    cudaStream_t st) {
+  if (mode == 0) {
+    const int64_t nb = rows * (cols / 32);
+    const int64_t grid = (nb + 255) / 256;
+    quant_row_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const uint4*>(src), nb, cols / 32,
+                                                      reinterpret_cast<uint4*>(q), s);
+  } else {
+    const int64_t nt = (rows / 32) * (cols / 8);
+    const int64_t grid = (nt + 255) / 256;
+    quant_col_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const uint4*>(src), rows, cols,
+                                                      reinterpret_cast<uint2*>(q), s);
+  }
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace moe

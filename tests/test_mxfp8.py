@@ -1,0 +1,186 @@
+"""MXFP8 on the GPU: quantisation must be bit-exact with the oracle's OCP-MX quantiser (codes and
+scales), and every block-scaled grouped GEMM op must match the oracle's GEMM step applied to the
+oracle's own MXFP8 fake-quantised operands (exact products of E4M3 codes and power-of-two scales, so
+only fp32 accumulation order and the bf16 output rounding differ)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe as O
+from oracle import mxfp8 as MX
+from _util import assert_close_rel, dev, idx_from_counts, np64
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    from mixture_experts_layer_row_b200 import _lib as L
+    return L
+
+
+def _bf16_matrix(rows, cols, seed):
+    """Values spanning many binades per block, with all-zero blocks, tiny and huge magnitudes."""
+    g = torch.Generator().manual_seed(seed)
+    v = torch.randn((rows, cols), generator=g) * torch.exp2(torch.randint(-20, 20, (rows, 1), generator=g).float())
+    v[::7, :32] = 0.0                       # all-zero blocks
+    v[1::11, 32:64] *= 2.0 ** -110          # near the bottom of the scale range
+    v[2::13, :] = torch.round(v[2::13, :])  # exact small integers
+    return v.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("rows,cols", [(64, 32), (96, 256), (1024, 4096), (7, 96)])
+def test_quantize_row_bitexact(rows, cols):
+    L = _lib()
+    x = _bf16_matrix(rows, cols, rows + cols)
+    q = torch.zeros((rows, cols), dtype=torch.uint8, device=dev())
+    s = torch.zeros((rows, cols // 32), dtype=torch.uint8, device=dev())
+    L.quantize_mxfp8(x.to(dev()), q, s, L.QUANT_ROW)
+    torch.cuda.synchronize()
+    rq, rs = MX.quantize_rows(x.double().numpy())
+    assert np.array_equal(s.cpu().numpy(), rs)
+    assert np.array_equal(q.cpu().numpy(), rq)
+
+
+@pytest.mark.parametrize("rows,cols", [(32, 8), (256, 128), (2048, 1536)])
+def test_quantize_col_bitexact(rows, cols):
+    L = _lib()
+    x = _bf16_matrix(rows, cols, 3 * rows + cols)
+    q = torch.zeros((rows, cols), dtype=torch.uint8, device=dev())
+    s = torch.zeros((cols, rows // 32), dtype=torch.uint8, device=dev())
+    L.quantize_mxfp8(x.to(dev()), q, s, L.QUANT_COL)
+    torch.cuda.synchronize()
+    rq, rs = MX.quantize_cols(x.double().numpy())
+    assert np.array_equal(s.cpu().numpy(), rs.T)  # scales are stored [cols, rows/32]
+    assert np.array_equal(q.cpu().numpy(), rq)
+
+
+SHAPES = {
+    "ragged": (512, 128, 256, 8, 2, [0, 1, 31, 33, 129, 200, 300, 330]),
+    "one_expert": (300, 128, 128, 4, 1, [300, 0, 0, 0]),
+    "wide": (2048, 2048, 1024, 16, 4, None),
+}
+
+
+class MxProblem:
+    def __init__(self, shape, seed=0):
+        L = _lib()
+        self.L = L
+        T, d, F, E, k, counts = SHAPES[shape]
+        self.T, self.d, self.F, self.E, self.k = T, d, F, E, k
+        rng = np.random.default_rng(seed)
+        idx = np.argsort(rng.random((T, E)), 1)[:, :k] if counts is None else idx_from_counts(counts, T, k, rng)
+        self.meta = O.route_metadata(idx.astype(np.int64), E)
+        self.cfg = L.make_config(T, d, F, E, k, L.DTYPE_MXFP8)
+        self.R32 = (L.max_rows(self.cfg) + 31) // 32 * 32
+        self.ws = torch.zeros(L.workspace_size(self.cfg), dtype=torch.uint8, device=dev())
+        self.g = torch.Generator().manual_seed(seed + 1)
+        t32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev())
+        self.counts, self.poff = t32(self.meta["counts"]), t32(self.meta["poff"])
+        self.valid = self.meta["row_token"] >= 0
+
+    def rows(self, cols, scale=1.0):
+        used = int(self.meta["poff"][-1])
+        t = torch.zeros((self.R32, cols), dtype=torch.float32)
+        v = torch.randn((used, cols), generator=self.g) * scale
+        v[torch.from_numpy(~self.valid)] = 0
+        t[:used] = v
+        return t.to(torch.bfloat16)
+
+    def weights(self, *shape):
+        return (torch.randn(shape, generator=self.g) * 0.05).to(torch.bfloat16)
+
+    def quant(self, x2d, mode):
+        rows, cols = x2d.shape
+        q = torch.zeros((rows, cols), dtype=torch.uint8, device=dev())
+        s = torch.zeros((rows, cols // 32) if mode == 0 else (cols, rows // 32), dtype=torch.uint8,
+                        device=dev())
+        self.L.quantize_mxfp8(x2d.to(dev()).contiguous(), q, s, mode)
+        return q, s
+
+    def groups(self):
+        for e in range(self.E):
+            yield e, int(self.meta["poff"][e]), int(self.meta["counts"][e]), int(self.meta["poff"][e + 1])
+
+    def run(self, op, A, B, C, C2=None, aux=None):
+        d = lambda t: t.to(dev()) if t is not None else None
+        Cd, C2d = d(C), d(C2)
+        self.L.grouped_gemm_mxfp8(self.cfg, op, A[0], A[1], B[0], B[1], Cd, C2d, d(aux), self.counts,
+                                  self.poff, self.ws)
+        torch.cuda.synchronize()
+        assert self.L.get_error(self.ws) == 0
+        return Cd, C2d
+
+
+TOL = 1e-2
+ROWQ, COLQ = O._mx_row, O._mx_col
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_mx_fwd1(shape):
+    P = MxProblem(shape)
+    X, W13 = P.rows(P.d), P.weights(P.E, 2 * P.F, P.d)
+    h13, a = P.run(P.L.GEMM_FWD1_SWIGLU, P.quant(X, 0), P.quant(W13.reshape(-1, P.d), 0),
+                   torch.zeros((P.R32, 2 * P.F), dtype=torch.bfloat16),
+                   torch.zeros((P.R32, P.F), dtype=torch.bfloat16))
+    Xn, Wn, H, A = np64(X), np64(W13), np64(h13), np64(a)
+    for e, r0, n, r1 in P.groups():
+        if n:
+            rh, ra = O.gemm_fwd1_swiglu(Xn[r0:r0 + n], Wn[e], ROWQ)
+            assert_close_rel(H[r0:r0 + n], rh, TOL, f"h13 e{e}")
+            assert_close_rel(A[r0:r0 + n], ra, TOL, f"a e{e}")
+        assert np.all(H[r0 + n:r1] == 0) and np.all(A[r0 + n:r1] == 0)
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_mx_fwd2(shape):
+    P = MxProblem(shape)
+    A, W2 = P.rows(P.F), P.weights(P.E, P.d, P.F)
+    y, _ = P.run(P.L.GEMM_FWD2, P.quant(A, 0), P.quant(W2.reshape(-1, P.F), 0),
+                 torch.zeros((P.R32, P.d), dtype=torch.bfloat16))
+    An, Wn, Y = np64(A), np64(W2), np64(y)
+    for e, r0, n, r1 in P.groups():
+        if n:
+            assert_close_rel(Y[r0:r0 + n], O.gemm_fwd2(An[r0:r0 + n], Wn[e], ROWQ), TOL, f"y e{e}")
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_mx_dgrad2(shape):
+    P = MxProblem(shape)
+    dY, W2, H13 = P.rows(P.d), P.weights(P.E, P.d, P.F), P.rows(2 * P.F, 2.0)
+    dh, _ = P.run(P.L.GEMM_DGRAD2_SWIGLU, P.quant(dY, 0), P.quant(W2.reshape(-1, P.F), 1),
+                  torch.zeros((P.R32, 2 * P.F), dtype=torch.bfloat16), aux=H13)
+    dYn, Wn, Hn, D = np64(dY), np64(W2), np64(H13), np64(dh)
+    for e, r0, n, r1 in P.groups():
+        if n:
+            ref = O.gemm_dgrad2_swiglu(dYn[r0:r0 + n], Wn[e], Hn[r0:r0 + n], ROWQ, COLQ)
+            assert_close_rel(D[r0:r0 + n], ref, TOL, f"dh13 e{e}")
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_mx_dgrad1(shape):
+    P = MxProblem(shape)
+    dH, W13 = P.rows(2 * P.F), P.weights(P.E, 2 * P.F, P.d)
+    dx, _ = P.run(P.L.GEMM_DGRAD1, P.quant(dH, 0), P.quant(W13.reshape(-1, P.d), 1),
+                  torch.zeros((P.R32, P.d), dtype=torch.bfloat16))
+    dHn, Wn, DX = np64(dH), np64(W13), np64(dx)
+    for e, r0, n, r1 in P.groups():
+        if n:
+            assert_close_rel(DX[r0:r0 + n], O.gemm_dgrad1(dHn[r0:r0 + n], Wn[e], ROWQ, COLQ), TOL,
+                             f"dx e{e}")
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+@pytest.mark.parametrize("which", ["w2", "w13"])
+def test_mx_wgrad(shape, which):
+    P = MxProblem(shape)
+    if which == "w2":
+        G, X, M, N, op = P.rows(P.d), P.rows(P.F), P.d, P.F, P.L.GEMM_WGRAD2
+    else:
+        G, X, M, N, op = P.rows(2 * P.F), P.rows(P.d), 2 * P.F, P.d, P.L.GEMM_WGRAD1
+    dW, _ = P.run(op, P.quant(G, 1), P.quant(X, 1), torch.full((P.E, M, N), 5.0, dtype=torch.bfloat16))
+    Gn, Xn, DW = np64(G), np64(X), np64(dW)
+    for e, r0, n, r1 in P.groups():
+        if n == 0:
+            assert np.all(DW[e] == 0)
+        else:
+            assert_close_rel(DW[e], O.gemm_wgrad(Gn[r0:r0 + n], Xn[r0:r0 + n], COLQ), TOL, f"dW e{e}")
