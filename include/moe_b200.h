@@ -27,8 +27,9 @@
  *     (rows 0..F-1 gate W1, rows F..2F-1 up W3), W2 [E,d,F].
  *   - "act" dtype is fp32 when cfg->dtype == MOE_DTYPE_FP32 and bf16 otherwise. Router scores,
  *     gates and gate gradients are always fp32; index arrays are int32.
- *   - Routed-row buffers have moe_max_rows(cfg) = T*k + 31*E rows: each expert's group starts on a
- *     32-row boundary (poff) and its pad rows are kept at zero by the kernels that write the buffer.
+ *   - Routed-row buffers have moe_max_rows(cfg) = T*k + 31*E rows rounded up to a multiple of 32: each
+ *     expert's group starts on a 32-row boundary (poff) and its pad rows are kept at zero by the
+ *     kernels that write the buffer.
  *   - Every function returns MOE_OK (0) or a negative MOE_ERR_* code. Arguments are validated on the
  *     host before anything is enqueued; on an error nothing is enqueued.
  *   - Device-side problems (an expert id outside [0,E), counts that do not add up to T*k, a
@@ -83,7 +84,7 @@ typedef struct {
   int renorm; /* 1: gates renormalised over the chosen k (required by the backward pass) */
 } moe_config_t;
 
-/* Rows of every routed-row buffer: T*k + 31*E. Returns 0 for an invalid config. */
+/* Rows of every routed-row buffer: T*k + 31*E rounded up to 32. Returns 0 for an invalid config. */
 MOE_API int64_t moe_max_rows(const moe_config_t* cfg);
 
 /* Bytes of scratch the layer-level calls need (routing histograms, router-gradient scratch and the
@@ -232,7 +233,7 @@ MOE_API int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode
  *   DGRAD1       A = dh13    ROW [R32,2F]         B = W13 COL [E*2F,d] (scales [d, E*2F/32])
  *   WGRAD2       A = dy      COL [R32,d]          B = a   COL [R32,F]
  *   WGRAD1       A = dh13    COL [R32,2F]         B = x_perm COL [R32,d]
- * where R32 = moe_max_rows(cfg) rounded up to 32 (rows past the last group are never read by the
+ * where R32 = moe_max_rows(cfg) (a multiple of 32; rows past the last group are never read by the
  * wgrads; COL scales of activations are [cols, R32/32]). aux (DGRAD2) is the bf16 h13. Requires
  * cfg->dtype == MOE_DTYPE_MXFP8 and d % 128 == 0. */
 MOE_API int moe_grouped_gemm_mxfp8(const moe_config_t* cfg, int op, const uint8_t* Aq, const uint8_t* As,
@@ -288,6 +289,47 @@ MOE_API int moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* w, const
 MOE_API int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_saved_t* saved,
                   const void* x, const void* dout, void* dx, moe_grads_t* g, void* ws,
                   size_t ws_bytes, void* stream);
+
+/* ---- whole layer, MXFP8 ---------------------------------------------------------------------------------- */
+
+/* Quantised copies of the expert weights (caller-owned; refresh after every weight update):
+ *   W13q/W13s  ROW along d  [E*2F, d] / [E*2F, d/32]      (forward GEMM1)
+ *   W13tq/W13ts COL along 2F [E*2F, d] / [d, E*2F/32]     (GEMM1 dgrad)
+ *   W2q/W2s    ROW along F  [E*d, F] / [E*d, F/32]        (forward GEMM2)
+ *   W2tq/W2ts  COL along d  [E*d, F] / [F, E*d/32]        (GEMM2 dgrad) */
+typedef struct {
+  uint8_t *W13q, *W13s, *W13tq, *W13ts;
+  uint8_t *W2q, *W2s, *W2tq, *W2ts;
+} moe_mxfp8_weights_t;
+
+/* Quantised routed activations (caller-owned scratch), R32 = moe_max_rows(cfg):
+ *   x*: x_perm [R32, d]   a*: a [R32, F]   dy*: dy [R32, d]   dh*: dh13 [R32, 2F]
+ *   ?q/?s ROW (scales [R32, cols/32]);  ?tq/?ts COL (scales [cols, R32/32]). */
+typedef struct {
+  uint8_t *xq, *xs, *xtq, *xts;
+  uint8_t *aq, *as, *atq, *ats;
+  uint8_t *dyq, *dys, *dytq, *dyts;
+  uint8_t *dhq, *dhs, *dhtq, *dhts;
+} moe_mxfp8_acts_t;
+
+/* Fill every buffer of qw from the bf16 weights (4 quantisation launches). */
+MOE_API int moe_quantize_weights_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
+                                       const moe_mxfp8_weights_t* qw, void* stream);
+
+/* moe_layer_fwd with MXFP8 expert GEMMs (cfg->dtype == MOE_DTYPE_MXFP8, bf16 storage): the routed
+ * activations are quantised along each GEMM's contraction axis right before it; SwiGLU, combine and
+ * all stored activations stay bf16. A learned router runs in bf16. */
+MOE_API int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
+                                const moe_mxfp8_weights_t* qw, const void* x, const float* bias,
+                                void* out, moe_saved_t* saved, const moe_mxfp8_acts_t* qa, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/* moe_layer_bwd with MXFP8 expert GEMMs (dgrad operands ROW/COL as listed above, wgrad operands COL
+ * along the expert's rows, in 32-row blocks of its zero-padded group). */
+MOE_API int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
+                                const moe_mxfp8_weights_t* qw, const moe_saved_t* saved,
+                                const moe_mxfp8_acts_t* qa, const void* x, const void* dout, void* dx,
+                                moe_grads_t* g, void* ws, size_t ws_bytes, void* stream);
 
 /* ---- test support ------------------------------------------------------------------------------------- */
 

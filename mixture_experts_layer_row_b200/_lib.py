@@ -26,7 +26,8 @@ EXPORTS = [
     "moe_route_topk", "moe_route_metadata", "moe_dispatch", "moe_combine", "moe_combine_bwd",
     "moe_token_reduce", "moe_grouped_gemm", "moe_router_wgrad", "moe_layer_fwd", "moe_layer_bwd",
     "moe_test_bounded_wait", "moe_version", "moe_launch_count", "moe_route_metadata_noalloc",
-    "moe_quantize_mxfp8", "moe_grouped_gemm_mxfp8",
+    "moe_quantize_mxfp8", "moe_grouped_gemm_mxfp8", "moe_quantize_weights_mxfp8",
+    "moe_layer_fwd_mxfp8", "moe_layer_bwd_mxfp8",
 ]
 
 
@@ -52,6 +53,17 @@ class Saved(ctypes.Structure):
 class Grads(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("dW_r", "dW13", "dW2", "dgates", "dy", "dh13", "dx_perm")]
+
+
+class MxWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("W13q", "W13s", "W13tq", "W13ts", "W2q", "W2s", "W2tq", "W2ts")]
+
+
+class MxActs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("xq", "xs", "xtq", "xts", "aq", "as_", "atq", "ats", "dyq", "dys", "dytq", "dyts",
+                 "dhq", "dhs", "dhtq", "dhts")]
 
 
 def _load():
@@ -85,6 +97,12 @@ def _load():
         "moe_route_metadata_noalloc": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp], i),
         "moe_quantize_mxfp8": ([vp, ctypes.c_int64, i, i, vp, vp, vp], i),
         "moe_grouped_gemm_mxfp8": ([cfgp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i),
+        "moe_quantize_weights_mxfp8": ([cfgp, ctypes.POINTER(Weights), ctypes.POINTER(MxWeights), vp], i),
+        "moe_layer_fwd_mxfp8": ([cfgp, ctypes.POINTER(Weights), ctypes.POINTER(MxWeights), vp, vp, vp,
+                                 ctypes.POINTER(Saved), ctypes.POINTER(MxActs), vp, sz, vp], i),
+        "moe_layer_bwd_mxfp8": ([cfgp, ctypes.POINTER(Weights), ctypes.POINTER(MxWeights),
+                                 ctypes.POINTER(Saved), ctypes.POINTER(MxActs), vp, vp, vp,
+                                 ctypes.POINTER(Grads), vp, sz, vp], i),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -237,6 +255,26 @@ def grouped_gemm_mxfp8(cfg, op, Aq, As, Bq, Bs, C, C2, aux, counts, poff, ws, st
     check(lib.moe_grouped_gemm_mxfp8(ctypes.byref(cfg), int(op), ptr(Aq), ptr(As), ptr(Bq), ptr(Bs),
                                      ptr(C), ptr(C2), ptr(aux), ptr(counts), ptr(poff), w, n,
                                      stream_handle(stream)), "moe_grouped_gemm_mxfp8")
+
+
+def quantize_weights_mxfp8(cfg, weights: Weights, qw: MxWeights, stream=None):
+    check(lib.moe_quantize_weights_mxfp8(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(qw),
+                                         stream_handle(stream)), "moe_quantize_weights_mxfp8")
+
+
+def layer_fwd_mxfp8(cfg, weights, qw, x, bias, out, saved, qa, ws, stream=None):
+    w, n = _ws(ws)
+    check(lib.moe_layer_fwd_mxfp8(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(qw), ptr(x),
+                                  ptr(bias), ptr(out), ctypes.byref(saved), ctypes.byref(qa), w, n,
+                                  stream_handle(stream)), "moe_layer_fwd_mxfp8")
+
+
+def layer_bwd_mxfp8(cfg, weights, qw, saved, qa, x, dout, dx, grads, ws, stream=None):
+    w, n = _ws(ws)
+    check(lib.moe_layer_bwd_mxfp8(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(qw),
+                                  ctypes.byref(saved), ctypes.byref(qa), ptr(x), ptr(dout), ptr(dx),
+                                  ctypes.byref(grads), w, n, stream_handle(stream)),
+          "moe_layer_bwd_mxfp8")
 
 
 def version() -> str:

@@ -30,13 +30,15 @@ int check_cfg(const moe_config_t* c) {
   if (c->k > c->E) return MOE_ERR_INVALID_ARG;
   if (c->E > 256 || c->k > 8) return MOE_ERR_UNSUPPORTED;
   if (c->d % 64 != 0 || c->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
-  const int64_t rows = (int64_t)c->T * c->k + 31ll * c->E;
+  const int64_t rows = (int64_t)c->T * c->k + 31ll * c->E + 31;
   if (rows >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
 inline int es_of(const moe_config_t* c) { return c->dtype == MOE_DTYPE_FP32 ? 4 : 2; }
-inline int64_t max_rows_of(const moe_config_t* c) { return (int64_t)c->T * c->k + 31ll * c->E; }
+inline int64_t max_rows_of(const moe_config_t* c) {
+  return ((int64_t)c->T * c->k + 31ll * c->E + 31) / 32 * 32;
+}
 
 struct WsLayout {
   size_t head, hist, dlsel, dlogits, total;
@@ -132,7 +134,7 @@ int gemm_op(const moe_config_t* c, int op, const void* A, const void* B, void* C
   }
 }
 
-int64_t r32_of(const moe_config_t* c) { return (max_rows_of(c) + 31) / 32 * 32; }
+int64_t r32_of(const moe_config_t* c) { return max_rows_of(c); }
 
 int gemm_op_mx(const moe_config_t* c, int op, const uint8_t* Aq, const uint8_t* As, const uint8_t* Bq,
                const uint8_t* Bs, void* Cout, void* C2, const void* aux, const int32_t* counts,
@@ -442,6 +444,115 @@ int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_sav
   MOE_TRY(launch_token_reduce(g->dx_perm, sv->prow, dlsel, router ? sv->idx : nullptr, w->W_r, dx,
                               cfg->T, cfg->k, cfg->E, rb, bf, s));
   if (router) MOE_TRY(router_wgrad_impl(cfg, dlog, x, g->dW_r, ws, s));
+  return MOE_OK;
+}
+
+int moe_quantize_weights_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
+                               const moe_mxfp8_weights_t* qw, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(cfg->dtype == MOE_DTYPE_MXFP8, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(w && qw && w->W13 && w->W2, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(qw->W13q && qw->W13s && qw->W13tq && qw->W13ts && qw->W2q && qw->W2s && qw->W2tq &&
+                  qw->W2ts,
+              MOE_ERR_INVALID_ARG);
+  const int64_t E = cfg->E, d = cfg->d, F = cfg->F;
+  cudaStream_t s = S(stream);
+  MOE_TRY(moe_quantize_mxfp8(w->W13, E * 2 * F, (int)d, MOE_QUANT_ROW, qw->W13q, qw->W13s, s));
+  MOE_TRY(moe_quantize_mxfp8(w->W13, E * 2 * F, (int)d, MOE_QUANT_COL, qw->W13tq, qw->W13ts, s));
+  MOE_TRY(moe_quantize_mxfp8(w->W2, E * d, (int)F, MOE_QUANT_ROW, qw->W2q, qw->W2s, s));
+  return moe_quantize_mxfp8(w->W2, E * d, (int)F, MOE_QUANT_COL, qw->W2tq, qw->W2ts, s);
+}
+
+int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const moe_mxfp8_weights_t* qw,
+                        const void* x, const float* bias, void* out, moe_saved_t* sv,
+                        const moe_mxfp8_acts_t* qa, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(cfg->dtype == MOE_DTYPE_MXFP8, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(cfg->d % 128 == 0, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(w && qw && qa && sv && x && out, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(sv->idx && sv->gates && sv->counts && sv->offsets && sv->poff && sv->perm && sv->prow &&
+                  sv->row_token && sv->x_perm && sv->h13 && sv->a && sv->y,
+              MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(qa->xq && qa->xs && qa->aq && qa->as, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(x) && aligned16(out) && aligned16(sv->x_perm) && aligned16(sv->h13) &&
+                  aligned16(sv->a) && aligned16(sv->y),
+              MOE_ERR_INVALID_ARG);
+  cudaStream_t s = S(stream);
+  const int64_t R = max_rows_of(cfg);
+  const int d = cfg->d, F = cfg->F;
+  if (w->W_r) {
+    MOE_REQUIRE(sv->logits && aligned16(w->W_r) && aligned16(sv->logits), MOE_ERR_INVALID_ARG);
+    moe_config_t rc = *cfg;
+    rc.dtype = MOE_DTYPE_BF16;  // the router GEMM runs in bf16
+    MOE_TRY(router_logits_impl(&rc, x, w->W_r, bias, sv->logits, ws, s));
+    MOE_TRY(launch_topk(sv->logits, nullptr, cfg->T, cfg->E, cfg->k, cfg->renorm, sv->idx, sv->gates,
+                        err_of(ws), s));
+  }
+  const WsLayout L = ws_layout(cfg);
+  int32_t* hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.hist);
+  MOE_TRY(launch_metadata(sv->idx, cfg->T, cfg->E, cfg->k, R, sv->counts, sv->offsets, sv->poff,
+                          sv->perm, sv->prow, sv->row_token, hist, err_of(ws), s));
+  MOE_TRY(launch_dispatch(x, sv->prow, sv->counts, sv->poff, sv->x_perm, cfg->T, cfg->k, cfg->E, d * 2,
+                          s));
+  MOE_TRY(launch_quantize(sv->x_perm, R, d, MOE_QUANT_ROW, qa->xq, qa->xs, s));
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_FWD1_SWIGLU, qa->xq, qa->xs, qw->W13q, qw->W13s, sv->h13, sv->a,
+                     nullptr, sv->counts, sv->poff, ws, s));
+  MOE_TRY(launch_quantize(sv->a, R, F, MOE_QUANT_ROW, qa->aq, qa->as, s));
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_FWD2, qa->aq, qa->as, qw->W2q, qw->W2s, sv->y, nullptr, nullptr,
+                     sv->counts, sv->poff, ws, s));
+  return launch_combine(sv->y, sv->gates, sv->prow, out, cfg->T, cfg->k, d * 2, true, s);
+}
+
+int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const moe_mxfp8_weights_t* qw,
+                        const moe_saved_t* sv, const moe_mxfp8_acts_t* qa, const void* x,
+                        const void* dout, void* dx, moe_grads_t* g, void* ws, size_t ws_bytes,
+                        void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(cfg->dtype == MOE_DTYPE_MXFP8, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(cfg->d % 128 == 0, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(w && qw && qa && sv && g && x && dout && dx, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(g->dW13 && g->dW2 && g->dgates && g->dy && g->dh13 && g->dx_perm, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(qa->xtq && qa->xts && qa->atq && qa->ats && qa->dyq && qa->dys && qa->dytq && qa->dyts &&
+                  qa->dhq && qa->dhs && qa->dhtq && qa->dhts,
+              MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(dout) && aligned16(dx) && aligned16(g->dW13) && aligned16(g->dW2) &&
+                  aligned16(g->dy) && aligned16(g->dh13) && aligned16(g->dx_perm),
+              MOE_ERR_INVALID_ARG);
+  const bool router = w->W_r != nullptr;
+  moe_config_t rc = *cfg;
+  rc.dtype = MOE_DTYPE_BF16;
+  if (router) {
+    MOE_REQUIRE(cfg->renorm == 1, MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(router_shape_ok(&rc), MOE_ERR_UNSUPPORTED);
+    MOE_REQUIRE(g->dW_r && aligned16(g->dW_r), MOE_ERR_INVALID_ARG);
+  }
+  cudaStream_t s = S(stream);
+  const int64_t R = max_rows_of(cfg);
+  const int d = cfg->d, F = cfg->F;
+  const WsLayout L = ws_layout(cfg);
+  float* dlsel = router ? reinterpret_cast<float*>(static_cast<char*>(ws) + L.dlsel) : nullptr;
+  void* dlog = router ? static_cast<void*>(static_cast<char*>(ws) + L.dlogits) : nullptr;
+  MOE_TRY(launch_combine_bwd(dout, sv->y, sv->gates, sv->prow, sv->idx, sv->counts, sv->poff, g->dy,
+                             g->dgates, dlsel, dlog, cfg->T, cfg->k, cfg->E, d * 2, true, s));
+  MOE_TRY(launch_quantize(g->dy, R, d, MOE_QUANT_ROW, qa->dyq, qa->dys, s));
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_DGRAD2_SWIGLU, qa->dyq, qa->dys, qw->W2tq, qw->W2ts, g->dh13,
+                     nullptr, sv->h13, sv->counts, sv->poff, ws, s));
+  MOE_TRY(launch_quantize(g->dy, R, d, MOE_QUANT_COL, qa->dytq, qa->dyts, s));
+  MOE_TRY(launch_quantize(sv->a, R, F, MOE_QUANT_COL, qa->atq, qa->ats, s));
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD2, qa->dytq, qa->dyts, qa->atq, qa->ats, g->dW2, nullptr,
+                     nullptr, sv->counts, sv->poff, ws, s));
+  MOE_TRY(launch_quantize(g->dh13, R, 2 * F, MOE_QUANT_ROW, qa->dhq, qa->dhs, s));
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_DGRAD1, qa->dhq, qa->dhs, qw->W13tq, qw->W13ts, g->dx_perm, nullptr,
+                     nullptr, sv->counts, sv->poff, ws, s));
+  MOE_TRY(launch_quantize(g->dh13, R, 2 * F, MOE_QUANT_COL, qa->dhtq, qa->dhts, s));
+  MOE_TRY(launch_quantize(sv->x_perm, R, d, MOE_QUANT_COL, qa->xtq, qa->xts, s));
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD1, qa->dhtq, qa->dhts, qa->xtq, qa->xts, g->dW13, nullptr,
+                     nullptr, sv->counts, sv->poff, ws, s));
+  MOE_TRY(launch_token_reduce(g->dx_perm, sv->prow, dlsel, router ? sv->idx : nullptr, w->W_r, dx,
+                              cfg->T, cfg->k, cfg->E, d * 2, true, s));
+  if (router) MOE_TRY(router_wgrad_impl(&rc, dlog, x, g->dW_r, ws, s));
   return MOE_OK;
 }
 

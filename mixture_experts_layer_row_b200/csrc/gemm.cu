@@ -130,6 +130,13 @@ __device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const i
   }
 }
 
+// Round an fp32 value to the output element type (bf16 for 2-byte outputs) and back.
+template <int OES>
+__device__ __forceinline__ float round_out(float v) {
+  if constexpr (OES == 2) return __bfloat162float(__float2bfloat16_rn(v));
+  else return v;
+}
+
 // SwiGLU helpers with the fast exponential and division intrinsics (bf16 outputs need ~8 bits).
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.f + __expf(-g)); }
 
@@ -540,8 +547,9 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
             float g[32], u[32], a[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              g[i] = __uint_as_float(rg[i]);
-              u[i] = __uint_as_float(ru[i]);
+              // round to the stored precision first: a is computed from the h13 that is kept
+              g[i] = round_out<C::OES>(__uint_as_float(rg[i]));
+              u[i] = round_out<C::OES>(__uint_as_float(ru[i]));
               a[i] = silu_f(g[i]) * u[i];
             }
             if (active) {

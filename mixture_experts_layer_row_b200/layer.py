@@ -9,7 +9,8 @@ import torch
 
 from . import _lib as L
 
-_DT = {"fp32": (L.DTYPE_FP32, torch.float32), "bf16": (L.DTYPE_BF16, torch.bfloat16)}
+_DT = {"fp32": (L.DTYPE_FP32, torch.float32), "bf16": (L.DTYPE_BF16, torch.bfloat16),
+       "mxfp8": (L.DTYPE_MXFP8, torch.bfloat16)}
 
 
 class MoELayer:
@@ -17,7 +18,8 @@ class MoELayer:
 
     Args:
         T, d, F, E, k: tokens, model width, expert hidden width, experts, experts per token.
-        dtype: "bf16" (bf16 storage, fp32 accumulate) or "fp32" (GEMMs on tf32 tensor cores).
+        dtype: "bf16" (bf16 storage, fp32 accumulate), "fp32" (GEMMs on tf32 tensor cores) or
+            "mxfp8" (bf16 storage, expert GEMMs on E4M3 operands with UE8M0 block scales).
         learned_router: allocate router buffers (scores, score gradients, dW_r).
     """
 
@@ -50,6 +52,24 @@ class MoELayer:
         self.dW_r = z((E, d), act) if learned_router else None
         self.dgates = z((T, k), f32)
         self.dy, self.dh13, self.dx_perm = z((R, d), act), z((R, 2 * F), act), z((R, d), act)
+        self.mx = dtype == "mxfp8"
+        if self.mx:
+            u8 = torch.uint8
+            self.qw_t = {  # quantised weights
+                "W13q": z((E * 2 * F, d), u8), "W13s": z((E * 2 * F, d // 32), u8),
+                "W13tq": z((E * 2 * F, d), u8), "W13ts": z((d, E * 2 * F // 32), u8),
+                "W2q": z((E * d, F), u8), "W2s": z((E * d, F // 32), u8),
+                "W2tq": z((E * d, F), u8), "W2ts": z((F, E * d // 32), u8)}
+            self.qa_t = {}
+            for nm, cols in (("x", d), ("a", F), ("dy", d), ("dh", 2 * F)):
+                self.qa_t[nm + "q"] = z((R, cols), u8)
+                self.qa_t[nm + "s"] = z((R, cols // 32), u8)
+                self.qa_t[nm + "tq"] = z((R, cols), u8)
+                self.qa_t[nm + "ts"] = z((cols, R // 32), u8)
+            self.qw = L.MxWeights(*[L.ptr(self.qw_t[n]) for n, _ in L.MxWeights._fields_])
+            order = ["xq", "xs", "xtq", "xts", "aq", "as", "atq", "ats", "dyq", "dys", "dytq", "dyts",
+                     "dhq", "dhs", "dhtq", "dhts"]
+            self.qa = L.MxActs(*[L.ptr(self.qa_t[n]) for n in order])
         self.saved = L.Saved(*[L.ptr(t) for t in (self.logits, self.idx, self.gates, self.counts,
                                                   self.offsets, self.poff, self.perm, self.prow,
                                                   self.row_token, self.x_perm, self.h13, self.a,
@@ -66,6 +86,12 @@ class MoELayer:
             raise ValueError("learned router needs W_r")
         self._keep = (W13, W2, W_r)
         self._w = L.Weights(L.ptr(W_r) if self.learned_router else None, L.ptr(W13), L.ptr(W2))
+        if self.mx:
+            self.quantize_weights()
+
+    def quantize_weights(self, stream=None):
+        """Refresh the MXFP8 weight copies (after every weight update)."""
+        L.quantize_weights_mxfp8(self.cfg, self._w, self.qw, stream)
 
     def forward(self, x, bias=None, idx=None, gates=None, stream=None):
         """out = layer(x). With a learned router, routing comes from x W_r^T (+ bias); otherwise
@@ -76,12 +102,21 @@ class MoELayer:
             self.idx.copy_(idx)
             self.gates.copy_(gates)
         self._x = x
-        L.layer_fwd(self.cfg, self._w, x, bias, self.out, self.saved, self.ws, stream)
+        if self.mx:
+            L.layer_fwd_mxfp8(self.cfg, self._w, self.qw, x, bias, self.out, self.saved, self.qa,
+                              self.ws, stream)
+        else:
+            L.layer_fwd(self.cfg, self._w, x, bias, self.out, self.saved, self.ws, stream)
         return self.out
 
     def backward(self, dout, stream=None):
         """Fills dx, dW13, dW2 (and dW_r, dgates)."""
-        L.layer_bwd(self.cfg, self._w, self.saved, self._x, dout, self.dx, self.grads, self.ws, stream)
+        if self.mx:
+            L.layer_bwd_mxfp8(self.cfg, self._w, self.qw, self.saved, self.qa, self._x, dout, self.dx,
+                              self.grads, self.ws, stream)
+        else:
+            L.layer_bwd(self.cfg, self._w, self.saved, self._x, dout, self.dx, self.grads, self.ws,
+                        stream)
         return self.dx
 
     def error_flags(self, stream=None) -> int:

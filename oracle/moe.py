@@ -187,6 +187,15 @@ def _ident(a):
     return a
 
 
+def bf16_round(a):
+    """Round to bfloat16 (nearest, ties to even) through fp32, the precision the MXFP8 workload stores
+    every GEMM output and activation in ("bf16 outputs"). Returned as float64."""
+    f = np.asarray(a, dtype=np.float64).astype(np.float32)
+    b = f.view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) >> 16 << 16
+    return b.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 def _mx_row(a):
     """MXFP8 fake-quantisation with blocks of 32 along the last (contraction) axis."""
     from . import mxfp8
@@ -238,8 +247,14 @@ def expert_fwd(X: np.ndarray, W13_e: np.ndarray, W2_e: np.ndarray, mx: bool = Fa
     """One expert on its rows X [n,d]: h13 = X W13_e^T = [gate | up], a = silu(gate)*up, y = a W2_e^T.
     With `mx`, every GEMM operand is MXFP8-quantised along that GEMM's contraction axis first."""
     qr = _mx_row if mx else _ident
-    h13, a = gemm_fwd1_swiglu(X, W13_e, qr)
-    return h13, a, gemm_fwd2(a, W2_e, qr)
+    if not mx:
+        h13, a = gemm_fwd1_swiglu(X, W13_e, qr)
+        return h13, a, gemm_fwd2(a, W2_e, qr)
+    # MXFP8 workload: GEMM outputs and activations are stored in bf16; SwiGLU reads the stored h13
+    F = W13_e.shape[0] // 2
+    h13 = bf16_round(qr(X) @ qr(W13_e).T)
+    a = bf16_round(silu(h13[:, :F]) * h13[:, F:])
+    return h13, a, bf16_round(gemm_fwd2(a, W2_e, qr))
 
 
 def expert_bwd(X, W13_e, W2_e, h13, a, dY, mx: bool = False):
@@ -248,7 +263,8 @@ def expert_bwd(X, W13_e, W2_e, h13, a, dY, mx: bool = False):
     operand of a dgrad GEMM and for both operands of a wgrad GEMM)."""
     qr = _mx_row if mx else _ident
     qc = _mx_col if mx else _ident
-    dH13 = gemm_dgrad2_swiglu(dY, W2_e, h13, qr, qc)   # [n,2F]
+    st = bf16_round if mx else _ident                  # MXFP8 workload: bf16 storage
+    dH13 = st(gemm_dgrad2_swiglu(dY, W2_e, h13, qr, qc))   # [n,2F]
     dW2 = gemm_wgrad(dY, a, qc)                        # [d,F]
     dW13 = gemm_wgrad(dH13, X, qc)                     # [2F,d]
     dX = gemm_dgrad1(dH13, W13_e, qr, qc)              # [n,d]
@@ -319,6 +335,8 @@ def layer_bwd(dout, x, W13, W2, idx, gates, saved, W_r=None, renorm=True, logits
     E, F2, d = W13.shape
     rows = saved["x_perm"].shape[0]
     dy, dgates = combine_bwd(dout, saved["y"], gates, meta)
+    if mx:
+        dy = bf16_round(dy)
     dW13 = np.zeros_like(W13, dtype=np.float64)
     dW2 = np.zeros_like(W2, dtype=np.float64)
     dxp = np.zeros((rows, d))
@@ -395,3 +413,53 @@ def expert_grads(e, x, W13, W2, idx, gates, dout):
         dW13[:F] += np.outer(da * up * silu_grad(gate), x[t])
         dW13[F:] += np.outer(da * silu(gate), x[t])
     return dW13, dW2
+
+
+# ----------------------------------------------------------------------------------------------
+# MXFP8 per-token forms (sampled checks at full size). Row-wise quantisation of an activation row
+# depends on that row only, so the forward and the input gradient of one token follow from the
+# token's own rows plus the quantised expert weights:
+#   qw[e] = (W13 fake-quantised along d, W2 along F, W13 along 2F, W2 along d)
+# ----------------------------------------------------------------------------------------------
+
+def quantised_expert_weights(W13_e, W2_e):
+    """The four MXFP8 forms of one expert's weights used by its forward and dgrad GEMMs."""
+    return (_mx_row(W13_e), _mx_row(W2_e), _mx_col(W13_e), _mx_col(W2_e))
+
+
+def token_out_mx(t, x, qw, idx, gates) -> np.ndarray:
+    """out_t with every expert GEMM operand MXFP8-quantised along its contraction axis."""
+    acc = np.zeros(x.shape[1])
+    for j in range(idx.shape[1]):
+        e = int(idx[t, j])
+        W13r, W2r, _, _ = qw[e]
+        h13, a = _token_fwd1_mx(x[t], W13r)
+        acc += gates[t, j] * bf16_round(gemm_fwd2(a, W2r, _mx_row))[0]
+    return acc
+
+
+def _token_fwd1_mx(xt, W13r):
+    """GEMM1 + SwiGLU of one token with bf16 storage (W13r already quantised along d)."""
+    F = W13r.shape[0] // 2
+    h13 = bf16_round(_mx_row(xt[None, :]) @ W13r.T)
+    return h13, bf16_round(silu(h13[:, :F]) * h13[:, F:])
+
+
+def token_dx_mx(t, x, qw, idx, gates, dout, W_r=None) -> np.ndarray:
+    """d(loss)/d(x_t) for the MXFP8 layer (renormalised gates; router term when W_r is given)."""
+    k = idx.shape[1]
+    dx = np.zeros(x.shape[1])
+    dg = np.zeros(k)
+    for j in range(k):
+        e = int(idx[t, j])
+        W13r, W2r, W13c, W2c = qw[e]
+        h13, a = _token_fwd1_mx(x[t], W13r)
+        dg[j] = float(dout[t] @ bf16_round(gemm_fwd2(a, W2r, _mx_row))[0])
+        dy = bf16_round(gates[t, j] * dout[t][None, :])
+        dH13 = bf16_round(gemm_dgrad2_swiglu(dy, W2c, h13, _mx_row, _ident))
+        dx += gemm_dgrad1(dH13, W13c, _mx_row, _ident)[0]
+    if W_r is not None:
+        s = float(np.dot(gates[t], dg))
+        for j in range(k):
+            dx += gates[t, j] * (dg[j] - s) * W_r[int(idx[t, j])]
+    return dx

@@ -27,8 +27,7 @@ SMALL = {
 def run_layer(w: Workload, inp: dict):
     from mixture_experts_layer_row_b200 import MoELayer
     learned = w.routing == "learned"
-    layer = MoELayer(w.T, w.d, w.F, w.E, w.k, dtype="fp32" if w.dtype == "fp32" else "bf16",
-                     learned_router=learned)
+    layer = MoELayer(w.T, w.d, w.F, w.E, w.k, dtype=w.dtype, learned_router=learned)
     layer.set_weights(inp["W13"], inp["W2"], inp["W_r"] if learned else None)
     out = layer.forward(inp["x"], bias=inp["bias"], idx=inp["idx"], gates=inp["gates"])
     layer.backward(inp["dout"])
@@ -144,3 +143,69 @@ def test_layer_twice_is_deterministic():
     o1, dx1, dw1 = o1.clone(), l1.dx.clone(), l1.dW13.clone()
     l2, o2 = run_layer(w, inp)
     assert torch.equal(o1, o2) and torch.equal(dx1, l2.dx) and torch.equal(dw1, l2.dW13)
+
+
+# ------------------------------------------------------------------------------------------------
+# MXFP8 layer: against the oracle with the same quantisation (OCP MX along every GEMM's contraction
+# axis); the tolerance is the MXFP8 bar, 8e-2 * max|ref|. The distance to the unquantised fp64 layer
+# is printed for the record (E4M3 itself carries several percent).
+# ------------------------------------------------------------------------------------------------
+
+TOL_MX = 8e-2
+MX_SMALL = {
+    "mx_uniform": Workload("mx_uniform", 512, 256, 256, 16, 4, "mxfp8", "uniform"),
+    "mx_learned": Workload("mx_learned", 384, 256, 384, 8, 2, "mxfp8", "learned"),
+}
+
+
+@pytest.mark.parametrize("name", list(MX_SMALL))
+def test_layer_mxfp8_small_full_oracle(name):
+    w = MX_SMALL[name]
+    inp = make_inputs(w, seed=0, device="cuda")
+    layer, out = run_layer(w, inp)
+    x64, W13, W2, Wr, dout = (np64(inp[n]) for n in ("x", "W13", "W2", "W_r", "dout"))
+    learned = w.routing == "learned"
+    idx, gates_ref = _routing_checks(w, layer, inp, x64, Wr)
+    ref_out, saved = O.layer_fwd(x64, W13, W2, idx, gates_ref, mx=True)
+    gr = O.layer_bwd(dout, x64, W13, W2, idx, gates_ref, saved, W_r=Wr if learned else None, mx=True)
+    errs = {"out": assert_close_rel(np64(out), ref_out, TOL_MX, "out"),
+            "dx": assert_close_rel(np64(layer.dx), gr["dx"], TOL_MX, "dx"),
+            "dW13": assert_close_rel(np64(layer.dW13), gr["dW13"], TOL_MX, "dW13"),
+            "dW2": assert_close_rel(np64(layer.dW2), gr["dW2"], TOL_MX, "dW2")}
+    if learned:
+        errs["dW_r"] = assert_close_rel(np64(layer.dW_r), gr["dW_r"], TOL_MX, "dW_r")
+    plain_out, _ = O.layer_fwd(x64, W13, W2, idx, gates_ref)
+    print(name, "rel err vs MXFP8 oracle", {k: round(v, 5) for k, v in errs.items()},
+          "| out vs unquantised fp64:",
+          round(float(np.max(np.abs(np64(out) - plain_out)) / np.max(np.abs(plain_out))), 4))
+
+
+def test_layer_mxfp8_full_size_sampled():
+    w = WORKLOADS["e128_mxfp8"]
+    inp = make_inputs(w, seed=0, device="cuda")
+    layer, out = run_layer(w, inp)
+    x64 = np64(inp["x"])
+    idx, gates_ref = _routing_checks(w, layer, inp, x64, None)
+    dout = np64(inp["dout"])
+    rng = np.random.default_rng(2)
+    toks = [0, w.T - 1] + [int(t) for t in rng.integers(0, w.T, 4)]
+    got_out, got_dx, ref_out, ref_dx = [], [], [], []
+    for t in toks:  # quantised weights of the token's experts only, built per token
+        qw = {int(e): O.quantised_expert_weights(np64(inp["W13"][int(e)]), np64(inp["W2"][int(e)]))
+              for e in idx[t]}
+        ref_out.append(O.token_out_mx(t, x64, qw, idx, gates_ref))
+        ref_dx.append(O.token_dx_mx(t, x64, qw, idx, gates_ref, dout))
+        got_out.append(np64(out[t]))
+        got_dx.append(np64(layer.dx[t]))
+    assert_close_rel(np.stack(got_out), np.stack(ref_out), TOL_MX, "sampled out")
+    assert_close_rel(np.stack(got_dx), np.stack(ref_dx), TOL_MX, "sampled dx")
+    counts = np.bincount(idx.reshape(-1), minlength=w.E)
+    for e in sorted({int(np.argmax(counts)), int(rng.integers(0, w.E))}):
+        tj = np.argwhere(idx == e)
+        X = x64[tj[:, 0]]
+        dY = O.bf16_round(gates_ref[tj[:, 0], tj[:, 1]][:, None] * dout[tj[:, 0]])  # stored bf16
+        W13e, W2e = np64(inp["W13"][e]), np64(inp["W2"][e])
+        h13, a, _ = O.expert_fwd(X, W13e, W2e, mx=True)
+        _, dW13, dW2, _ = O.expert_bwd(X, W13e, W2e, h13, a, dY, mx=True)
+        assert_close_rel(np64(layer.dW13[e]), dW13, TOL_MX, f"dW13[{e}]")
+        assert_close_rel(np64(layer.dW2[e]), dW2, TOL_MX, f"dW2[{e}]")

@@ -420,3 +420,22 @@ def test_mxfp8_quantisation_axes():
     _, sv = O.layer_fwd(x, W13, W2, idx, g)
     _, svq = O.layer_fwd(x, W13, W2, idx, g, mx=True)
     np.testing.assert_array_equal(svq["h13"], sv["h13"])
+
+
+def test_mxfp8_per_token_forms_match_grouped():
+    """Row-wise quantisation is per row, so the per-token MXFP8 output and input gradient equal the
+    grouped MXFP8 layer's (the wgrads, whose blocks span tokens, are not per-token)."""
+    rng = np.random.default_rng(15)
+    T, d, F, E, k = 40, 64, 64, 4, 2
+    x = rng.standard_normal((T, d))
+    W13 = rng.standard_normal((E, 2 * F, d)) * 0.1
+    W2 = rng.standard_normal((E, d, F)) * 0.1
+    dout = rng.standard_normal((T, d))
+    idx, g = O.route(rng.standard_normal((T, E)), k)
+    out, sv = O.layer_fwd(x, W13, W2, idx, g, mx=True)
+    gr = O.layer_bwd(dout, x, W13, W2, idx, g, sv, mx=True)
+    qw = {e: O.quantised_expert_weights(W13[e], W2[e]) for e in range(E)}
+    for t in range(0, T, 3):
+        np.testing.assert_allclose(O.token_out_mx(t, x, qw, idx, g), out[t], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(O.token_dx_mx(t, x, qw, idx, g, dout), gr["dx"][t], rtol=1e-10,
+                                   atol=1e-12)
