@@ -45,7 +45,44 @@ def load_peaks():
 # algorithmic work per op (bytes moved once, flops of the definition); R = routed rows = T*k
 # ------------------------------------------------------------------------------------------------
 
+def op_work_mx(w):
+    """Per-op algorithmic (bytes, flops) of the MXFP8 layer step: fp8 codes + 1/32 scale bytes for GEMM
+    operands, bf16 for everything stored."""
+    T, d, F, E, k = w.T, w.d, w.F, w.E, w.k
+    R = T * k
+    Rp = R + 31 * E
+    q = lambda n: n + n // 32          # codes + scales of n elements
+    ops = {}
+    ops["route_metadata"] = (T * k * 4 * 3 + Rp * 4, 0)
+    ops["dispatch"] = ((T + R) * d * 2, 0)
+    ops["quant_x_row"] = (R * d * 2 + q(R * d), 0)
+    ops["gemm_fwd1_swiglu"] = (q(R * d) + q(E * 2 * F * d) + (R * 2 * F + R * F) * 2, 4 * R * d * F)
+    ops["quant_a_row"] = (R * F * 2 + q(R * F), 0)
+    ops["gemm_fwd2"] = (q(R * F) + q(E * d * F) + R * d * 2, 2 * R * F * d)
+    ops["combine"] = ((R * d + T * d) * 2 + T * k * 8, 0)
+    ops["combine_bwd"] = ((T * d + 2 * R * d) * 2 + T * k * 12, 0)
+    ops["quant_dy_row"] = (R * d * 2 + q(R * d), 0)
+    ops["gemm_dgrad2_swiglu"] = (q(R * d) + q(E * d * F) + 2 * R * 2 * F * 2, 2 * R * d * F)
+    ops["quant_dy_col"] = (R * d * 2 + q(R * d), 0)
+    ops["quant_a_col"] = (R * F * 2 + q(R * F), 0)
+    ops["gemm_wgrad2"] = (q(R * d) + q(R * F) + E * d * F * 2, 2 * R * d * F)
+    ops["quant_dh_row"] = (R * 2 * F * 2 + q(R * 2 * F), 0)
+    ops["gemm_dgrad1"] = (q(R * 2 * F) + q(E * 2 * F * d) + R * d * 2, 4 * R * F * d)
+    ops["quant_dh_col"] = (R * 2 * F * 2 + q(R * 2 * F), 0)
+    ops["quant_x_col"] = (R * d * 2 + q(R * d), 0)
+    ops["gemm_wgrad1"] = (q(R * 2 * F) + q(R * d) + E * 2 * F * d * 2, 4 * R * F * d)
+    ops["token_reduce"] = ((R * d + T * d) * 2, 0)
+    return ops
+
+
+def weight_quant_work(w):
+    n = w.E * 2 * w.F * w.d + w.E * w.d * w.F  # W13 + W2 elements
+    return 2 * (n * 2 + n + n // 32)            # two orientations: read bf16, write codes + scales
+
+
 def op_work(w, es=2):
+    if w.dtype == "mxfp8":
+        return op_work_mx(w)
     T, d, F, E, k = w.T, w.d, w.F, w.E, w.k
     R = T * k
     Rp = R + 31 * E  # upper bound of padded rows written (pad rows are written as zeros)
@@ -94,6 +131,8 @@ class Step:
                    for _ in range(n_steps)]
 
     def run(self, i=None):
+        if self.layer.mx:
+            return self.run_mx(i)
         L, lay, w, inp = self.L, self.layer, self.w, self.inp
         ev = self.ev[i] if (i is not None and self.ev is not None) else None
         c = lay.cfg
@@ -132,6 +171,51 @@ class Step:
                                lay.idx if self.learned else None, inp["W_r"] if self.learned else None)
         if self.learned:
             mark(); L.router_wgrad(c, self.dlogits, inp["x"], lay.dW_r, lay.ws)
+        mark()
+
+
+    def run_mx(self, i=None):
+        """The kernels of moe_layer_fwd_mxfp8 / moe_layer_bwd_mxfp8, op by op (uniform routing)."""
+        L, lay, w, inp = self.L, self.layer, self.w, self.inp
+        ev = self.ev[i] if (i is not None and self.ev is not None) else None
+        c, qa, qw = lay.cfg, lay.qa_t, lay.qw_t
+        n = 0
+
+        def mark():
+            nonlocal n
+            if ev is not None:
+                ev[n].record()
+            n += 1
+
+        R, ROW, COL = lay.R, L.QUANT_ROW, L.QUANT_COL
+        cnt, po, ws = lay.counts, lay.poff, lay.ws
+        mark(); L.route_metadata(c, lay.idx, lay.counts, lay.offsets, lay.poff, lay.perm, lay.prow,
+                                 lay.row_token, ws)
+        mark(); L.dispatch(c, inp["x"], lay.prow, cnt, po, lay.x_perm)
+        mark(); L.quantize_mxfp8(lay.x_perm, qa["xq"], qa["xs"], ROW)
+        mark(); L.grouped_gemm_mxfp8(c, L.GEMM_FWD1_SWIGLU, qa["xq"], qa["xs"], qw["W13q"], qw["W13s"],
+                                     lay.h13, lay.a, None, cnt, po, ws)
+        mark(); L.quantize_mxfp8(lay.a, qa["aq"], qa["as"], ROW)
+        mark(); L.grouped_gemm_mxfp8(c, L.GEMM_FWD2, qa["aq"], qa["as"], qw["W2q"], qw["W2s"], lay.y,
+                                     None, None, cnt, po, ws)
+        mark(); L.combine(c, lay.y, lay.gates, lay.prow, lay.out)
+        mark(); L.combine_bwd(c, inp["dout"], lay.y, lay.gates, lay.prow, lay.idx, cnt, po, lay.dy,
+                              lay.dgates)
+        mark(); L.quantize_mxfp8(lay.dy, qa["dyq"], qa["dys"], ROW)
+        mark(); L.grouped_gemm_mxfp8(c, L.GEMM_DGRAD2_SWIGLU, qa["dyq"], qa["dys"], qw["W2tq"],
+                                     qw["W2ts"], lay.dh13, None, lay.h13, cnt, po, ws)
+        mark(); L.quantize_mxfp8(lay.dy, qa["dytq"], qa["dyts"], COL)
+        mark(); L.quantize_mxfp8(lay.a, qa["atq"], qa["ats"], COL)
+        mark(); L.grouped_gemm_mxfp8(c, L.GEMM_WGRAD2, qa["dytq"], qa["dyts"], qa["atq"], qa["ats"],
+                                     lay.dW2, None, None, cnt, po, ws)
+        mark(); L.quantize_mxfp8(lay.dh13, qa["dhq"], qa["dhs"], ROW)
+        mark(); L.grouped_gemm_mxfp8(c, L.GEMM_DGRAD1, qa["dhq"], qa["dhs"], qw["W13tq"], qw["W13ts"],
+                                     lay.dx_perm, None, None, cnt, po, ws)
+        mark(); L.quantize_mxfp8(lay.dh13, qa["dhtq"], qa["dhts"], COL)
+        mark(); L.quantize_mxfp8(lay.x_perm, qa["xtq"], qa["xts"], COL)
+        mark(); L.grouped_gemm_mxfp8(c, L.GEMM_WGRAD1, qa["dhtq"], qa["dhts"], qa["xtq"], qa["xts"],
+                                     lay.dW13, None, None, cnt, po, ws)
+        mark(); L.token_reduce(c, lay.dx_perm, lay.prow, lay.dx)
         mark()
 
 
@@ -193,7 +277,44 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def cpu_baseline_experts(w, inp, n_experts, label):
+    """The fp64 oracle's per-expert forward + backward (MXFP8 emulated when the workload is MXFP8) on
+    every routed row of the first n_experts experts; for workloads whose fp64 weights do not fit the
+    host comfortably. Throughput = processed routed rows / k per second."""
+    import numpy as np
+    import torch
+    from oracle import moe as O
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    mx = w.dtype == "mxfp8"
+    idx = inp["idx"].cpu().numpy().astype(np.int64)
+    gates = f64(inp["gates"])
+    x = f64(inp["x"])
+    dout = f64(inp["dout"])
+    rows = 0
+    t0 = time.perf_counter()
+    for e in range(n_experts):
+        tj = np.argwhere(idx == e)
+        X = x[tj[:, 0]]
+        dY = gates[tj[:, 0], tj[:, 1]][:, None] * dout[tj[:, 0]]
+        W13e, W2e = f64(inp["W13"][e]), f64(inp["W2"][e])
+        h13, a, y = O.expert_fwd(X, W13e, W2e, mx)
+        O.expert_bwd(X, W13e, W2e, h13, a, dY, mx)
+        rows += len(tj)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+    except Exception:
+        cores = 1
+    return {"value": rows / w.k / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{label}: experts 0..{n_experts - 1}, all {rows} of their routed rows "
+                      f"({'MXFP8-emulated ' if mx else ''}fp64 per-expert forward + backward incl. "
+                      f"weight conversion), {dt:.1f} s; tokens/s = rows / k / s"}
+
+
 def cpu_baseline(w, inp, n_tokens, label):
+    if w.E * 3 * w.F * w.d > 1_500_000_000 or w.dtype == "mxfp8":
+        return cpu_baseline_experts(w, inp, 6, label)
     """The fp64 oracle, as it stands, on the first n_tokens tokens of the workload (their routing,
     the full expert weights), forward + backward; returns tokens/s and what was run."""
     import numpy as np
@@ -279,9 +400,6 @@ def main():
 
     from moe_workloads import WORKLOADS
     w = WORKLOADS[args.workload]
-    if w.dtype not in ("bf16", "fp32"):
-        print(json.dumps({"error": f"workload {w.name} ({w.dtype}) is not built yet"}))
-        return 2
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -359,7 +477,10 @@ def main():
     peaks = load_peaks()
     work = op_work(w, 4 if w.dtype == "fp32" else 2)
     bw = peaks["hbm_gbs"]
-    tc = peaks["bf16_tflops"] * (0.5 if w.dtype == "fp32" else 1.0)  # tf32 dense = half of bf16
+    # tensor peak of the GEMMs' own dtype: the measured bf16 figure times the nominal dense ratio
+    # (tf32 1.1 / bf16 2.25 PFLOP/s; fp8 4.5 / 2.25)
+    ratio = {"fp32": 0.5, "bf16": 1.0, "mxfp8": 2.0}[w.dtype]
+    tc = peaks["bf16_tflops"] * ratio
     roof_time = 0.0
     for n, (b, f) in work.items():
         roof_time += max(b / (bw * 1e9), f / (tc * 1e12))
@@ -378,7 +499,21 @@ def main():
         roof = {"kernel": dom, "bound": "tensor", "achieved": f / t_dom / 1e12, "peak": tc,
                 "unit": "TFLOP/s", "frac": (f / t_dom / 1e12) / tc, "traffic": None,
                 "algorithmic_bytes": b, "flops": f, "ms": per_op[dom],
-                "peak_source": f"{peaks['source']} bf16_tflops (burst)"}
+                "peak_source": f"{peaks['source']} bf16_tflops (burst) x {ratio} ({w.dtype})"}
+
+    wq = None
+    if layer.mx:  # weights are quantised once per update: timed on their own, not in the step
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        layer.quantize_weights()
+        q0.record()
+        for _ in range(5):
+            layer.quantize_weights()
+        q1.record()
+        torch.cuda.synchronize()
+        wq_ms = q0.elapsed_time(q1) / 5
+        wq = {"ms": wq_ms, "GB/s": weight_quant_work(w) / (wq_ms / 1e3) / 1e9,
+              "tokens_per_s_including_it": world * w.T / ((ms_per_step + wq_ms) / 1e3),
+              "note": "once per weight update (optimizer step), outside the timed layer step"}
 
     # end to end through the public layer API: host inputs in, host results out, every step
     e2e = None
@@ -446,6 +581,7 @@ def main():
                                "peaks": peaks},
             "roofline": roof,
             "per_op_ms": {n: round(v, 4) for n, v in per_op.items()},
+            "weight_quantisation": wq,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
