@@ -50,7 +50,7 @@ def op_work_mx(w):
     operands, bf16 for everything stored."""
     T, d, F, E, k = w.T, w.d, w.F, w.E, w.k
     R = T * k
-    Rp = R + 31 * E
+    Rp = R + 127 * E                   # 128-row groups in MXFP8 mode
     q = lambda n: n + n // 32          # codes + scales of n elements
     ops = {}
     ops["route_metadata"] = (T * k * 4 * 3 + Rp * 4, 0)
@@ -187,7 +187,7 @@ class Step:
                 ev[n].record()
             n += 1
 
-        R, ROW, COL = lay.R, L.QUANT_ROW, L.QUANT_COL
+        R, ROW, COL = lay.R, L.QUANT_ROW_TILED, L.QUANT_COL_TILED
         cnt, po, ws = lay.counts, lay.poff, lay.ws
         mark(); L.route_metadata(c, lay.idx, lay.counts, lay.offsets, lay.poff, lay.perm, lay.prow,
                                  lay.row_token, ws)

@@ -27,9 +27,10 @@
  *     (rows 0..F-1 gate W1, rows F..2F-1 up W3), W2 [E,d,F].
  *   - "act" dtype is fp32 when cfg->dtype == MOE_DTYPE_FP32 and bf16 otherwise. Router scores,
  *     gates and gate gradients are always fp32; index arrays are int32.
- *   - Routed-row buffers have moe_max_rows(cfg) = T*k + 31*E rows rounded up to a multiple of 32: each
- *     expert's group starts on a 32-row boundary (poff) and its pad rows are kept at zero by the
- *     kernels that write the buffer.
+ *   - Routed-row buffers have moe_max_rows(cfg) rows: T*k + (A-1)*E rounded up to a multiple of A,
+ *     where A, the group alignment, is 32 rows (128 in MXFP8 mode, whose scales move in 128-row
+ *     chunks). Each expert's group starts on an A-row boundary (poff) and its pad rows are kept at
+ *     zero by the kernels that write the buffer.
  *   - Every function returns MOE_OK (0) or a negative MOE_ERR_* code. Arguments are validated on the
  *     host before anything is enqueued; on an error nothing is enqueued.
  *   - Device-side problems (an expert id outside [0,E), counts that do not add up to T*k, a
@@ -84,7 +85,8 @@ typedef struct {
   int renorm; /* 1: gates renormalised over the chosen k (required by the backward pass) */
 } moe_config_t;
 
-/* Rows of every routed-row buffer: T*k + 31*E rounded up to 32. Returns 0 for an invalid config. */
+/* Rows of every routed-row buffer: T*k + (A-1)*E rounded up to A (A = 32, or 128 in MXFP8 mode).
+ * Returns 0 for an invalid config. */
 MOE_API int64_t moe_max_rows(const moe_config_t* cfg);
 
 /* Bytes of scratch the layer-level calls need (routing histograms, router-gradient scratch and the
@@ -116,8 +118,9 @@ MOE_API int moe_route_topk(const moe_config_t* cfg, const float* logits, const f
  * "Como funciona"). Outputs (all int32):
  *   counts[E]      rows routed to each expert;
  *   offsets[E+1]   exclusive prefix sum of counts, offsets[E] = T*k;
- *   poff[E+1]      exclusive prefix sum of counts rounded up to 32: expert e owns padded rows
- *                  [poff[e], poff[e+1]) of every routed-row buffer;
+ *   poff[E+1]      exclusive prefix sum of counts rounded up to the group alignment (32 rows,
+ *                  128 for MXFP8 configs): expert e owns padded rows [poff[e], poff[e+1]) of every
+ *                  routed-row buffer;
  *   perm[T*k]      position of entry t*k+j in the expert-sorted order, ascending token id within an
  *                  expert (a stable counting sort; deterministic, no atomics in the ordering);
  *   prow[T*k]      padded row of entry t*k+j: poff[e] + perm - offsets[e];
@@ -150,7 +153,8 @@ MOE_API int moe_route_metadata_noalloc(const moe_config_t* cfg, const int32_t* i
 
 /* Row-wise dispatch (unite.ai, "Parallelismo, precisione e tecniche di memoria": each routed token is
  * written directly into its expert's input buffer): x_perm[prow[t*k+j]] = x[t] for all j, and every
- * pad row [poff[e]+counts[e], poff[e+1]) is zeroed. x: act [T,d]; x_perm: act [max_rows,d]. */
+ * pad row [poff[e]+counts[e], poff[e+1]) is zeroed. x: act [T,d]; x_perm: act [max_rows,d] (bf16 in
+ * MXFP8 mode, quantised afterwards with moe_quantize_mxfp8). */
 MOE_API int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* prow, const int32_t* counts,
                  const int32_t* poff, void* x_perm, void* stream);
 
@@ -215,27 +219,37 @@ MOE_API int moe_router_wgrad(const moe_config_t* cfg, const void* dlogits, const
  * definitions (the pages only name the format: unite.ai, "Parallelismo, precisione e tecniche di
  * memoria"): per block of 32 elements, scale byte e+127 with e = clamp(floor(log2 amax) - 8, -127,
  * 127) (0 for an all-zero block) and E4M3 codes round-to-nearest-even(x / 2^e) saturated to +-448.
- *   mode MOE_QUANT_ROW: blocks of 32 along a row; q [rows, cols], s [rows, cols/32]; cols % 32 == 0.
- *   mode MOE_QUANT_COL: blocks of 32 down a column; q [rows, cols], s [cols, rows/32];
- *                       rows % 32 == 0, cols % 8 == 0.
- * src 16-byte aligned; q 16-byte (ROW) / 8-byte (COL) aligned. */
+ * Codes q always keep the layout of src. Blocks and scale layouts by mode:
+ *   MOE_QUANT_ROW        blocks along a row;    s [rows, cols/32]                       (cols % 32)
+ *   MOE_QUANT_COL        blocks down a column;  s [cols, rows/32]              (rows % 32, cols % 8)
+ *   MOE_QUANT_ROW_TILED  blocks along a row;    s tiled over (row, block)    (rows, cols % 128)
+ *   MOE_QUANT_COL_TILED  blocks down a column;  s tiled over (column, block) (rows, cols % 128)
+ *   MOE_QUANT_ROW_TILED_GATEUP  as ROW_TILED for stacks of [G gate rows; G up rows] (W13 with
+ *                        G = F), rows remapped so each 64 gate + 64 up rows share chunks (G % 64).
+ * Tiled: the scale of (MN index i, K-block b) -- i = row for ROW modes, column for COL modes -- sits in
+ * 512-byte chunk (i/128, b/4) (chunks of one i/128 consecutive), at byte (i%32)*16 + ((i%128)/32)*4 +
+ * b%4: the layout the MXFP8 grouped GEMM streams. `G` is used by the GATEUP mode only.
+ * src 16-byte aligned; q 16-byte (ROW modes) / 8-byte (COL modes) aligned. */
 #define MOE_QUANT_ROW 0
 #define MOE_QUANT_COL 1
-MOE_API int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode, uint8_t* q,
+#define MOE_QUANT_ROW_TILED 2
+#define MOE_QUANT_COL_TILED 3
+#define MOE_QUANT_ROW_TILED_GATEUP 4
+MOE_API int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode, int64_t G, uint8_t* q,
                                uint8_t* s, void* stream);
 
 /* The grouped GEMM of moe_grouped_gemm with MXFP8 operands (tcgen05 kind::mxf8f6f4.block_scale, fp32
  * accumulation, bf16 outputs). Each operand is E4M3 codes in the layout its bf16 counterpart has in
- * moe_grouped_gemm plus UE8M0 scales along that GEMM's contraction axis:
- *   FWD1_SWIGLU  A = x_perm  ROW [R32,d]          B = W13 ROW [E*2F,d]
- *   FWD2         A = a       ROW [R32,F]          B = W2  ROW [E*d,F]
- *   DGRAD2_SWIGLU A = dy     ROW [R32,d]          B = W2  COL [E*d,F] (scales [F, E*d/32])
- *   DGRAD1       A = dh13    ROW [R32,2F]         B = W13 COL [E*2F,d] (scales [d, E*2F/32])
- *   WGRAD2       A = dy      COL [R32,d]          B = a   COL [R32,F]
- *   WGRAD1       A = dh13    COL [R32,2F]         B = x_perm COL [R32,d]
- * where R32 = moe_max_rows(cfg) (a multiple of 32; rows past the last group are never read by the
- * wgrads; COL scales of activations are [cols, R32/32]). aux (DGRAD2) is the bf16 h13. Requires
- * cfg->dtype == MOE_DTYPE_MXFP8 and d % 128 == 0. */
+ * moe_grouped_gemm plus UE8M0 scales, tiled, along that GEMM's contraction axis:
+ *   FWD1_SWIGLU   A = x_perm ROW_TILED [R,d]     B = W13 ROW_TILED_GATEUP [E*2F,d] (G = F)
+ *   FWD2          A = a      ROW_TILED [R,F]     B = W2  ROW_TILED [E*d,F]
+ *   DGRAD2_SWIGLU A = dy     ROW_TILED [R,d]     B = W2  COL_TILED [E*d,F]
+ *   DGRAD1        A = dh13   ROW_TILED [R,2F]    B = W13 COL_TILED [E*2F,d]
+ *   WGRAD2        A = dy     COL_TILED [R,d]     B = a   COL_TILED [R,F]
+ *   WGRAD1        A = dh13   COL_TILED [R,2F]    B = x_perm COL_TILED [R,d]
+ * with R = moe_max_rows(cfg) (a multiple of 128 in MXFP8 mode; expert groups start on 128-row
+ * boundaries, so the wgrads' contraction blocks never straddle two experts). aux (DGRAD2) is the bf16
+ * h13. Requires cfg->dtype == MOE_DTYPE_MXFP8, d % 128 == 0. */
 MOE_API int moe_grouped_gemm_mxfp8(const moe_config_t* cfg, int op, const uint8_t* Aq, const uint8_t* As,
                                    const uint8_t* Bq, const uint8_t* Bs, void* C, void* C2,
                                    const void* aux, const int32_t* counts, const int32_t* poff,

@@ -95,7 +95,7 @@ def _load():
         "moe_version": ([], ctypes.c_char_p),
         "moe_launch_count": ([], ctypes.c_uint64),
         "moe_route_metadata_noalloc": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp], i),
-        "moe_quantize_mxfp8": ([vp, ctypes.c_int64, i, i, vp, vp, vp], i),
+        "moe_quantize_mxfp8": ([vp, ctypes.c_int64, i, i, ctypes.c_int64, vp, vp, vp], i),
         "moe_grouped_gemm_mxfp8": ([cfgp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i),
         "moe_quantize_weights_mxfp8": ([cfgp, ctypes.POINTER(Weights), ctypes.POINTER(MxWeights), vp], i),
         "moe_layer_fwd_mxfp8": ([cfgp, ctypes.POINTER(Weights), ctypes.POINTER(MxWeights), vp, vp, vp,
@@ -240,14 +240,14 @@ def layer_bwd(cfg, weights: Weights, saved: Saved, x, dout, dx, grads: Grads, ws
           "moe_layer_bwd")
 
 
-QUANT_ROW, QUANT_COL = 0, 1
+QUANT_ROW, QUANT_COL, QUANT_ROW_TILED, QUANT_COL_TILED, QUANT_ROW_TILED_GATEUP = range(5)
 
 
-def quantize_mxfp8(src, q, s, mode, stream=None):
+def quantize_mxfp8(src, q, s, mode, G=0, stream=None):
     """MXFP8 quantisation of a bf16 matrix src [rows, cols] into codes q and scales s."""
     rows, cols = src.shape
-    check(lib.moe_quantize_mxfp8(ptr(src), rows, cols, mode, ptr(q), ptr(s), stream_handle(stream)),
-          "moe_quantize_mxfp8")
+    check(lib.moe_quantize_mxfp8(ptr(src), rows, cols, mode, int(G), ptr(q), ptr(s),
+                                 stream_handle(stream)), "moe_quantize_mxfp8")
 
 
 def grouped_gemm_mxfp8(cfg, op, Aq, As, Bq, Bs, C, C2, aux, counts, poff, ws, stream=None):

@@ -30,14 +30,15 @@ int check_cfg(const moe_config_t* c) {
   if (c->k > c->E) return MOE_ERR_INVALID_ARG;
   if (c->E > 256 || c->k > 8) return MOE_ERR_UNSUPPORTED;
   if (c->d % 64 != 0 || c->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
-  const int64_t rows = (int64_t)c->T * c->k + 31ll * c->E + 31;
+  const int64_t rows = (int64_t)c->T * c->k + 128ll * c->E + 128;
   if (rows >= (1ll << 31) - 256) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
 inline int es_of(const moe_config_t* c) { return c->dtype == MOE_DTYPE_FP32 ? 4 : 2; }
 inline int64_t max_rows_of(const moe_config_t* c) {
-  return ((int64_t)c->T * c->k + 31ll * c->E + 31) / 32 * 32;
+  const int64_t a = group_align(c->dtype);
+  return ((int64_t)c->T * c->k + (a - 1) * c->E + a - 1) / a * a;
 }
 
 struct WsLayout {
@@ -154,38 +155,38 @@ int gemm_op_mx(const moe_config_t* c, int op, const uint8_t* Aq, const uint8_t* 
       a = {Aq, R, d, d};
       b = {Bq, (int64_t)E * 2 * F, d, d};
       p.K = d; p.N = F; p.b_rows_per_group = 2 * F; p.ldc = 2 * F; p.C2 = C2; p.ldc2 = F;
-      p.sA_ld = d / 32; p.a_mn_limit = R; p.sB_ld = d / 32; p.b_mn_limit = (int64_t)E * 2 * F;
+      p.sA_ld = d / 128; p.sB_ld = d / 128;
       return launch_gemm(GK_FWD1_SWIGLU, 1, 128, a, b, p, s);
     case MOE_GEMM_FWD2:
       a = {Aq, R, F, F};
       b = {Bq, (int64_t)E * d, F, F};
       p.K = F; p.N = d; p.b_rows_per_group = d; p.ldc = d;
-      p.sA_ld = F / 32; p.a_mn_limit = R; p.sB_ld = F / 32; p.b_mn_limit = (int64_t)E * d;
+      p.sA_ld = F / 128; p.sB_ld = F / 128;
       return launch_gemm(GK_FWD2, 1, 128, a, b, p, s);
     case MOE_GEMM_DGRAD2_SWIGLU:
       MOE_REQUIRE(aux && aligned16(aux), MOE_ERR_INVALID_ARG);
       a = {Aq, R, d, d};
       b = {Bq, (int64_t)E * d, F, F};
       p.K = d; p.N = F; p.b_rows_per_group = d; p.aux = aux; p.ldaux = 2 * F; p.ldc = 2 * F;
-      p.sA_ld = d / 32; p.a_mn_limit = R; p.sB_ld = (int64_t)E * d / 32; p.b_mn_limit = F;
+      p.sA_ld = d / 128; p.sB_ld = (int64_t)E * d / 128;
       return launch_gemm(GK_DGRAD2_SWIGLU, 1, 128, a, b, p, s);
     case MOE_GEMM_DGRAD1:
       a = {Aq, R, 2 * F, 2 * F};
       b = {Bq, (int64_t)E * 2 * F, d, d};
       p.K = 2 * F; p.N = d; p.b_rows_per_group = 2 * F; p.ldc = d;
-      p.sA_ld = 2 * F / 32; p.a_mn_limit = R; p.sB_ld = (int64_t)E * 2 * F / 32; p.b_mn_limit = d;
+      p.sA_ld = 2 * F / 128; p.sB_ld = (int64_t)E * 2 * F / 128;
       return launch_gemm(GK_DGRAD1, 1, 128, a, b, p, s);
     case MOE_GEMM_WGRAD2:
       a = {Aq, R, d, d};
       b = {Bq, R, F, F};
       p.M = d; p.N = F; p.ldc = F; p.c_group_stride = (int64_t)d * F;
-      p.sA_ld = R / 32; p.a_mn_limit = d; p.sB_ld = R / 32; p.b_mn_limit = F;
+      p.sA_ld = R / 128; p.sB_ld = R / 128;
       return launch_gemm(GK_WGRAD, 1, 128, a, b, p, s);
     case MOE_GEMM_WGRAD1:
       a = {Aq, R, 2 * F, 2 * F};
       b = {Bq, R, d, d};
       p.M = 2 * F; p.N = d; p.ldc = d; p.c_group_stride = (int64_t)2 * F * d;
-      p.sA_ld = R / 32; p.a_mn_limit = 2 * F; p.sB_ld = R / 32; p.b_mn_limit = d;
+      p.sA_ld = R / 128; p.sB_ld = R / 128;
       return launch_gemm(GK_WGRAD, 1, 128, a, b, p, s);
     default:
       return MOE_ERR_INVALID_ARG;
@@ -277,14 +278,13 @@ int moe_route_metadata(const moe_config_t* cfg, const int32_t* idx, int32_t* cou
   MOE_REQUIRE(idx && counts && offsets && poff && perm && prow && row_token, MOE_ERR_INVALID_ARG);
   const WsLayout L = ws_layout(cfg);
   int32_t* hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.hist);
-  return launch_metadata(idx, cfg->T, cfg->E, cfg->k, max_rows_of(cfg), counts, offsets, poff, perm,
-                         prow, row_token, hist, err_of(ws), S(stream));
+  return launch_metadata(idx, cfg->T, cfg->E, cfg->k, group_align(cfg->dtype), max_rows_of(cfg),
+                         counts, offsets, poff, perm, prow, row_token, hist, err_of(ws), S(stream));
 }
 
 int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* prow, const int32_t* counts,
                  const int32_t* poff, void* x_perm, void* stream) {
   MOE_TRY(check_cfg(cfg));
-  MOE_REQUIRE(cfg->dtype != MOE_DTYPE_MXFP8, MOE_ERR_UNSUPPORTED);
   MOE_REQUIRE(x && prow && counts && poff && x_perm, MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(aligned16(x) && aligned16(x_perm), MOE_ERR_INVALID_ARG);
   return launch_dispatch(x, prow, counts, poff, x_perm, cfg->T, cfg->k, cfg->E, cfg->d * es_of(cfg),
@@ -334,19 +334,23 @@ int moe_grouped_gemm(const moe_config_t* cfg, int op, const void* A, const void*
   return gemm_op(cfg, op, A, B, C, C2, aux, counts, poff, ws, S(stream));
 }
 
-int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode, uint8_t* q, uint8_t* s,
-                       void* stream) {
+int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode, int64_t G, uint8_t* q,
+                       uint8_t* s, void* stream) {
   MOE_REQUIRE(src && q && s && rows >= 1 && cols >= 1, MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(aligned16(src), MOE_ERR_INVALID_ARG);
-  if (mode == MOE_QUANT_ROW) {
-    MOE_REQUIRE(cols % 32 == 0 && aligned16(q), MOE_ERR_INVALID_ARG);
-  } else if (mode == MOE_QUANT_COL) {
-    MOE_REQUIRE(rows % 32 == 0 && cols % 8 == 0 && (reinterpret_cast<uintptr_t>(q) & 7u) == 0,
-                MOE_ERR_INVALID_ARG);
-  } else {
-    return MOE_ERR_INVALID_ARG;
+  const bool q16 = aligned16(q), q8 = (reinterpret_cast<uintptr_t>(q) & 7u) == 0;
+  switch (mode) {
+    case MOE_QUANT_ROW: MOE_REQUIRE(cols % 32 == 0 && q16, MOE_ERR_INVALID_ARG); break;
+    case MOE_QUANT_COL: MOE_REQUIRE(rows % 32 == 0 && cols % 8 == 0 && q8, MOE_ERR_INVALID_ARG); break;
+    case MOE_QUANT_ROW_TILED: MOE_REQUIRE(rows % 128 == 0 && cols % 128 == 0 && q16, MOE_ERR_INVALID_ARG); break;
+    case MOE_QUANT_COL_TILED: MOE_REQUIRE(rows % 128 == 0 && cols % 128 == 0 && q8, MOE_ERR_INVALID_ARG); break;
+    case MOE_QUANT_ROW_TILED_GATEUP:
+      MOE_REQUIRE(G >= 64 && G % 64 == 0 && rows % (2 * G) == 0 && cols % 128 == 0 && q16,
+                  MOE_ERR_INVALID_ARG);
+      break;
+    default: return MOE_ERR_INVALID_ARG;
   }
-  return launch_quantize(src, rows, cols, mode, q, s, S(stream));
+  return launch_quantize(src, rows, cols, mode, G, q, s, S(stream));
 }
 
 int moe_grouped_gemm_mxfp8(const moe_config_t* cfg, int op, const uint8_t* Aq, const uint8_t* As,
@@ -396,8 +400,9 @@ int moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* w, const void* x
   }
   const WsLayout L = ws_layout(cfg);
   int32_t* hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.hist);
-  MOE_TRY(launch_metadata(sv->idx, cfg->T, cfg->E, cfg->k, max_rows_of(cfg), sv->counts, sv->offsets,
-                          sv->poff, sv->perm, sv->prow, sv->row_token, hist, err_of(ws), s));
+  MOE_TRY(launch_metadata(sv->idx, cfg->T, cfg->E, cfg->k, group_align(cfg->dtype), max_rows_of(cfg),
+                          sv->counts, sv->offsets, sv->poff, sv->perm, sv->prow, sv->row_token, hist,
+                          err_of(ws), s));
   MOE_TRY(launch_dispatch(x, sv->prow, sv->counts, sv->poff, sv->x_perm, cfg->T, cfg->k, cfg->E,
                           cfg->d * es_of(cfg), s));
   MOE_TRY(gemm_op(cfg, MOE_GEMM_FWD1_SWIGLU, sv->x_perm, w->W13, sv->h13, sv->a, nullptr, sv->counts,
@@ -457,10 +462,11 @@ int moe_quantize_weights_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
               MOE_ERR_INVALID_ARG);
   const int64_t E = cfg->E, d = cfg->d, F = cfg->F;
   cudaStream_t s = S(stream);
-  MOE_TRY(moe_quantize_mxfp8(w->W13, E * 2 * F, (int)d, MOE_QUANT_ROW, qw->W13q, qw->W13s, s));
-  MOE_TRY(moe_quantize_mxfp8(w->W13, E * 2 * F, (int)d, MOE_QUANT_COL, qw->W13tq, qw->W13ts, s));
-  MOE_TRY(moe_quantize_mxfp8(w->W2, E * d, (int)F, MOE_QUANT_ROW, qw->W2q, qw->W2s, s));
-  return moe_quantize_mxfp8(w->W2, E * d, (int)F, MOE_QUANT_COL, qw->W2tq, qw->W2ts, s);
+  MOE_TRY(moe_quantize_mxfp8(w->W13, E * 2 * F, (int)d, MOE_QUANT_ROW_TILED_GATEUP, F, qw->W13q,
+                             qw->W13s, s));
+  MOE_TRY(moe_quantize_mxfp8(w->W13, E * 2 * F, (int)d, MOE_QUANT_COL_TILED, 0, qw->W13tq, qw->W13ts, s));
+  MOE_TRY(moe_quantize_mxfp8(w->W2, E * d, (int)F, MOE_QUANT_ROW_TILED, 0, qw->W2q, qw->W2s, s));
+  return moe_quantize_mxfp8(w->W2, E * d, (int)F, MOE_QUANT_COL_TILED, 0, qw->W2tq, qw->W2ts, s);
 }
 
 int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const moe_mxfp8_weights_t* qw,
@@ -491,14 +497,15 @@ int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
   }
   const WsLayout L = ws_layout(cfg);
   int32_t* hist = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.hist);
-  MOE_TRY(launch_metadata(sv->idx, cfg->T, cfg->E, cfg->k, R, sv->counts, sv->offsets, sv->poff,
-                          sv->perm, sv->prow, sv->row_token, hist, err_of(ws), s));
+  MOE_TRY(launch_metadata(sv->idx, cfg->T, cfg->E, cfg->k, group_align(cfg->dtype), R, sv->counts,
+                          sv->offsets, sv->poff, sv->perm, sv->prow, sv->row_token, hist, err_of(ws),
+                          s));
   MOE_TRY(launch_dispatch(x, sv->prow, sv->counts, sv->poff, sv->x_perm, cfg->T, cfg->k, cfg->E, d * 2,
                           s));
-  MOE_TRY(launch_quantize(sv->x_perm, R, d, MOE_QUANT_ROW, qa->xq, qa->xs, s));
+  MOE_TRY(launch_quantize(sv->x_perm, R, d, MOE_QUANT_ROW_TILED, 0, qa->xq, qa->xs, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_FWD1_SWIGLU, qa->xq, qa->xs, qw->W13q, qw->W13s, sv->h13, sv->a,
                      nullptr, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize(sv->a, R, F, MOE_QUANT_ROW, qa->aq, qa->as, s));
+  MOE_TRY(launch_quantize(sv->a, R, F, MOE_QUANT_ROW_TILED, 0, qa->aq, qa->as, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_FWD2, qa->aq, qa->as, qw->W2q, qw->W2s, sv->y, nullptr, nullptr,
                      sv->counts, sv->poff, ws, s));
   return launch_combine(sv->y, sv->gates, sv->prow, out, cfg->T, cfg->k, d * 2, true, s);
@@ -536,18 +543,18 @@ int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
   void* dlog = router ? static_cast<void*>(static_cast<char*>(ws) + L.dlogits) : nullptr;
   MOE_TRY(launch_combine_bwd(dout, sv->y, sv->gates, sv->prow, sv->idx, sv->counts, sv->poff, g->dy,
                              g->dgates, dlsel, dlog, cfg->T, cfg->k, cfg->E, d * 2, true, s));
-  MOE_TRY(launch_quantize(g->dy, R, d, MOE_QUANT_ROW, qa->dyq, qa->dys, s));
+  MOE_TRY(launch_quantize(g->dy, R, d, MOE_QUANT_ROW_TILED, 0, qa->dyq, qa->dys, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_DGRAD2_SWIGLU, qa->dyq, qa->dys, qw->W2tq, qw->W2ts, g->dh13,
                      nullptr, sv->h13, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize(g->dy, R, d, MOE_QUANT_COL, qa->dytq, qa->dyts, s));
-  MOE_TRY(launch_quantize(sv->a, R, F, MOE_QUANT_COL, qa->atq, qa->ats, s));
+  MOE_TRY(launch_quantize(g->dy, R, d, MOE_QUANT_COL_TILED, 0, qa->dytq, qa->dyts, s));
+  MOE_TRY(launch_quantize(sv->a, R, F, MOE_QUANT_COL_TILED, 0, qa->atq, qa->ats, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD2, qa->dytq, qa->dyts, qa->atq, qa->ats, g->dW2, nullptr,
                      nullptr, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize(g->dh13, R, 2 * F, MOE_QUANT_ROW, qa->dhq, qa->dhs, s));
+  MOE_TRY(launch_quantize(g->dh13, R, 2 * F, MOE_QUANT_ROW_TILED, 0, qa->dhq, qa->dhs, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_DGRAD1, qa->dhq, qa->dhs, qw->W13tq, qw->W13ts, g->dx_perm, nullptr,
                      nullptr, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize(g->dh13, R, 2 * F, MOE_QUANT_COL, qa->dhtq, qa->dhts, s));
-  MOE_TRY(launch_quantize(sv->x_perm, R, d, MOE_QUANT_COL, qa->xtq, qa->xts, s));
+  MOE_TRY(launch_quantize(g->dh13, R, 2 * F, MOE_QUANT_COL_TILED, 0, qa->dhtq, qa->dhts, s));
+  MOE_TRY(launch_quantize(sv->x_perm, R, d, MOE_QUANT_COL_TILED, 0, qa->xtq, qa->xts, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD1, qa->dhtq, qa->dhts, qa->xtq, qa->xts, g->dW13, nullptr,
                      nullptr, sv->counts, sv->poff, ws, s));
   MOE_TRY(launch_token_reduce(g->dx_perm, sv->prow, dlsel, router ? sv->idx : nullptr, w->W_r, dx,

@@ -46,7 +46,7 @@ struct Cfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   // output staging: each epilogue warp owns NBUF swizzled 32-row x 128-byte boxes
   static constexpr bool MX = (ES == 1);      // MXFP8 block-scaled (E4M3 operands, UE8M0 scales)
-  static constexpr int THREADS = MX ? kThreads + 32 : kThreads;  // + scale-loader warp
+  static constexpr int THREADS = kThreads;
   static constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : (MX ? 2 : ES);  // output element size
   static constexpr int OEPR = 128 / OES;     // output columns per staged box
   static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3 : 2;
@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], C::MX ? 2 : 1);  // TMA bytes (+ the scale loader's arrival)
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -310,9 +310,42 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
           }
           uint8_t* a_dst = smA + (size_t)s * C::A_BYTES;
           uint8_t* b_dst = smB + (size_t)s * C::B_BYTES;
+          const uint8_t* sf_a = nullptr;
+          const uint8_t* sf_b = nullptr;
+          uint8_t* sf_dst = nullptr;
+          if constexpr (C::MX) {
+            // this stage's scales: one 512-byte chunk for the 128 rows of A, one per 128 of B
+            uint8_t* sf = sfs + (size_t)s * C::SF_BYTES;
+            int64_t amb, akq, bmb, bkq;
+            if constexpr (MODE == GROUP_M) {
+              amb = ((int64_t)ti.row_base + ti.m0) >> 7;
+              akq = ks;
+              if constexpr (B_MN) {
+                bmb = ti.n0 >> 7;
+                bkq = (int64_t)ti.e * (p.b_rows_per_group >> 7) + ks;
+              } else if constexpr (EPI == EPI_SWIGLU_FWD) {
+                bmb = (int64_t)ti.e * (p.b_rows_per_group >> 7) + ti.n0 / (BN / 2);
+                bkq = ks;
+              } else {
+                bmb = ((int64_t)ti.e * p.b_rows_per_group + ti.n0) >> 7;
+                bkq = ks;
+              }
+            } else {
+              amb = ti.m0 >> 7;
+              bmb = ti.n0 >> 7;
+              akq = bkq = (ti.kstart >> 7) + ks;
+            }
+            sf_a = p.sA + (amb * p.sA_ld + akq) * 512;
+            sf_b = p.sB + (bmb * p.sB_ld + bkq) * 512;
+            sf_dst = sf;
+          }
           if constexpr (MODE == GROUP_M) {
             const int k0 = ks * C::BK;
-            mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+            mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES + C::SF_BYTES);
+            if constexpr (C::MX) {
+              bulk_load(sf_dst, sf_a, 512, &full[s]);
+              bulk_load(sf_dst + 512, sf_b, 512, &full[s]);
+            }
             // A: K-major rows of the routed buffer (or the token matrix)
             tma_load_2d(a_dst, &tmA, &full[s], k0, ti.row_base + ti.m0);
             if constexpr (!B_MN) {
@@ -337,7 +370,11 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
             // GROUP_K: both operands MN-major, contraction rows kstart + 32*chunk
             const int c0 = ks * C::CHUNKS;
             const int nch = min(C::CHUNKS, ti.nchunks - c0);
-            mbar_arrive_expect_tx(&full[s], nch * 32 * 128 * ((BM + BN) / C::EPR));
+            mbar_arrive_expect_tx(&full[s], nch * 32 * 128 * ((BM + BN) / C::EPR) + C::SF_BYTES);
+            if constexpr (C::MX) {
+              bulk_load(sf_dst, sf_a, 512, &full[s]);
+              bulk_load(sf_dst + 512, sf_b, 512, &full[s]);
+            }
             for (int ch = 0; ch < nch; ++ch) {
               const int krow = ti.kstart + (c0 + ch) * 32;
 #pragma unroll
@@ -420,89 +457,6 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
         umma_commit(done);
         mbar_wait_bounded(done, 0, p.wait_limit_ns, nullptr, p.err);
       }
-    }
-  } else if (C::MX && warp == 6) {
-    // ===================== MXFP8 scale loader (warp 6) =====================
-    // For every stage, lane L assembles smem row L of each 512-byte scale chunk: the 4 K-block
-    // scales of rows L, L+32, L+64, L+96 (4 bytes each), the layout tcgen05.cp spreads over TMEM.
-    int it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      TileInfo ti;
-      tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
-      const int nst = num_kstages<C, MODE>(ti);
-      bool ok = true;
-      for (int ks = 0; ks < nst; ++ks, ++it) {
-        const int s = it % C::STAGES;
-        int w = 1;
-        if (lane == 0)
-          w = mbar_wait_bounded(&empty[s], ((it / C::STAGES) & 1) ^ 1, p.wait_limit_ns, abort_word,
-                                p.err);
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (!w) {
-          ok = false;
-          break;
-        }
-        int64_t kb0;   // first K-block of this stage (global K-block index of the scale arrays)
-        int nkb = 4;   // valid K-blocks in this stage
-        if constexpr (MODE == GROUP_M) {
-          kb0 = ks * 4;
-        } else {
-          kb0 = ti.kstart / 32 + ks * 4;
-          nkb = min(4, ti.nchunks - ks * 4);
-        }
-        uint8_t* sfa = sfs + (size_t)s * C::SF_BYTES;
-        // A: rows of the accumulator
-        {
-          uint32_t wv[4];
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            const int r = lane + 32 * qq;
-            int64_t mn, kb = kb0;
-            if constexpr (MODE == GROUP_M) mn = (int64_t)ti.row_base + ti.m0 + r;
-            else mn = (int64_t)ti.m0 + r;
-            uint32_t v = 0;
-            if (mn < p.a_mn_limit) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                if (j < nkb) v |= (uint32_t)p.sA[mn * p.sA_ld + kb + j] << (8 * j);
-            }
-            wv[qq] = v;
-          }
-          st_shared_v4(sfa + lane * 16, make_uint4(wv[0], wv[1], wv[2], wv[3]));
-        }
-        // B: columns of the accumulator, 128 per chunk
-#pragma unroll
-        for (int c = 0; c < BN / 128; ++c) {
-          uint32_t wv[4];
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            const int n = 128 * c + lane + 32 * qq;
-            int64_t mn, kb = kb0;
-            if constexpr (MODE == GROUP_K) {
-              mn = (int64_t)ti.n0 + n;
-            } else if constexpr (B_MN) {
-              mn = (int64_t)ti.n0 + n;
-              kb = (int64_t)ti.e * (p.b_rows_per_group / 32) + kb0;
-            } else if constexpr (EPI == EPI_SWIGLU_FWD) {
-              mn = (int64_t)ti.e * p.b_rows_per_group + (n < BN / 2 ? ti.n0 + n : p.F + ti.n0 + n - BN / 2);
-            } else {
-              mn = (int64_t)ti.e * p.b_rows_per_group + ti.n0 + n;
-            }
-            uint32_t v = 0;
-            if (mn < p.b_mn_limit) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                if (j < nkb) v |= (uint32_t)p.sB[mn * p.sB_ld + kb + j] << (8 * j);
-            }
-            wv[qq] = v;
-          }
-          st_shared_v4(sfa + 512 * (1 + c) + lane * 16, make_uint4(wv[0], wv[1], wv[2], wv[3]));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[s]);
-      }
-      if (!ok) break;
     }
   } else if (warp >= 2 && warp < 6) {
     // ===================== epilogue (warps 2..5) =====================

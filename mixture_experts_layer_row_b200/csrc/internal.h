@@ -35,11 +35,11 @@ struct GemmParams {
   int F;
   int64_t c_group_stride;  // GROUP_K: elements between two groups' outputs
   int vec_ok;              // output rows allow 16-byte vector stores
-  // MXFP8 operands: UE8M0 scale of (MN index i, 32-element K-block b) at s[i * s_ld + b]
+  // MXFP8 operands: UE8M0 scales in the tiled layout (512-byte chunks per 128 MN indices x 4
+  // K-blocks); sA_ld / sB_ld = chunks per 128 MN indices (= K-blocks / 4 of that operand)
   const uint8_t* sA;
   const uint8_t* sB;
   int64_t sA_ld, sB_ld;
-  int64_t a_mn_limit, b_mn_limit;  // valid MN indices of each operand's scales
   uint32_t* err;
   uint64_t wait_limit_ns;
 };
@@ -56,15 +56,17 @@ int sm_count();
 
 int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
                 const GemmParams& p, cudaStream_t s);
-int launch_quantize(const void* src, int64_t rows, int cols, int mode, uint8_t* q, uint8_t* s,
-                    cudaStream_t st);
+int launch_quantize(const void* src, int64_t rows, int cols, int mode, int64_t G, uint8_t* q,
+                    uint8_t* s, cudaStream_t st);
 int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s);
 
 int launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm, int32_t* idx,
                 float* gates, uint32_t* err, cudaStream_t s);
 size_t metadata_ws_bytes(int T, int E);
-int launch_metadata(const int32_t* idx, int T, int E, int k, int64_t max_rows, int32_t* counts,
-                    int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
+// Group alignment of the routed-row buffers: 32 rows, 128 in MXFP8 mode (whole 128-row scale chunks).
+inline int group_align(int dtype) { return dtype == MOE_DTYPE_MXFP8 ? 128 : 32; }
+int launch_metadata(const int32_t* idx, int T, int E, int k, int align, int64_t max_rows,
+                    int32_t* counts, int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
                     int32_t* row_token, int32_t* hist_ws, uint32_t* err, cudaStream_t s);
 
 int launch_dispatch(const void* x, const int32_t* prow, const int32_t* counts, const int32_t* poff,

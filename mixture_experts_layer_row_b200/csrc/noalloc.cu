@@ -59,7 +59,7 @@ extern "C" MOE_API int moe_route_metadata_noalloc(const moe_config_t* cfg, const
   if (rc != MOE_OK) return rc;
   // Device-side routing errors are not reported by this variant (there is no workspace flag);
   // invalid expert ids are still skipped by the kernels.
-  return moe::launch_metadata(idx, cfg->T, cfg->E, cfg->k, moe_max_rows(cfg), counts, offsets, poff,
-                              perm, prow, row_token, hist, nullptr,
-                              reinterpret_cast<cudaStream_t>(stream));
+  return moe::launch_metadata(idx, cfg->T, cfg->E, cfg->k, moe::group_align(cfg->dtype),
+                              moe_max_rows(cfg), counts, offsets, poff, perm, prow, row_token, hist,
+                              nullptr, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -8,9 +8,17 @@
 // floor(log2) is read from the fp32 exponent bits (exact, subnormals included); the scaling by a power
 // of two is exact in fp32, and the conversion is the hardware's cvt.rn.satfinite.e4m3x2.f32.
 //
-// Two layouts, both HBM-bound streaming kernels with 16-byte loads:
-//   ROW  blocks of 32 consecutive elements of a row: codes [rows, cols], scales [rows, cols/32]
-//   COL  blocks of 32 consecutive rows of a column:  codes [rows, cols], scales [cols, rows/32]
+// Blocks run along rows (ROW: 32 consecutive elements of a row) or down columns (COL: 32 consecutive
+// rows of a column); codes keep the source layout [rows, cols]. Scale layouts:
+//   plain  ROW [rows, cols/32], COL [cols, rows/32];
+//   tiled  the layout the MXFP8 grouped GEMM streams: for the scale of (MN index i, K-block b), with
+//          i = row (ROW) or column (COL), 512-byte chunks per (128 MN indices, 4 K-blocks) at chunk
+//          (i/128, b/4), byte (i%32)*16 + ((i%128)/32)*4 + b%4 inside -- exactly the rows that
+//          tcgen05.cp 32x128b.warpx4 spreads over the four TMEM lane quadrants;
+//   tiled gate/up  like tiled ROW for a stack of [gate; up] blocks of 2*G rows each, with the MN
+//          index of row f of gate (up) remapped to 128*(f/64) + f%64 (+64), so that the 64 gate and
+//          64 up rows of one fused GEMM1 tile share one chunk.
+// Both kernels are HBM-bound streams with 16-byte loads.
 #include "internal.h"
 
 namespace moe {
@@ -48,8 +56,23 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Byte offset of the scale of (MN index i, K-block b) in the tiled layout with KB K-blocks per MN index.
+__device__ __forceinline__ int64_t tiled_sf_offset(int64_t i, int64_t b, int64_t KB) {
+  return ((i >> 7) * (KB >> 2) + (b >> 2)) * 512 + (i & 31) * 16 + ((i >> 5) & 3) * 4 + (b & 3);
+}
+
+__device__ __forceinline__ int64_t scale_index(int layout, int64_t i, int64_t b, int64_t KB, int64_t G) {
+  if (layout == 0) return i * KB + b;  // plain
+  if (layout == 2) {                   // tiled gate/up: remap the row inside its [gate; up] stack
+    const int64_t e = i / (2 * G), rr = i % (2 * G), f = rr % G, up = rr / G;
+    i = e * 2 * G + (f / 64) * 128 + up * 64 + f % 64;
+  }
+  return tiled_sf_offset(i, b, KB);
+}
+
 __global__ void __launch_bounds__(256) quant_row_kernel(const uint4* __restrict__ src, int64_t nblocks,
-                                                        int blocks_per_row, uint4* __restrict__ q,
+                                                        int blocks_per_row, int layout, int64_t G,
+                                                        uint4* __restrict__ q,
                                                         uint8_t* __restrict__ s) {
   const int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= nblocks) return;
@@ -81,13 +104,12 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const uint4* __restrict_
   }
   q[b * 2] = make_uint4(c[0], c[1], c[2], c[3]);
   q[b * 2 + 1] = make_uint4(c[4], c[5], c[6], c[7]);
-  s[b] = sb;
-  (void)blocks_per_row;
+  s[scale_index(layout, b / blocks_per_row, b % blocks_per_row, blocks_per_row, G)] = sb;
 }
 
 // One thread per (32-row block, 8 consecutive columns).
 __global__ void __launch_bounds__(256) quant_col_kernel(const uint4* __restrict__ src, int64_t rows,
-                                                        int cols, uint2* __restrict__ q,
+                                                        int cols, int layout, uint2* __restrict__ q,
                                                         uint8_t* __restrict__ s) {
   const int groups = cols / 8;
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -115,7 +137,7 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const uint4* __restrict_
     uint8_t sb;
     const int e = block_exponent(amax[j], &sb);
     inv[j] = amax[j] > 0.f ? exp2_exact(-e) : 0.f;
-    s[(int64_t)(cg * 8 + j) * rblocks + rb] = sb;
+    s[scale_index(layout, (int64_t)cg * 8 + j, rb, rblocks, 0)] = sb;
   }
   uint2* qb = q + (rb * 32) * groups + cg;
 #pragma unroll 4
@@ -136,18 +158,24 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const uint4* __restrict_
 
 }  // namespace
 
-int launch_quantize(const void* src, int64_t rows, int cols, int mode, uint8_t* q, uint8_t* s,
-                    cudaStream_t st) {
-  if (mode == 0) {
+// mode: MOE_QUANT_ROW / COL / ROW_TILED / COL_TILED / ROW_TILED_GATEUP (G = gate rows per stack)
+int launch_quantize(const void* src, int64_t rows, int cols, int mode, int64_t G, uint8_t* q,
+                    uint8_t* s, cudaStream_t st) {
+  const bool row = mode == MOE_QUANT_ROW || mode == MOE_QUANT_ROW_TILED ||
+                   mode == MOE_QUANT_ROW_TILED_GATEUP;
+  const int layout = (mode == MOE_QUANT_ROW || mode == MOE_QUANT_COL) ? 0
+                     : (mode == MOE_QUANT_ROW_TILED_GATEUP)           ? 2
+                                                                       : 1;
+  if (row) {
     const int64_t nb = rows * (cols / 32);
     const int64_t grid = (nb + 255) / 256;
     quant_row_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const uint4*>(src), nb, cols / 32,
-                                                      reinterpret_cast<uint4*>(q), s);
+                                                      layout, G, reinterpret_cast<uint4*>(q), s);
   } else {
     const int64_t nt = (rows / 32) * (cols / 8);
     const int64_t grid = (nt + 255) / 256;
     quant_col_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const uint4*>(src), rows, cols,
-                                                      reinterpret_cast<uint2*>(q), s);
+                                                      layout, reinterpret_cast<uint2*>(q), s);
   }
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

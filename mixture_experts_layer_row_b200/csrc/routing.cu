@@ -8,7 +8,7 @@
 // Metadata: three small kernels over chunks of 256 tokens:
 //   1. per-chunk expert histogram (shared-memory counters; counts do not depend on arrival order);
 //   2. one CTA turns the histograms into per-chunk bases (exclusive scan over chunks), counts,
-//      offsets and 32-aligned padded offsets (exclusive scans over experts), checks sum = T*k;
+//      offsets and aligned padded offsets (exclusive scans over experts), checks sum = T*k;
 //   3. per chunk, the stable rank of every entry inside its expert: within a warp by
 //      __match_any_sync + popc of the lower lanes, across warps and chunks by the scanned bases.
 //      The order is ascending (token, slot): deterministic, no atomics decide it.
@@ -152,7 +152,7 @@ __device__ int block_exclusive_scan_256(int val, int* smem_warp, int* total) {
 }
 
 __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ hist, int nchunks, int T,
-                                                   int E, int k, int64_t max_rows,
+                                                   int E, int k, int align, int64_t max_rows,
                                                    int32_t* __restrict__ counts,
                                                    int32_t* __restrict__ offsets,
                                                    int32_t* __restrict__ poff,
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ hist, i
     }
   }
   const int cnt = e < E ? run : 0;
-  const int pcnt = (cnt + 31) & ~31;
+  const int pcnt = (cnt + align - 1) / align * align;
   int tot, ptot;
   const int off = block_exclusive_scan_256(cnt, sw, &tot);
   const int poffe = block_exclusive_scan_256(pcnt, sw, &ptot);
@@ -275,12 +275,12 @@ size_t metadata_ws_bytes(int T, int E) {
   return nchunks * E * sizeof(int32_t);
 }
 
-int launch_metadata(const int32_t* idx, int T, int E, int k, int64_t max_rows, int32_t* counts,
-                    int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
+int launch_metadata(const int32_t* idx, int T, int E, int k, int align, int64_t max_rows,
+                    int32_t* counts, int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
                     int32_t* row_token, int32_t* hist_ws, uint32_t* err, cudaStream_t s) {
   const int nchunks = (T + kChunk - 1) / kChunk;
   hist_kernel<<<nchunks, kChunk, 0, s>>>(idx, T, E, k, hist_ws, err);
-  scan_kernel<<<1, 256, 0, s>>>(hist_ws, nchunks, T, E, k, max_rows, counts, offsets, poff,
+  scan_kernel<<<1, 256, 0, s>>>(hist_ws, nchunks, T, E, k, align, max_rows, counts, offsets, poff,
                                 row_token, err);
   rank_kernel<<<nchunks, kChunk, 0, s>>>(idx, T, E, k, hist_ws, offsets, poff, perm, prow, row_token);
   count_launches(3);

@@ -99,5 +99,11 @@ def test_host_validation_before_any_launch(L):
                                   10 ** 9, None) == -1  # SwiGLU forward needs its second output
     assert L.lib.moe_get_error(None, None, None) == -1
     mx = L.make_config(64, 64, 128, 8, 2, L.DTYPE_MXFP8)
-    assert L.lib.moe_dispatch(ctypes.byref(mx), fake, fake, fake, fake, fake, None) == -2
+    # the router GEMM and the bf16/fp32 grouped GEMM entry points do not take MXFP8 configs
+    assert L.lib.moe_router_logits(ctypes.byref(mx), fake, fake, None, fake, fake, 10 ** 9, None) == -2
+    assert L.lib.moe_grouped_gemm(ctypes.byref(mx), 1, fake, fake, fake, None, None, fake, fake, fake,
+                                  10 ** 9, None) == -2
+    # and the MXFP8 grouped GEMM needs d % 128 == 0
+    assert L.lib.moe_grouped_gemm_mxfp8(ctypes.byref(mx), 1, fake, fake, fake, fake, fake, None, None,
+                                        fake, fake, fake, 10 ** 9, None) == -2
     assert L.lib.moe_layer_fwd(c, None, fake, None, fake, None, fake, 10 ** 9, None) == -1

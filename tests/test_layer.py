@@ -52,7 +52,7 @@ def _routing_checks(w, layer, inp, x64, Wr64):
     else:
         idx = inp["idx"].cpu().numpy().astype(np.int64)
         gates_ref = np64(inp["gates"])
-    meta = O.route_metadata(idx, w.E)
+    meta = O.route_metadata(idx, w.E, 128 if w.dtype == "mxfp8" else 32)  # MXFP8 groups: 128 rows
     for key in ("counts", "offsets", "poff", "perm", "prow"):
         assert np.array_equal(getattr(layer, key).cpu().numpy(), meta[key]), key
     used = int(meta["poff"][-1])

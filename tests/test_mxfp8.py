@@ -1,7 +1,8 @@
 """MXFP8 on the GPU: quantisation must be bit-exact with the oracle's OCP-MX quantiser (codes and
-scales), and every block-scaled grouped GEMM op must match the oracle's GEMM step applied to the
-oracle's own MXFP8 fake-quantised operands (exact products of E4M3 codes and power-of-two scales, so
-only fp32 accumulation order and the bf16 output rounding differ)."""
+scales, in the plain and in the tiled scale layouts), and every block-scaled grouped GEMM op must
+match the oracle's GEMM step applied to the oracle's own MXFP8 fake-quantised operands (exact products
+of E4M3 codes and power-of-two scales, so only fp32 accumulation order and the bf16 output rounding
+differ)."""
 import numpy as np
 import pytest
 import torch
@@ -54,6 +55,44 @@ def test_quantize_col_bitexact(rows, cols):
     assert np.array_equal(q.cpu().numpy(), rq)
 
 
+def tiled(plain, gateup_G=0):
+    """Re-index plain scales [MN, KB] into the tiled layout the GEMM streams: chunk (i/128, b/4) of 512
+    bytes, byte (i%32)*16 + ((i%128)/32)*4 + b%4 (rows of [gate; up] stacks remapped for GATEUP)."""
+    MN, KB = plain.shape
+    out = np.zeros(MN * KB, dtype=np.uint8)
+    i = np.arange(MN)[:, None]
+    b = np.arange(KB)[None, :]
+    if gateup_G:
+        G = gateup_G
+        e, rr = i // (2 * G), i % (2 * G)
+        f, up = rr % G, rr // G
+        i = e * 2 * G + (f // 64) * 128 + up * 64 + f % 64
+    off = ((i // 128) * (KB // 4) + b // 4) * 512 + (i % 32) * 16 + ((i % 128) // 32) * 4 + b % 4
+    out[off.reshape(-1)] = plain.reshape(-1)
+    return out
+
+
+@pytest.mark.parametrize("rows,cols,mode", [(128, 128, "row"), (256, 384, "col"), (1024, 2048, "row"),
+                                            (2048, 1536, "col"), (1536, 256, "gateup")])
+def test_quantize_tiled_bitexact(rows, cols, mode):
+    L = _lib()
+    x = _bf16_matrix(rows, cols, 5 * rows + cols)
+    q = torch.zeros((rows, cols), dtype=torch.uint8, device=dev())
+    s = torch.zeros(rows * cols // 32, dtype=torch.uint8, device=dev())
+    m = {"row": L.QUANT_ROW_TILED, "col": L.QUANT_COL_TILED, "gateup": L.QUANT_ROW_TILED_GATEUP}[mode]
+    G = 384 if mode == "gateup" else 0   # two [384 gate; 384 up] stacks
+    L.quantize_mxfp8(x.to(dev()), q, s, m, G)
+    torch.cuda.synchronize()
+    if mode == "col":
+        rq, rs = MX.quantize_cols(x.double().numpy())
+        ref_s = tiled(rs.T)
+    else:
+        rq, rs = MX.quantize_rows(x.double().numpy())
+        ref_s = tiled(rs, G)
+    assert np.array_equal(q.cpu().numpy(), rq)
+    assert np.array_equal(s.cpu().numpy(), ref_s)
+
+
 SHAPES = {
     "ragged": (512, 128, 256, 8, 2, [0, 1, 31, 33, 129, 200, 300, 330]),
     "one_expert": (300, 128, 128, 4, 1, [300, 0, 0, 0]),
@@ -69,9 +108,9 @@ class MxProblem:
         self.T, self.d, self.F, self.E, self.k = T, d, F, E, k
         rng = np.random.default_rng(seed)
         idx = np.argsort(rng.random((T, E)), 1)[:, :k] if counts is None else idx_from_counts(counts, T, k, rng)
-        self.meta = O.route_metadata(idx.astype(np.int64), E)
+        self.meta = O.route_metadata(idx.astype(np.int64), E, 128)  # MXFP8 groups: 128 rows
         self.cfg = L.make_config(T, d, F, E, k, L.DTYPE_MXFP8)
-        self.R32 = (L.max_rows(self.cfg) + 31) // 32 * 32
+        self.R32 = L.max_rows(self.cfg)
         self.ws = torch.zeros(L.workspace_size(self.cfg), dtype=torch.uint8, device=dev())
         self.g = torch.Generator().manual_seed(seed + 1)
         t32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).to(dev())
@@ -89,12 +128,13 @@ class MxProblem:
     def weights(self, *shape):
         return (torch.randn(shape, generator=self.g) * 0.05).to(torch.bfloat16)
 
-    def quant(self, x2d, mode):
+    def quant(self, x2d, mode, G=0):
+        """mode 0: ROW (tiled scales), 1: COL (tiled), 2: ROW gate/up tiled (W13, G = F)."""
         rows, cols = x2d.shape
         q = torch.zeros((rows, cols), dtype=torch.uint8, device=dev())
-        s = torch.zeros((rows, cols // 32) if mode == 0 else (cols, rows // 32), dtype=torch.uint8,
-                        device=dev())
-        self.L.quantize_mxfp8(x2d.to(dev()).contiguous(), q, s, mode)
+        s = torch.zeros(rows * cols // 32, dtype=torch.uint8, device=dev())
+        m = [self.L.QUANT_ROW_TILED, self.L.QUANT_COL_TILED, self.L.QUANT_ROW_TILED_GATEUP][mode]
+        self.L.quantize_mxfp8(x2d.to(dev()).contiguous(), q, s, m, G)
         return q, s
 
     def groups(self):
@@ -119,7 +159,7 @@ ROWQ, COLQ = O._mx_row, O._mx_col
 def test_mx_fwd1(shape):
     P = MxProblem(shape)
     X, W13 = P.rows(P.d), P.weights(P.E, 2 * P.F, P.d)
-    h13, a = P.run(P.L.GEMM_FWD1_SWIGLU, P.quant(X, 0), P.quant(W13.reshape(-1, P.d), 0),
+    h13, a = P.run(P.L.GEMM_FWD1_SWIGLU, P.quant(X, 0), P.quant(W13.reshape(-1, P.d), 2, P.F),
                    torch.zeros((P.R32, 2 * P.F), dtype=torch.bfloat16),
                    torch.zeros((P.R32, P.F), dtype=torch.bfloat16))
     Xn, Wn, H, A = np64(X), np64(W13), np64(h13), np64(a)
