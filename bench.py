@@ -30,6 +30,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
                   "source": "fallback"}
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The slowest rank's value (the job's time): all-reduce MAX over the process group, if any."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -277,39 +288,49 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def cpu_baseline_experts(w, inp, n_experts, label):
-    """The fp64 oracle's per-expert forward + backward (MXFP8 emulated when the workload is MXFP8) on
-    every routed row of the first n_experts experts; for workloads whose fp64 weights do not fit the
-    host comfortably. Throughput = processed routed rows / k per second."""
-    import numpy as np
-    import torch
-    from oracle import moe as O
-    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
-    mx = w.dtype == "mxfp8"
-    idx = inp["idx"].cpu().numpy().astype(np.int64)
-    gates = f64(inp["gates"])
-    x = f64(inp["x"])
-    dout = f64(inp["dout"])
-    rows = 0
-    t0 = time.perf_counter()
-    for e in range(n_experts):
-        tj = np.argwhere(idx == e)
-        X = x[tj[:, 0]]
-        dY = gates[tj[:, 0], tj[:, 1]][:, None] * dout[tj[:, 0]]
-        W13e, W2e = f64(inp["W13"][e]), f64(inp["W2"][e])
-        h13, a, y = O.expert_fwd(X, W13e, W2e, mx)
-        O.expert_bwd(X, W13e, W2e, h13, a, dY, mx)
-        rows += len(tj)
-    dt = time.perf_counter() - t0
+class ExpertSample:
+    """The fp64 oracle's per-expert forward + backward (MXFP8-emulated for the MXFP8 workload) over
+    every routed row of a subset of experts. The experts' weights are converted to fp64 once, outside
+    the timed region. Throughput = processed routed rows / k per second."""
+
+    def __init__(self, w, inp, n_experts):
+        import numpy as np
+        import torch
+        f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+        self.w, self.mx = w, w.dtype == "mxfp8"
+        idx = inp["idx"].cpu().numpy().astype(np.int64)
+        gates, x, dout = f64(inp["gates"]), f64(inp["x"]), f64(inp["dout"])
+        self.work = []
+        for e in range(n_experts):
+            tj = np.argwhere(idx == e)
+            self.work.append((x[tj[:, 0]], gates[tj[:, 0], tj[:, 1]][:, None] * dout[tj[:, 0]],
+                              f64(inp["W13"][e]), f64(inp["W2"][e])))
+        self.rows = sum(len(wk[0]) for wk in self.work)
+
+    def run(self):
+        from oracle import moe as O
+        t0 = time.perf_counter()
+        for X, dY, W13e, W2e in self.work:
+            h13, a, _ = O.expert_fwd(X, W13e, W2e, self.mx)
+            O.expert_bwd(X, W13e, W2e, h13, a, dY, self.mx)
+        return time.perf_counter() - t0
+
+
+def blas_threads():
     try:
         from threadpoolctl import threadpool_info
-        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+        return max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
     except Exception:
-        cores = 1
-    return {"value": rows / w.k / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{label}: experts 0..{n_experts - 1}, all {rows} of their routed rows "
-                      f"({'MXFP8-emulated ' if mx else ''}fp64 per-expert forward + backward incl. "
-                      f"weight conversion), {dt:.1f} s; tokens/s = rows / k / s"}
+        return 1
+
+
+def cpu_baseline_experts(w, inp, n_experts, label):
+    smp = ExpertSample(w, inp, n_experts)
+    dt = smp.run()
+    return {"value": smp.rows / w.k / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{label}: experts 0..{n_experts - 1}, all {smp.rows} of their routed rows "
+                      f"({'MXFP8-emulated ' if smp.mx else ''}fp64 per-expert forward + backward), "
+                      f"{dt:.1f} s; tokens/s = rows / k / s"}
 
 
 def cpu_baseline(w, inp, n_tokens, label):
@@ -337,39 +358,51 @@ def cpu_baseline(w, inp, n_tokens, label):
     out, saved = O.layer_fwd(x, W13, W2, idx, gates)
     O.layer_bwd(dout, x, W13, W2, idx, gates, saved, W_r=Wr)
     dt = time.perf_counter() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
-    except Exception:
-        cores = 1
-    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{label}: first {n_tokens} tokens ({n_tokens * w.k} routed rows), full expert "
                       f"weights, fp64 forward + backward, {dt:.1f} s"}
 
 
 def run_reference(args, w):
-    """The oracle timed as it stands on the host cores (rank 0 only), on bounded samples."""
+    """The oracle timed as it stands on the host cores (rank 0 only). Each step is the oracle's
+    per-expert forward + backward over the routed rows of a subset of experts, the subset sized from
+    a one-expert probe so that warm-up + timed steps take about two and a half minutes."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    import torch
     from moe_workloads import make_inputs
-    inp = make_inputs(w, seed=0, device="cpu")
-    ntok = args.ref_tokens
+    import torch
+    if w.routing == "learned":  # the oracle routes from its own fp64 router scores
+        from oracle import moe as O
+        import numpy as np
+        inp = make_inputs(w, seed=0, device="cpu")
+        f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+        lg = O.router_logits(f64(inp["x"]), f64(inp["W_r"]), None if inp["bias"] is None else f64(inp["bias"]))
+        idx, g = O.route(lg, w.k)
+        inp["idx"], inp["gates"] = torch.from_numpy(idx.astype(np.int32)), torch.from_numpy(g)
+    else:
+        inp = make_inputs(w, seed=0, device="cpu")
+    probe = ExpertSample(w, inp, 1)
+    t1 = max(probe.run(), 1e-3)
+    budget = min(30.0, 150.0 / max(1, args.steps + args.warmup))
+    m = max(1, min(w.E, int(budget / t1)))
+    smp = ExpertSample(w, inp, m)
     times = []
-    info = None
     for i in range(args.warmup + args.steps):
-        info = cpu_baseline(w, inp, ntok, w.name)
+        dt = smp.run()
         if i >= args.warmup:
-            times.append(ntok / info["value"])
+            times.append(dt)
     per = statistics.mean(times)
-    val = ntok / per
+    val = smp.rows / w.k / per
+    sample = (f"{w.name}: per step the fp64 oracle's per-expert forward + backward over experts "
+              f"0..{m - 1} ({smp.rows} routed rows = {smp.rows / w.k:.0f} token-equivalents), "
+              f"{'MXFP8-emulated, ' if smp.mx else ''}{per:.2f} s per step")
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(w),
-            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": info["cores"],
-                             "kind": "oracle", "sample": info["sample"]},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -458,11 +491,7 @@ def main():
     launches = L.launch_count() - n0
     clk = clocks.stop()
     barrier()
-    ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end), "cuda")
     ms_per_step = ms / args.steps
     value = world * w.T / (ms_per_step / 1e3)
 
@@ -554,11 +583,7 @@ def main():
             e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([ems], device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), "cuda")
         e2e = {"value": world * w.T / (ems / args.steps / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ems / args.steps, "api": "MoELayer.forward/backward -> moe_layer_fwd/bwd"}
