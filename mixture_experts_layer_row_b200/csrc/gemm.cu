@@ -357,34 +357,50 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
                 tma_load_2d(b_dst, &tmB, &full[s], k0, brow + ti.n0);
               }
             } else {
-              // MN-major weight [E*K rows, N cols]: BN/EPR column blocks x BK rows, 32-row boxes
+              // MN-major weight [E*K rows, N cols]: BN/EPR column blocks x BK rows
               const int krow = ti.e * p.b_rows_per_group + k0;
+              if (p.b_box3d) {
+                tma_load_3d(b_dst, &tmB, &full[s], 0, krow, ti.n0 / C::EPR);
+              } else {
 #pragma unroll
-              for (int blk = 0; blk < BN / C::EPR; ++blk)
+                for (int blk = 0; blk < BN / C::EPR; ++blk)
 #pragma unroll
-                for (int ch = 0; ch < C::CHUNKS; ++ch)
-                  tma_load_2d(b_dst + blk * (C::BK * 128) + ch * 4096, &tmB, &full[s],
-                              ti.n0 + blk * C::EPR, krow + ch * 32);
+                  for (int ch = 0; ch < C::CHUNKS; ++ch)
+                    tma_load_2d(b_dst + blk * (C::BK * 128) + ch * 4096, &tmB, &full[s],
+                                ti.n0 + blk * C::EPR, krow + ch * 32);
+              }
             }
           } else {
-            // GROUP_K: both operands MN-major, contraction rows kstart + 32*chunk
+            // GROUP_K: both operands MN-major, contraction rows kstart + 32*chunk. A 3-D box always
+            // brings BK rows; in the group's last stage the rows past its end (the next group's, or
+            // zero fill past the tensor) land in shared memory but the MMA loop stops before them.
             const int c0 = ks * C::CHUNKS;
             const int nch = min(C::CHUNKS, ti.nchunks - c0);
-            mbar_arrive_expect_tx(&full[s], nch * 32 * 128 * ((BM + BN) / C::EPR) + C::SF_BYTES);
+            const int krow0 = ti.kstart + c0 * 32;
+            const uint32_t a_bytes = p.a_box3d ? C::A_BYTES : nch * 32 * 128 * (BM / C::EPR);
+            const uint32_t b_bytes = p.b_box3d ? C::B_BYTES : nch * 32 * 128 * (BN / C::EPR);
+            mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes + C::SF_BYTES);
             if constexpr (C::MX) {
               bulk_load(sf_dst, sf_a, 512, &full[s]);
               bulk_load(sf_dst + 512, sf_b, 512, &full[s]);
             }
-            for (int ch = 0; ch < nch; ++ch) {
-              const int krow = ti.kstart + (c0 + ch) * 32;
+            if (p.a_box3d) {
+              tma_load_3d(a_dst, &tmA, &full[s], 0, krow0, ti.m0 / C::EPR);
+            } else {
+              for (int ch = 0; ch < nch; ++ch)
 #pragma unroll
-              for (int blk = 0; blk < BM / C::EPR; ++blk)
-                tma_load_2d(a_dst + blk * (C::BK * 128) + ch * 4096, &tmA, &full[s],
-                            ti.m0 + blk * C::EPR, krow);
+                for (int blk = 0; blk < BM / C::EPR; ++blk)
+                  tma_load_2d(a_dst + blk * (C::BK * 128) + ch * 4096, &tmA, &full[s],
+                              ti.m0 + blk * C::EPR, krow0 + ch * 32);
+            }
+            if (p.b_box3d) {
+              tma_load_3d(b_dst, &tmB, &full[s], 0, krow0, ti.n0 / C::EPR);
+            } else {
+              for (int ch = 0; ch < nch; ++ch)
 #pragma unroll
-              for (int blk = 0; blk < BN / C::EPR; ++blk)
-                tma_load_2d(b_dst + blk * (C::BK * 128) + ch * 4096, &tmB, &full[s],
-                            ti.n0 + blk * C::EPR, krow);
+                for (int blk = 0; blk < BN / C::EPR; ++blk)
+                  tma_load_2d(b_dst + blk * (C::BK * 128) + ch * 4096, &tmB, &full[s],
+                              ti.n0 + blk * C::EPR, krow0 + ch * 32);
             }
           }
         }
@@ -656,6 +672,19 @@ bool make_tmap_nd(CUtensorMap* m, const void* ptr, int es, int rank, const uint6
   return r == CUDA_SUCCESS;
 }
 
+// MN-major operand as a 3-D tensor: (128-byte column block, row, column block), so that one box of
+// box_rows rows x nblk column blocks lands in shared memory as nblk consecutive [box_rows x 128 B]
+// blocks -- the MN-major layout the MMA descriptors expect. cols must be a multiple of 128 bytes.
+bool make_tmap_mn(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t cols, int64_t ld,
+                  int box_rows, int nblk, int swizzle) {
+  const int epr = 128 / es;
+  if (cols % epr != 0) return false;
+  const uint64_t dims[3] = {(uint64_t)epr, (uint64_t)rows, (uint64_t)(cols / epr)};
+  const uint64_t strides[2] = {(uint64_t)(ld * es), 128};
+  const uint32_t box[3] = {(uint32_t)epr, (uint32_t)box_rows, (uint32_t)nblk};
+  return make_tmap_nd(m, ptr, es, 3, dims, strides, box, swizzle);
+}
+
 // 2-D row-major tensor [rows, cols] of `es`-byte elements, box [box_rows, box_cols]; swizzle as in
 // make_tmap_nd (2: 128B, 1: 128B with 32-byte atoms, 0: none).
 bool make_tmap(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t cols, int64_t ld,
@@ -692,13 +721,25 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
       return MOE_ERR_CUDA;
     attr_done[dev] = true;
   }
+  GemmParams q = p;
   CUtensorMap ta, tb;
-  // A box: K-major -> [BM rows, EPR cols]; MN-major -> [32 rows, EPR cols]
-  if (!make_tmap(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, A_MN ? 32 : BM, (A_MN && ES == 4) ? 1 : 2))
+  // A box: K-major -> [BM rows, EPR cols]; MN-major -> [BK rows, BM/EPR column blocks] as one 3-D
+  // box when the columns are whole 128-byte blocks, else [32 rows, EPR cols] 2-D boxes
+  const int mn_sw = ES == 4 ? 1 : 2;
+  q.a_box3d = A_MN && (A.cols % C::EPR == 0);
+  q.b_box3d = B_MN && (B.cols % C::EPR == 0);
+  if (q.a_box3d) {
+    if (!make_tmap_mn(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::BK, BM / C::EPR, mn_sw)) return MOE_ERR_CUDA;
+  } else if (!make_tmap(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, A_MN ? 32 : BM, A_MN ? mn_sw : 2)) {
     return MOE_ERR_CUDA;
-  int b_box_rows = B_MN ? 32 : (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN);
-  if (!make_tmap(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, b_box_rows, (B_MN && ES == 4) ? 1 : 2))
-    return MOE_ERR_CUDA;
+  }
+  if (q.b_box3d) {
+    if (!make_tmap_mn(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::BK, BN / C::EPR, mn_sw)) return MOE_ERR_CUDA;
+  } else {
+    const int b_box_rows = B_MN ? 32 : (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN);
+    if (!make_tmap(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, b_box_rows, B_MN ? mn_sw : 2))
+      return MOE_ERR_CUDA;
+  }
   // outputs: 32-row x 128-byte boxes stored from the epilogue's swizzled staging
   CUtensorMap tc, tc2;
   const int64_t out_rows = (MODE == GROUP_K) ? (int64_t)(p.counts ? p.E : 1) * p.M : A.rows;
@@ -710,7 +751,7 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   int grid = sm_count();
   if (grid_cap > 0 && grid_cap < grid) grid = grid_cap;
   if (grid < 1) grid = 1;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, tc, tc2, p);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, tc, tc2, q);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

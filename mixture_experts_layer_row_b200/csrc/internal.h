@@ -42,6 +42,9 @@ struct GemmParams {
   int64_t sA_ld, sB_ld;
   uint32_t* err;
   uint64_t wait_limit_ns;
+  // MN-major operands whose column count is a whole number of 128-byte blocks are loaded as one
+  // 3-D box per stage (set by the launcher); otherwise as 32-row x 128-byte 2-D boxes.
+  int a_box3d, b_box3d;
 };
 
 // Host-side count of kernels enqueued (every launcher adds the kernels it launched).
@@ -52,6 +55,10 @@ bool make_tmap_nd(CUtensorMap* m, const void* ptr, int es, int rank, const uint6
                   const uint64_t* strides_bytes, const uint32_t* box, int swizzle);
 bool make_tmap(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t cols, int64_t ld,
                int box_cols, int box_rows, int swizzle);
+// MN-major operand [rows, cols] (cols a multiple of 128 bytes) as a 3-D tensor
+// (128-byte column block, row, column block), box = box_rows rows x nblk column blocks.
+bool make_tmap_mn(CUtensorMap* m, const void* ptr, int es, int64_t rows, int64_t cols, int64_t ld,
+                  int box_rows, int nblk, int swizzle);
 int sm_count();
 
 int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
