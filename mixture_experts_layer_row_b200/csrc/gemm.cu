@@ -173,25 +173,28 @@ __device__ __forceinline__ void box_store(const CUtensorMap* map, const uint8_t*
   }
 }
 
+// 32 stored values (bf16 or fp32) as raw 16-byte words, and their unpacking to fp32.
 template <int ES>
-__device__ __forceinline__ void load32(const void* src, float* v) {
+__device__ __forceinline__ void raw_load32(const void* src, uint4* w) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 2 * ES; ++q) w[q] = s[q];
+}
+template <int ES>
+__device__ __forceinline__ void unpack32(const uint4* w, float* v) {
   if constexpr (ES == 2) {
-    const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint4 w = s[q];
-      v[8 * q + 0] = bf16lo(w.x); v[8 * q + 1] = bf16hi(w.x);
-      v[8 * q + 2] = bf16lo(w.y); v[8 * q + 3] = bf16hi(w.y);
-      v[8 * q + 4] = bf16lo(w.z); v[8 * q + 5] = bf16hi(w.z);
-      v[8 * q + 6] = bf16lo(w.w); v[8 * q + 7] = bf16hi(w.w);
+      v[8 * q + 0] = bf16lo(w[q].x); v[8 * q + 1] = bf16hi(w[q].x);
+      v[8 * q + 2] = bf16lo(w[q].y); v[8 * q + 3] = bf16hi(w[q].y);
+      v[8 * q + 4] = bf16lo(w[q].z); v[8 * q + 5] = bf16hi(w[q].z);
+      v[8 * q + 6] = bf16lo(w[q].w); v[8 * q + 7] = bf16hi(w[q].w);
     }
   } else {
-    const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const uint4 w = s[q];
-      v[4 * q] = __uint_as_float(w.x); v[4 * q + 1] = __uint_as_float(w.y);
-      v[4 * q + 2] = __uint_as_float(w.z); v[4 * q + 3] = __uint_as_float(w.w);
+      v[4 * q] = __uint_as_float(w[q].x); v[4 * q + 1] = __uint_as_float(w[q].y);
+      v[4 * q + 2] = __uint_as_float(w[q].z); v[4 * q + 3] = __uint_as_float(w[q].w);
     }
   }
 }
@@ -500,20 +503,33 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
       int c1;                                               // tensor row of this slab
       if constexpr (MODE == GROUP_K) c1 = ti.e * p.M + ti.m0 + q * 32;
       else c1 = ti.row_base + ti.m0 + q * 32;
+      // Every variant walks the accumulator in 32-column chunks and keeps the TMEM load of the next
+      // chunk in flight while it converts and stages the current one; CPB chunks fill one box.
+      constexpr int CPB = C::OEPR / 32;
       if constexpr (EPI == EPI_SWIGLU_FWD) {
         // accumulator columns [0, BN/2) gate, [BN/2, BN) up for output columns n0 + [0, BN/2)
-        for (int c = 0; c < BN / 2; c += C::OEPR) {
+        constexpr int NCH = BN / 2 / 32;
+        if (active) {
+          uint32_t ga[32], ua[32], gb[32], ub[32];
+          tmem_ld_32x32b_x32(t_row, ga);
+          tmem_ld_32x32b_x32(t_row + BN / 2, ua);
           uint8_t* bg = wstg;
           uint8_t* bu = wstg + 4096;
           uint8_t* ba = wstg + 8192;
-          if (lane == 0) bulk_wait_read<0>();
-          __syncwarp();
-#pragma unroll 1
-          for (int h = 0; h < C::OEPR; h += 32) {
-            uint32_t rg[32], ru[32];
-            tmem_ld_32x32b_x32(t_row + c + h, rg);
-            tmem_ld_32x32b_x32(t_row + BN / 2 + c + h, ru);
-            tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < NCH; ++j) {
+            uint32_t(&rg)[32] = (j & 1) ? gb : ga;
+            uint32_t(&ru)[32] = (j & 1) ? ub : ua;
+            tmem_ld_wait_regs(rg);
+            tmem_regs_after(ru);
+            if (j + 1 < NCH) {
+              tmem_ld_32x32b_x32(t_row + (j + 1) * 32, (j & 1) ? ga : gb);
+              tmem_ld_32x32b_x32(t_row + BN / 2 + (j + 1) * 32, (j & 1) ? ua : ub);
+            }
+            if (j % CPB == 0) {
+              if (lane == 0) bulk_wait_read<0>();
+              __syncwarp();
+            }
             float g[32], u[32], a[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -522,90 +538,118 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
               u[i] = round_out<C::OES>(__uint_as_float(ru[i]));
               a[i] = silu_f(g[i]) * u[i];
             }
-            if (active) {
-              const int ch0 = (h * C::OES) >> 4;
-              stage_row32<C::OES>(bg, lane, ch0, g);
-              stage_row32<C::OES>(bu, lane, ch0, u);
-              stage_row32<C::OES>(ba, lane, ch0, a);
+            const int ch0 = ((j % CPB) * 32 * C::OES) >> 4;
+            stage_row32<C::OES>(bg, lane, ch0, g);
+            stage_row32<C::OES>(bu, lane, ch0, u);
+            stage_row32<C::OES>(ba, lane, ch0, a);
+            if (j % CPB == CPB - 1) {
+              const int c = (j / CPB) * C::OEPR;
+              box_store(&tmC, bg, lane, ti.n0 + c, c1);
+              box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
+              box_store(&tmC2, ba, lane, ti.n0 + c, c1);
             }
-          }
-          if (active) {
-            box_store(&tmC, bg, lane, ti.n0 + c, c1);
-            box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
-            box_store(&tmC2, ba, lane, ti.n0 + c, c1);
           }
         }
       } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+        // dA chunk from TMEM; gate and up of the saved h13 for the same 32 columns from global
+        // memory, both fetched one chunk ahead
+        constexpr int NCH = BN / 32;
+        constexpr int RW = 2 * C::OES;  // 16-byte words per 32 stored values
         const char* hrow = reinterpret_cast<const char*>(p.aux) +
                            ((size_t)ti.row_base + ti.m0 + q * 32 + lane) * p.ldaux * C::OES;
-        for (int c = 0; c < BN; c += C::OEPR) {
+        if (active) {
+          uint32_t da[32], db[32];
+          uint4 gwa[RW], uwa[RW], gwb[RW], uwb[RW];
+          tmem_ld_32x32b_x32(t_row, da);
+          if (ti.n0 < p.N) {
+            raw_load32<C::OES>(hrow + (size_t)ti.n0 * C::OES, gwa);
+            raw_load32<C::OES>(hrow + (size_t)(p.F + ti.n0) * C::OES, uwa);
+          }
           uint8_t* bg = wstg;
           uint8_t* bu = wstg + 4096;
-          if (lane == 0) bulk_wait_read<0>();
-          __syncwarp();
-          const bool cols = active && (ti.n0 + c < p.N);
-#pragma unroll 1
-          for (int h = 0; h < C::OEPR; h += 32) {
-            uint32_t rd[32];
-            tmem_ld_32x32b_x32(t_row + c + h, rd);
-            tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < NCH; ++j) {
+            uint32_t(&rd)[32] = (j & 1) ? db : da;
+            const uint4* gw = (j & 1) ? gwb : gwa;
+            const uint4* uw = (j & 1) ? uwb : uwa;
+            const int col = ti.n0 + j * 32;
+            const bool cols = col < p.N;  // warp-uniform; N is a multiple of the box width
+            tmem_ld_wait_regs(rd);
+            if (j + 1 < NCH) {
+              tmem_ld_32x32b_x32(t_row + (j + 1) * 32, (j & 1) ? da : db);
+              if (col + 32 < p.N) {
+                raw_load32<C::OES>(hrow + (size_t)(col + 32) * C::OES, (j & 1) ? gwa : gwb);
+                raw_load32<C::OES>(hrow + (size_t)(p.F + col + 32) * C::OES, (j & 1) ? uwa : uwb);
+              }
+            }
             if (cols) {
-              float g[32], u[32], dg[32], du[32];
-              load32<C::OES>(hrow + (size_t)(ti.n0 + c + h) * C::OES, g);
-              load32<C::OES>(hrow + (size_t)(p.F + ti.n0 + c + h) * C::OES, u);
+              if (j % CPB == 0) {
+                if (lane == 0) bulk_wait_read<0>();
+                __syncwarp();
+              }
+              float g[32], u[32];
+              unpack32<C::OES>(gw, g);
+              unpack32<C::OES>(uw, u);
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
-                const float da = __uint_as_float(rd[i]);
+                const float dav = __uint_as_float(rd[i]);
                 const float sg = __fdividef(1.f, 1.f + __expf(-g[i]));
-                du[i] = da * g[i] * sg;
-                dg[i] = da * u[i] * sg * (1.f + g[i] * (1.f - sg));
+                const float gi = g[i];
+                g[i] = dav * u[i] * sg * (1.f + gi * (1.f - sg));  // d gate
+                u[i] = dav * gi * sg;                              // d up
               }
-              const int ch0 = (h * C::OES) >> 4;
-              stage_row32<C::OES>(bg, lane, ch0, dg);
-              stage_row32<C::OES>(bu, lane, ch0, du);
+              const int ch0 = ((j % CPB) * 32 * C::OES) >> 4;
+              stage_row32<C::OES>(bg, lane, ch0, g);
+              stage_row32<C::OES>(bu, lane, ch0, u);
+              if (j % CPB == CPB - 1) {
+                const int c = (j / CPB) * C::OEPR;
+                box_store(&tmC, bg, lane, ti.n0 + c, c1);
+                box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
+              }
             }
-          }
-          if (cols) {
-            box_store(&tmC, bg, lane, ti.n0 + c, c1);
-            box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
           }
         }
       } else {
-        // plain store (act dtype), fp32 + bias (router scores), or a weight gradient (GROUP_K)
-        for (int c = 0; c < BN; c += C::OEPR) {
-          uint8_t* bx = wstg + nb * 4096;
-          const bool cols = active && (ti.n0 + c < p.N);
-          if (cols) {
-            if (lane == 0) bulk_wait_read<C::NBUF - 1>();
-            __syncwarp();
-          }
-#pragma unroll 1
-          for (int h = 0; h < C::OEPR; h += 32) {
-            float v[32];
-            if (nst > 0) {
-              uint32_t raw[32];
-              tmem_ld_32x32b_x32(t_row + c + h, raw);
-              tmem_ld_wait();
+        // plain store (act dtype), fp32 + bias (router scores), or a weight gradient (GROUP_K; an
+        // expert without rows has nst == 0 and gets zeros)
+        constexpr int NCH = BN / 32;
+        if (active) {
+          const bool acc = nst > 0;
+          uint32_t ra[32], rb[32];
+          if (acc) tmem_ld_32x32b_x32(t_row, ra);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(raw[i]);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          for (int j = 0; j < NCH; ++j) {
+            uint32_t(&rc)[32] = (j & 1) ? rb : ra;
+            const int c = (j / CPB) * C::OEPR;  // first column of this chunk's box
+            const bool cols = ti.n0 + c < p.N;
+            if (acc) {
+              tmem_ld_wait_regs(rc);
+              if (j + 1 < NCH) tmem_ld_32x32b_x32(t_row + (j + 1) * 32, (j & 1) ? ra : rb);
             }
+            uint8_t* bx = wstg + nb * 4096;
+            if (cols && j % CPB == 0) {
+              if (lane == 0) bulk_wait_read<C::NBUF - 1>();
+              __syncwarp();
+            }
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = acc ? __uint_as_float(rc[i]) : 0.f;
             if constexpr (EPI == EPI_STORE_F32_BIAS) {
               if (p.bias) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                  const int col = ti.n0 + c + h + i;
+                  const int col = ti.n0 + j * 32 + i;
                   if (col < p.N) v[i] += p.bias[col];
                 }
               }
             }
-            if (cols) stage_row32<C::OES>(bx, lane, (h * C::OES) >> 4, v);
-          }
-          if (cols) {
-            box_store(&tmC, bx, lane, ti.n0 + c, c1);
-            nb = (nb + 1) % C::NBUF;
+            if (cols) {
+              stage_row32<C::OES>(bx, lane, ((j % CPB) * 32 * C::OES) >> 4, v);
+              if (j % CPB == CPB - 1) {
+                box_store(&tmC, bx, lane, ti.n0 + c, c1);
+                nb = (nb + 1) % C::NBUF;
+              }
+            }
           }
         }
       }
