@@ -4,7 +4,7 @@
 // parallelism completely synchronisation-free", unite.ai "Parallelismo, precisione e tecniche di
 // memoria").
 //
-// Structure (one persistent CTA per SM, 192 threads):
+// Structure (one persistent CTA per SM, or CTA pair per two SMs; 192 threads each):
 //   warp 0      TMA producer: one elected thread streams A/B tiles into a STAGES-deep shared-memory
 //               ring (128-byte swizzle), completion counted on a "full" mbarrier per stage;
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, fp32 accumulate) into
@@ -19,6 +19,12 @@
 //   GROUP_K  ragged contraction per expert (wgrad): tiles (expert, m-block, n-block), the K loop runs
 //            over the expert's 32-aligned row range in 32-row chunks (zero pad rows make the tail
 //            exact); an expert with no rows writes a zero gradient.
+// CTA pairs (PAIR, a cluster of two CTAs on neighbouring SMs): a tile covers 256 rows; each CTA
+// loads its 128 rows of A and half of B's columns into its own shared memory (TMA with
+// .cta_group::2, completing on the leader's barrier, no multicast), the leader's MMA thread issues
+// tcgen05.mma.cta_group::2 (M=256) that reads both CTAs' shared memory and writes each CTA's 128
+// accumulator rows into that CTA's TMEM, and its commits arrive on both CTAs' barriers. Each CTA's
+// epilogue drains its own rows and releases the accumulator with a remote arrive on the leader.
 // Every mbarrier wait is bounded; on a timeout the CTA raises MOE_DEVERR_TIMEOUT, drains what it has
 // in flight (bounded), frees TMEM and returns.
 #include "internal.h"
@@ -34,18 +40,24 @@ constexpr int kEpiThreads = 128;
 constexpr int kSmemBudget = 232448;  // 227 KB of opt-in shared memory per CTA
 constexpr int kCtrlBytes = 2048;      // mbarriers, TMEM slot, abort word, tile prefix [<=257 ints]
 
-template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
+template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE, bool PAIR>
 struct Cfg {
+  // PAIR: a cluster of two CTAs computes a 256-row tile with cta_group::2 MMAs; each CTA holds 128
+  // rows of A, half of B's BN columns, and its 128 accumulator rows in its own tensor memory.
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;  // output rows per tile
+  static constexpr int TILE_N = BN;                  // accumulator columns per tile
+  static constexpr int BN_CTA = PAIR ? BN / 2 : BN;  // rows of B (along N) held by one CTA
   static constexpr int EPR = 128 / ES;       // elements per 128-byte smem row
   static constexpr int BK = EPR;             // K elements per pipeline stage
   static constexpr int UK = 32 / ES;         // K per tcgen05.mma (32 bytes)
   static constexpr int KSTEPS = BK / UK;     // MMAs per full stage (4)
   static constexpr int CHUNKS = BK / 32;     // 32-row K chunks per stage (MN-major operands)
   static constexpr int A_BYTES = BM * 128;
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_BYTES = BN_CTA * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   // output staging: each epilogue warp owns NBUF swizzled 32-row x 128-byte boxes
   static constexpr bool MX = (ES == 1);      // MXFP8 block-scaled (E4M3 operands, UE8M0 scales)
+  static_assert(!(PAIR && MX), "block-scaled MMAs run on single CTAs");
   static constexpr int THREADS = kThreads;
   static constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : (MX ? 2 : ES);  // output element size
   static constexpr int OEPR = 128 / OES;     // output columns per staged box
@@ -62,7 +74,7 @@ struct Cfg {
   static_assert(!MX || 2 * BN + STAGES * SF_COLS <= 512, "TMEM overflow");
   static constexpr int BN_OUT = (EPI == EPI_SWIGLU_FWD) ? BN / 2 : BN;  // output columns per tile
   static constexpr uint32_t IDESC =
-      MX ? instr_desc_mx(A_MN, B_MN, BM, BN) : instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, BM, BN);
+      MX ? instr_desc_mx(A_MN, B_MN, BM, BN) : instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, TILE_M, BN);
   // MN-major operands: 16-bit types use the plain 128B swizzle (8-row atoms of 1 KB); 32-bit (tf32)
   // operands need the 128B swizzle with 32-byte chunks (4-row atoms of 512 B).
   static constexpr uint32_t MN_LAYOUT = ES == 4 ? kLayoutSW128Atom32 : kLayoutSW128;
@@ -103,10 +115,10 @@ __device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const i
     }
     const int local = tile - prefix[e];
     const int rows = p.counts ? (p.poff[e + 1] - p.poff[e]) : p.M;
-    const int mt = (rows + BM - 1) / BM;
+    const int mt = (rows + C::TILE_M - 1) / C::TILE_M;
     ti.e = e;
     ti.n0 = (local / mt) * C::BN_OUT;
-    ti.m0 = (local % mt) * BM;
+    ti.m0 = (local % mt) * C::TILE_M;
     ti.rows = rows;
     ti.row_base = p.counts ? p.poff[e] : 0;
     ti.kstart = 0;
@@ -116,8 +128,8 @@ __device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const i
     const int e = tile / per;
     const int local = tile - e * per;
     ti.e = e;
-    ti.m0 = (local / n_tiles) * BM;
-    ti.n0 = (local % n_tiles) * (C::B_BYTES / 128);
+    ti.m0 = (local / n_tiles) * C::TILE_M;
+    ti.n0 = (local % n_tiles) * C::TILE_N;
     ti.rows = p.M;
     ti.row_base = 0;
     if (p.counts) {
@@ -199,13 +211,13 @@ __device__ __forceinline__ void unpack32(const uint4* w, float* v) {
   }
 }
 
-template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
-__global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1)
+template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE, bool PAIR>
+__global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmC,
                         const __grid_constant__ CUtensorMap tmC2, const GemmParams p) {
-  using C = Cfg<ES, A_MN, B_MN, BN, EPI, MODE>;
+  using C = Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>;
   static_assert(MODE == GROUP_M || (A_MN && B_MN), "wgrad mode needs MN-major operands");
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw);  // control area first
@@ -225,6 +237,10 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
   int* prefix = reinterpret_cast<int*>(tmem_slot + 2);  // [E+1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // CTA pairs walk the tile list together: pair index = cluster index, rank 0 = leader
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tstep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   // ---- device-side tile schedule ----
   int n_tiles, m_tiles_fixed = 0, total;
@@ -233,7 +249,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
     const int G = p.counts ? p.E : 1;
     for (int e = threadIdx.x; e < G; e += blockDim.x) {
       const int rows = p.counts ? (p.poff[e + 1] - p.poff[e]) : p.M;
-      prefix[e + 1] = ((rows + BM - 1) / BM) * n_tiles;
+      prefix[e + 1] = ((rows + C::TILE_M - 1) / C::TILE_M) * n_tiles;
     }
     __syncthreads();
     if (warp == 0) {  // inclusive scan of per-group tile counts, 8 groups per lane
@@ -263,7 +279,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
     total = prefix[p.counts ? p.E : 1];
   } else {
     n_tiles = (p.N + BN - 1) / BN;
-    m_tiles_fixed = (p.M + BM - 1) / BM;
+    m_tiles_fixed = (p.M + C::TILE_M - 1) / C::TILE_M;
     total = (p.counts ? p.E : 1) * m_tiles_fixed * n_tiles;
   }
 
@@ -274,11 +290,13 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kEpiThreads);
+      // single CTA: every epilogue thread arrives; pair: lane 0 of the 4 epilogue warps of each CTA
+      mbar_init(&tempty[b], PAIR ? 8 : kEpiThreads);
     }
     mbar_init(done, 1);
     *abort_word = 0;
-    fence_barrier_init();
+    if constexpr (PAIR) fence_barrier_init_cluster();
+    else fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmA);
@@ -287,20 +305,79 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
     if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmC2);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // leader's barriers as shared::cluster addresses (pair: TMA completion and accumulator release)
+  const uint32_t full_lead = PAIR ? cluster_addr(full, 0) : 0u;
+  const uint32_t tempty_lead = PAIR ? cluster_addr(tempty, 0) : 0u;
 
   if (warp == 0) {
     // ===================== TMA producer =====================
-    if (lane == 0) {
+    if (lane == 0 && PAIR) {
+      // Both CTAs of a pair load their own halves (A rows m0 + 128*rank, B columns n0 +
+      // BN/2*rank) into their own shared memory; every copy completes on the leader's full barrier,
+      // which the leader arms with the bytes of both halves. A half past the group's rows is not
+      // loaded (its accumulator rows are never stored).
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = tile0; tile < total && ok; tile += tstep) {
+        TileInfo ti;
+        tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
+        const int nst = num_kstages<C, MODE>(ti);
+        const bool a0 = ti.m0 < ti.rows, a1 = ti.m0 + BM < ti.rows;
+        const bool mine = rank == 0 ? a0 : a1;
+        const uint32_t tx = (a0 ? C::A_BYTES : 0) + (a1 ? C::A_BYTES : 0) + 2 * C::B_BYTES;
+        const int m_cta = ti.m0 + (int)rank * BM;
+        const int n_cta = ti.n0 + (int)rank * C::BN_CTA;
+        for (int ks = 0; ks < nst; ++ks, ++it) {
+          const int s = it % C::STAGES;
+          if (!mbar_wait_bounded(&empty[s], ((it / C::STAGES) & 1) ^ 1, p.wait_limit_ns, abort_word,
+                                 p.err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* a_dst = smA + (size_t)s * C::A_BYTES;
+          uint8_t* b_dst = smB + (size_t)s * C::B_BYTES;
+          const uint32_t fb = full_lead + 8u * (uint32_t)s;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], tx);
+          if constexpr (MODE == GROUP_M) {
+            const int k0 = ks * C::BK;
+            if (mine) tma_load_2d_pair(a_dst, &tmA, fb, k0, ti.row_base + m_cta);
+            const int brow = ti.e * p.b_rows_per_group;
+            if constexpr (B_MN) {
+              tma_load_3d_pair(b_dst, &tmB, fb, 0, brow + k0, n_cta / C::EPR);
+            } else if constexpr (EPI == EPI_SWIGLU_FWD) {
+              // leader: the gate rows of the tile's outputs; peer: the matching up rows
+              tma_load_2d_pair(b_dst, &tmB, fb, k0, brow + (rank ? p.F : 0) + ti.n0);
+            } else {
+              tma_load_2d_pair(b_dst, &tmB, fb, k0, brow + n_cta);
+            }
+          } else {
+            const int krow0 = ti.kstart + ks * C::CHUNKS * 32;
+            if (mine) tma_load_3d_pair(a_dst, &tmA, fb, 0, krow0, m_cta / C::EPR);
+            tma_load_3d_pair(b_dst, &tmB, fb, 0, krow0, n_cta / C::EPR);
+          }
+        }
+      }
+      // drain: the leader's MMAs have consumed every stage this CTA filled (so its copies have
+      // landed) before the CTA exits
+      for (int j = max(0, it - C::STAGES); j < it; ++j)
+        mbar_wait_bounded(&empty[j % C::STAGES], (j / C::STAGES) & 1, p.wait_limit_ns, nullptr, p.err);
+    } else if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = tile0; tile < total && ok; tile += tstep) {
         TileInfo ti;
         tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
         const int nst = num_kstages<C, MODE>(ti);
@@ -414,17 +491,23 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
     }
   } else if (warp == 1) {
     // ===================== MMA issuer =====================
-    if (lane == 0) {
+    // (a pair's MMAs are issued by the leader alone; they read both CTAs' shared memory and write
+    // both CTAs' tensor memory)
+    if (lane == 0 && rank == 0) {
       int it = 0, local = 0;
       bool ok = true;
       bool issued = false;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+      for (int tile = tile0; tile < total && ok; tile += tstep, ++local) {
         TileInfo ti;
         tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
         const int nst = num_kstages<C, MODE>(ti);
         const int buf = local & 1;
-        if (!mbar_wait_bounded(&tempty[buf], ((local >> 1) & 1) ^ 1, p.wait_limit_ns, abort_word,
-                               p.err)) {
+        const bool drained =
+            PAIR ? mbar_wait_bounded_cluster(&tempty[buf], ((local >> 1) & 1) ^ 1, p.wait_limit_ns,
+                                             abort_word, p.err)
+                 : mbar_wait_bounded(&tempty[buf], ((local >> 1) & 1) ^ 1, p.wait_limit_ns,
+                                     abort_word, p.err);
+        if (!drained) {
           ok = false;
           break;
         }
@@ -460,20 +543,29 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
               const uint32_t id = C::IDESC | ((uint32_t)kk << 29) | ((uint32_t)kk << 4);
               umma_mx(d_tmem, ad, bd, id, sf_col | ((uint32_t)kk << 30),
                       (sf_col + 4) | ((uint32_t)kk << 30), (ks > 0 || kk > 0) ? 1u : 0u);
+            } else if constexpr (PAIR) {
+              umma_pair<ES == 2 ? 0 : 1>(d_tmem, ad, bd, C::IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
             } else {
               umma<ES == 2 ? 0 : 1>(d_tmem, ad, bd, C::IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
             }
             issued = true;
           }
-          umma_commit(&empty[s]);
+          if constexpr (PAIR) umma_commit_pair(&empty[s], 0x3);  // frees the stage in both CTAs
+          else umma_commit(&empty[s]);
         }
         if (!ok) break;
-        if (nst > 0) umma_commit(&tfull[buf]);
-        else mbar_arrive(&tfull[buf]);
+        if (nst > 0) {
+          if constexpr (PAIR) umma_commit_pair(&tfull[buf], 0x3);
+          else umma_commit(&tfull[buf]);
+        } else {
+          mbar_arrive(&tfull[buf]);
+          if constexpr (PAIR) mbar_arrive_cluster(cluster_addr(&tfull[buf], 1));
+        }
       }
       // all MMAs issued by this thread must be complete before TMEM is released
       if (issued) {
-        umma_commit(done);
+        if constexpr (PAIR) umma_commit_pair(done, 0x1);
+        else umma_commit(done);
         mbar_wait_bounded(done, 0, p.wait_limit_ns, nullptr, p.err);
       }
     }
@@ -487,7 +579,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
     uint8_t* wstg = stg + (size_t)q * C::NBUF * 4096;
     int nb = 0;                           // next staging box (round robin)
     int local = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+    for (int tile = tile0; tile < total; tile += tstep, ++local) {
       TileInfo ti;
       tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
       const int nst = num_kstages<C, MODE>(ti);
@@ -499,10 +591,11 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-      const bool active = (ti.m0 + q * 32) < ti.rows;       // warp-uniform
+      const int m_cta = ti.m0 + (int)rank * BM;             // this CTA's first tile row
+      const bool active = (m_cta + q * 32) < ti.rows;       // warp-uniform
       int c1;                                               // tensor row of this slab
-      if constexpr (MODE == GROUP_K) c1 = ti.e * p.M + ti.m0 + q * 32;
-      else c1 = ti.row_base + ti.m0 + q * 32;
+      if constexpr (MODE == GROUP_K) c1 = ti.e * p.M + m_cta + q * 32;
+      else c1 = ti.row_base + m_cta + q * 32;
       // Every variant walks the accumulator in 32-column chunks and keeps the TMEM load of the next
       // chunk in flight while it converts and stages the current one; CPB chunks fill one box.
       constexpr int CPB = C::OEPR / 32;
@@ -556,7 +649,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
         constexpr int NCH = BN / 32;
         constexpr int RW = 2 * C::OES;  // 16-byte words per 32 stored values
         const char* hrow = reinterpret_cast<const char*>(p.aux) +
-                           ((size_t)ti.row_base + ti.m0 + q * 32 + lane) * p.ldaux * C::OES;
+                           ((size_t)ti.row_base + m_cta + q * 32 + lane) * p.ldaux * C::OES;
         if (active) {
           uint32_t da[32], db[32];
           uint4 gwa[RW], uwa[RW], gwb[RW], uwb[RW];
@@ -654,17 +747,25 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE>::THREADS, 1
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[buf]);
+      if constexpr (PAIR) {
+        // the leader's MMA thread waits for all eight epilogue warps of the pair
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * (uint32_t)buf);
+      } else {
+        mbar_arrive(&tempty[buf]);
+      }
     }
     if (lane == 0) bulk_wait_all();  // every staged box written out before the CTA ends
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the peer's tensor memory stays allocated until both finish
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -750,12 +851,12 @@ int sm_count() {
 
 namespace {
 
-template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE>
-int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p, int grid_cap,
-                cudaStream_t s) {
-  using C = Cfg<ES, A_MN, B_MN, BN, EPI, MODE>;
-  auto kern = grouped_gemm_kernel<ES, A_MN, B_MN, BN, EPI, MODE>;
+template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE, bool PAIR>
+int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p, cudaStream_t s) {
+  using C = Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>;
+  auto kern = grouped_gemm_kernel<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>;
   static bool attr_done[64] = {false};
+  static int pair_slots[64] = {0};  // co-resident CTA pairs (clusters of 2) per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
@@ -768,19 +869,22 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   GemmParams q = p;
   CUtensorMap ta, tb;
   // A box: K-major -> [BM rows, EPR cols]; MN-major -> [BK rows, BM/EPR column blocks] as one 3-D
-  // box when the columns are whole 128-byte blocks, else [32 rows, EPR cols] 2-D boxes
+  // box when the columns are whole 128-byte blocks, else [32 rows, EPR cols] 2-D boxes (single
+  // CTAs only). B likewise, with the BN_CTA rows (or columns) one CTA holds.
   const int mn_sw = ES == 4 ? 1 : 2;
   q.a_box3d = A_MN && (A.cols % C::EPR == 0);
   q.b_box3d = B_MN && (B.cols % C::EPR == 0);
+  if (PAIR && ((A_MN && !q.a_box3d) || (B_MN && !q.b_box3d))) return MOE_ERR_UNSUPPORTED;
   if (q.a_box3d) {
     if (!make_tmap_mn(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::BK, BM / C::EPR, mn_sw)) return MOE_ERR_CUDA;
   } else if (!make_tmap(&ta, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, A_MN ? 32 : BM, A_MN ? mn_sw : 2)) {
     return MOE_ERR_CUDA;
   }
   if (q.b_box3d) {
-    if (!make_tmap_mn(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::BK, BN / C::EPR, mn_sw)) return MOE_ERR_CUDA;
+    if (!make_tmap_mn(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::BK, C::BN_CTA / C::EPR, mn_sw))
+      return MOE_ERR_CUDA;
   } else {
-    const int b_box_rows = B_MN ? 32 : (EPI == EPI_SWIGLU_FWD ? BN / 2 : BN);
+    const int b_box_rows = B_MN ? 32 : ((PAIR || EPI != EPI_SWIGLU_FWD) ? C::BN_CTA : BN / 2);
     if (!make_tmap(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, b_box_rows, B_MN ? mn_sw : 2))
       return MOE_ERR_CUDA;
   }
@@ -792,10 +896,40 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   tc2 = tc;
   if (EPI == EPI_SWIGLU_FWD && !make_tmap(&tc2, p.C2, C::OES, out_rows, p.F, p.ldc2, C::OEPR, 32, 2))
     return MOE_ERR_CUDA;
-  int grid = sm_count();
-  if (grid_cap > 0 && grid_cap < grid) grid = grid_cap;
-  if (grid < 1) grid = 1;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, tc, tc2, q);
+  // persistent grid: one CTA (pair) per SM (pair of SMs), capped by the tile count where the host
+  // knows it (GROUP_K: fixed tiles per group)
+  int64_t cap = 0;
+  if (MODE == GROUP_K) {
+    cap = (int64_t)(p.counts ? p.E : 1) * ((p.M + C::TILE_M - 1) / C::TILE_M) * ((p.N + BN - 1) / BN);
+    if (cap < 1) cap = 1;
+  }
+  if constexpr (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (!pair_slots[dev]) {
+      cfg.gridDim = dim3(2 * (sm_count() / 2));
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return MOE_ERR_CUDA;
+      pair_slots[dev] = n;
+    }
+    int64_t pairs = pair_slots[dev];
+    if (cap > 0 && cap < pairs) pairs = cap;
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tc2, q) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    int64_t grid = sm_count();
+    if (cap > 0 && cap < grid) grid = cap;
+    kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, tc, tc2, q);
+  }
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -803,36 +937,33 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
 }  // namespace
 
 // Dispatch a GEMM request to its compiled variant. The caller (api.cu) has validated shapes.
+// The SwiGLU forward GEMM (bf16 / tf32) runs on CTA pairs: 256 x 256 tiles with cta_group::2 MMAs,
+// so each weight tile is fetched once per 256 routed rows. The other GEMMs are bound by their
+// epilogues, which a pair would couple (the MMA then waits for the slower CTA of the two), and run
+// on single CTAs with 128-row tiles, as do the router GEMM and MXFP8.
 int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
                 const GemmParams& p, cudaStream_t s) {
-  // GROUP_K launches know their tile count on the host; cap the grid there.
-  int cap = 0;
-  if (kind == GK_WGRAD) {
-    const int mt = (p.M + BM - 1) / BM, nt = (p.N + bn - 1) / bn;
-    const int64_t total = (int64_t)(p.counts ? p.E : 1) * mt * nt;
-    cap = total < 1 ? 1 : (int)(total < (1 << 30) ? total : (1 << 30));
-  }
-#define MOE_GEMM_CASES(ES_)                                                                          \
-  switch (kind) {                                                                                    \
-    case GK_FWD1_SWIGLU:                                                                             \
-      return launch_impl<ES_, false, false, 256, EPI_SWIGLU_FWD, GROUP_M>(A, B, p, cap, s);          \
-    case GK_FWD2:                                                                                    \
-      if (bn == 256) return launch_impl<ES_, false, false, 256, EPI_STORE, GROUP_M>(A, B, p, cap, s); \
-      return launch_impl<ES_, false, false, 128, EPI_STORE, GROUP_M>(A, B, p, cap, s);               \
-    case GK_DGRAD2_SWIGLU:                                                                           \
-      if (bn == 256)                                                                                 \
-        return launch_impl<ES_, false, true, 256, EPI_SWIGLU_BWD, GROUP_M>(A, B, p, cap, s);         \
-      return launch_impl<ES_, false, true, 128, EPI_SWIGLU_BWD, GROUP_M>(A, B, p, cap, s);           \
-    case GK_DGRAD1:                                                                                  \
-      if (bn == 256) return launch_impl<ES_, false, true, 256, EPI_STORE, GROUP_M>(A, B, p, cap, s);  \
-      return launch_impl<ES_, false, true, 128, EPI_STORE, GROUP_M>(A, B, p, cap, s);                \
-    case GK_WGRAD:                                                                                   \
-      if (bn == 256) return launch_impl<ES_, true, true, 256, EPI_STORE, GROUP_K>(A, B, p, cap, s);   \
-      return launch_impl<ES_, true, true, 128, EPI_STORE, GROUP_K>(A, B, p, cap, s);                 \
-    case GK_ROUTER:                                                                                  \
-      if (bn == 256)                                                                                 \
-        return launch_impl<ES_, false, false, 256, EPI_STORE_F32_BIAS, GROUP_M>(A, B, p, cap, s);    \
-      return launch_impl<ES_, false, false, 128, EPI_STORE_F32_BIAS, GROUP_M>(A, B, p, cap, s);      \
+#define MOE_GEMM_CASES(ES_)                                                                        \
+  switch (kind) {                                                                                  \
+    case GK_FWD1_SWIGLU:                                                                           \
+      return launch_impl<ES_, false, false, 256, EPI_SWIGLU_FWD, GROUP_M, true>(A, B, p, s);       \
+    case GK_FWD2:                                                                                  \
+      if (bn == 256) return launch_impl<ES_, false, false, 256, EPI_STORE, GROUP_M, false>(A, B, p, s); \
+      return launch_impl<ES_, false, false, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);           \
+    case GK_DGRAD2_SWIGLU:                                                                         \
+      if (bn == 256)                                                                               \
+        return launch_impl<ES_, false, true, 256, EPI_SWIGLU_BWD, GROUP_M, false>(A, B, p, s);     \
+      return launch_impl<ES_, false, true, 128, EPI_SWIGLU_BWD, GROUP_M, false>(A, B, p, s);       \
+    case GK_DGRAD1:                                                                                \
+      if (bn == 256) return launch_impl<ES_, false, true, 256, EPI_STORE, GROUP_M, false>(A, B, p, s); \
+      return launch_impl<ES_, false, true, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);            \
+    case GK_WGRAD:                                                                                 \
+      if (bn == 256) return launch_impl<ES_, true, true, 256, EPI_STORE, GROUP_K, false>(A, B, p, s); \
+      return launch_impl<ES_, true, true, 128, EPI_STORE, GROUP_K, false>(A, B, p, s);             \
+    case GK_ROUTER:                                                                                \
+      if (bn == 256)                                                                               \
+        return launch_impl<ES_, false, false, 256, EPI_STORE_F32_BIAS, GROUP_M, false>(A, B, p, s); \
+      return launch_impl<ES_, false, false, 128, EPI_STORE_F32_BIAS, GROUP_M, false>(A, B, p, s);  \
   }
   if (es == 2) {
     MOE_GEMM_CASES(2)
@@ -840,11 +971,11 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
     MOE_GEMM_CASES(4)
   } else if (es == 1) {  // MXFP8: BN = 128 (TMEM holds two accumulators plus per-stage scales)
     switch (kind) {
-      case GK_FWD1_SWIGLU: return launch_impl<1, false, false, 128, EPI_SWIGLU_FWD, GROUP_M>(A, B, p, cap, s);
-      case GK_FWD2: return launch_impl<1, false, false, 128, EPI_STORE, GROUP_M>(A, B, p, cap, s);
-      case GK_DGRAD2_SWIGLU: return launch_impl<1, false, true, 128, EPI_SWIGLU_BWD, GROUP_M>(A, B, p, cap, s);
-      case GK_DGRAD1: return launch_impl<1, false, true, 128, EPI_STORE, GROUP_M>(A, B, p, cap, s);
-      case GK_WGRAD: return launch_impl<1, true, true, 128, EPI_STORE, GROUP_K>(A, B, p, cap, s);
+      case GK_FWD1_SWIGLU: return launch_impl<1, false, false, 128, EPI_SWIGLU_FWD, GROUP_M, false>(A, B, p, s);
+      case GK_FWD2: return launch_impl<1, false, false, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);
+      case GK_DGRAD2_SWIGLU: return launch_impl<1, false, true, 128, EPI_SWIGLU_BWD, GROUP_M, false>(A, B, p, s);
+      case GK_DGRAD1: return launch_impl<1, false, true, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);
+      case GK_WGRAD: return launch_impl<1, true, true, 128, EPI_STORE, GROUP_K, false>(A, B, p, s);
       default: return MOE_ERR_UNSUPPORTED;
     }
   }
