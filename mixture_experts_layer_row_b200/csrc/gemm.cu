@@ -61,7 +61,10 @@ struct Cfg {
   static constexpr int THREADS = kThreads;
   static constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : (MX ? 2 : ES);  // output element size
   static constexpr int OEPR = 128 / OES;     // output columns per staged box
-  static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3 : 2;
+  // accumulators in TMEM: two (the epilogue drains one while the MMA fills the other), or one for
+  // MXFP8 tiles of 256 columns, whose per-stage scale columns leave no room for a second
+  static constexpr int NACC = (MX && BN == 256) ? 1 : 2;
+  static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3 : (NACC == 1 ? 1 : 2);
   static constexpr int STAGING_BYTES = 4 * NBUF * 4096;
   // MXFP8: per stage, one 512-byte scale chunk per 128 rows of A and of B (TMEM: 4 columns each)
   static constexpr int SF_BYTES = MX ? 512 + (BN / 128) * 512 : 0;
@@ -70,8 +73,9 @@ struct Cfg {
       (kSmemBudget - kCtrlBytes - 1024 - STAGING_BYTES) / (STAGE_BYTES + SF_BYTES);
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static_assert(STAGES >= 2, "pipeline too shallow");
-  static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;  // two accumulators (+ scale columns)
-  static_assert(!MX || 2 * BN + STAGES * SF_COLS <= 512, "TMEM overflow");
+  static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;  // accumulators (+ scale columns)
+  static_assert(!MX || NACC * BN + STAGES * SF_COLS <= 512, "TMEM overflow");
+  static_assert(!MX || EPI != EPI_SWIGLU_FWD || BN == 128, "MXFP8 gate/up tiles are 128 wide");
   static constexpr int BN_OUT = (EPI == EPI_SWIGLU_FWD) ? BN / 2 : BN;  // output columns per tile
   static constexpr uint32_t IDESC =
       MX ? instr_desc_mx(A_MN, B_MN, BM, BN) : instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, TILE_M, BN);
@@ -424,7 +428,9 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES + C::SF_BYTES);
             if constexpr (C::MX) {
               bulk_load(sf_dst, sf_a, 512, &full[s]);
-              bulk_load(sf_dst + 512, sf_b, 512, &full[s]);
+#pragma unroll
+              for (int c = 0; c < BN / 128; ++c)  // B: one chunk per 128 rows (chunk rows are sB_ld apart)
+                bulk_load(sf_dst + 512 * (c + 1), sf_b + (int64_t)c * p.sB_ld * 512, 512, &full[s]);
             }
             // A: K-major rows of the routed buffer (or the token matrix)
             tma_load_2d(a_dst, &tmA, &full[s], k0, ti.row_base + ti.m0);
@@ -462,7 +468,9 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes + C::SF_BYTES);
             if constexpr (C::MX) {
               bulk_load(sf_dst, sf_a, 512, &full[s]);
-              bulk_load(sf_dst + 512, sf_b, 512, &full[s]);
+#pragma unroll
+              for (int c = 0; c < BN / 128; ++c)  // B: one chunk per 128 rows (chunk rows are sB_ld apart)
+                bulk_load(sf_dst + 512 * (c + 1), sf_b + (int64_t)c * p.sB_ld * 512, 512, &full[s]);
             }
             if (p.a_box3d) {
               tma_load_3d(a_dst, &tmA, &full[s], 0, krow0, ti.m0 / C::EPR);
@@ -501,12 +509,11 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
         TileInfo ti;
         tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
         const int nst = num_kstages<C, MODE>(ti);
-        const int buf = local & 1;
+        const int buf = local % C::NACC;
+        const uint32_t use = (uint32_t)(local / C::NACC) & 1u;  // parity of this buffer's use
         const bool drained =
-            PAIR ? mbar_wait_bounded_cluster(&tempty[buf], ((local >> 1) & 1) ^ 1, p.wait_limit_ns,
-                                             abort_word, p.err)
-                 : mbar_wait_bounded(&tempty[buf], ((local >> 1) & 1) ^ 1, p.wait_limit_ns,
-                                     abort_word, p.err);
+            PAIR ? mbar_wait_bounded_cluster(&tempty[buf], use ^ 1u, p.wait_limit_ns, abort_word, p.err)
+                 : mbar_wait_bounded(&tempty[buf], use ^ 1u, p.wait_limit_ns, abort_word, p.err);
         if (!drained) {
           ok = false;
           break;
@@ -527,7 +534,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           uint32_t sf_col = 0;
           if constexpr (C::MX) {
             // this stage's scales: smem chunks -> TMEM columns after the two accumulators
-            sf_col = tmem_base + 2 * BN + s * C::SF_COLS;
+            sf_col = tmem_base + C::NACC * BN + s * C::SF_COLS;
             const uint32_t sf_smem = smem_u32(sfs + (size_t)s * C::SF_BYTES);
 #pragma unroll
             for (int c = 0; c < 1 + BN / 128; ++c)
@@ -583,10 +590,11 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       TileInfo ti;
       tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
       const int nst = num_kstages<C, MODE>(ti);
-      const int buf = local & 1;
+      const int buf = local % C::NACC;
       int ok = 1;
       if (lane == 0)
-        ok = mbar_wait_bounded(&tfull[buf], (local >> 1) & 1, p.wait_limit_ns, abort_word, p.err);
+        ok = mbar_wait_bounded(&tfull[buf], (uint32_t)(local / C::NACC) & 1u, p.wait_limit_ns,
+                               abort_word, p.err);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
@@ -969,13 +977,23 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
     MOE_GEMM_CASES(2)
   } else if (es == 4) {
     MOE_GEMM_CASES(4)
-  } else if (es == 1) {  // MXFP8: BN = 128 (TMEM holds two accumulators plus per-stage scales)
+  } else if (es == 1) {
+    // MXFP8: the SwiGLU GEMMs use 128-column tiles with two accumulators; the plain-store GEMMs use
+    // 256-column tiles (twice the work per block-scaled MMA) with one accumulator when N is a
+    // multiple of 256 (every B scale chunk a tile reads then exists).
+    const bool wide = p.N % 256 == 0;
     switch (kind) {
       case GK_FWD1_SWIGLU: return launch_impl<1, false, false, 128, EPI_SWIGLU_FWD, GROUP_M, false>(A, B, p, s);
-      case GK_FWD2: return launch_impl<1, false, false, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);
+      case GK_FWD2:
+        if (wide) return launch_impl<1, false, false, 256, EPI_STORE, GROUP_M, false>(A, B, p, s);
+        return launch_impl<1, false, false, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);
       case GK_DGRAD2_SWIGLU: return launch_impl<1, false, true, 128, EPI_SWIGLU_BWD, GROUP_M, false>(A, B, p, s);
-      case GK_DGRAD1: return launch_impl<1, false, true, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);
-      case GK_WGRAD: return launch_impl<1, true, true, 128, EPI_STORE, GROUP_K, false>(A, B, p, s);
+      case GK_DGRAD1:
+        if (wide) return launch_impl<1, false, true, 256, EPI_STORE, GROUP_M, false>(A, B, p, s);
+        return launch_impl<1, false, true, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);
+      case GK_WGRAD:
+        if (wide) return launch_impl<1, true, true, 256, EPI_STORE, GROUP_K, false>(A, B, p, s);
+        return launch_impl<1, true, true, 128, EPI_STORE, GROUP_K, false>(A, B, p, s);
       default: return MOE_ERR_UNSUPPORTED;
     }
   }

@@ -129,7 +129,8 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const uint4* __res
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kWarps * 32) combine_bwd_kernel(
+// 64 registers at most: four blocks (32 warps) per SM keep enough loads in flight
+__global__ void __launch_bounds__(kWarps * 32, 4) combine_bwd_kernel(
     const uint4* __restrict__ dout, const uint4* __restrict__ y, const float* __restrict__ gates,
     const int32_t* __restrict__ prow, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ counts, const int32_t* __restrict__ poff, uint4* __restrict__ dy,
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_bwd_kernel(
     g[j] = __shfl_sync(0xffffffffu, myg, j);
     dot[j] = 0.f;
   }
-#pragma unroll 2
+#pragma unroll 1
   for (int v = lane; v < vpr; v += 32) {
     float fd[V::N];
     V::unpack(ldg_stream(dout + (size_t)t * vpr + v), fd);

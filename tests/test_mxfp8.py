@@ -95,6 +95,8 @@ def test_quantize_tiled_bitexact(rows, cols, mode):
 
 SHAPES = {
     "ragged": (512, 128, 256, 8, 2, [0, 1, 31, 33, 129, 200, 300, 330]),
+    # d and F multiples of 256: the plain-store GEMMs take 256-column tiles with ragged groups
+    "ragged_wide": (512, 256, 256, 8, 2, [0, 1, 31, 33, 129, 200, 300, 330]),
     "one_expert": (300, 128, 128, 4, 1, [300, 0, 0, 0]),
     "wide": (2048, 2048, 1024, 16, 4, None),
 }
