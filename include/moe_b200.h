@@ -225,7 +225,9 @@ MOE_API int moe_router_wgrad(const moe_config_t* cfg, const void* dlogits, const
  *   MOE_QUANT_ROW_TILED  blocks along a row;    s tiled over (row, block)    (rows, cols % 128)
  *   MOE_QUANT_COL_TILED  blocks down a column;  s tiled over (column, block) (rows, cols % 128)
  *   MOE_QUANT_ROW_TILED_GATEUP  as ROW_TILED for stacks of [G gate rows; G up rows] (W13 with
- *                        G = F), rows remapped so each 64 gate + 64 up rows share chunks (G % 64).
+ *                        G = F), rows remapped so each 64 gate + 64 up rows share chunks (G % 64);
+ *                        a layout for 64 + 64-row fused tiles (the layer's grouped GEMM takes
+ *                        128 + 128-row tiles and plain ROW_TILED W13 scales).
  * Tiled: the scale of (MN index i, K-block b) -- i = row for ROW modes, column for COL modes -- sits in
  * 512-byte chunk (i/128, b/4) (chunks of one i/128 consecutive), at byte (i%32)*16 + ((i%128)/32)*4 +
  * b%4: the layout the MXFP8 grouped GEMM streams. `G` is used by the GATEUP mode only.
@@ -241,7 +243,7 @@ MOE_API int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode
 /* The grouped GEMM of moe_grouped_gemm with MXFP8 operands (tcgen05 kind::mxf8f6f4.block_scale, fp32
  * accumulation, bf16 outputs). Each operand is E4M3 codes in the layout its bf16 counterpart has in
  * moe_grouped_gemm plus UE8M0 scales, tiled, along that GEMM's contraction axis:
- *   FWD1_SWIGLU   A = x_perm ROW_TILED [R,d]     B = W13 ROW_TILED_GATEUP [E*2F,d] (G = F)
+ *   FWD1_SWIGLU   A = x_perm ROW_TILED [R,d]     B = W13 ROW_TILED [E*2F,d]
  *   FWD2          A = a      ROW_TILED [R,F]     B = W2  ROW_TILED [E*d,F]
  *   DGRAD2_SWIGLU A = dy     ROW_TILED [R,d]     B = W2  COL_TILED [E*d,F]
  *   DGRAD1        A = dh13   ROW_TILED [R,2F]    B = W13 COL_TILED [E*2F,d]
@@ -306,7 +308,8 @@ MOE_API int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const
 
 /* ---- whole layer, MXFP8 ---------------------------------------------------------------------------------- */
 
-/* Quantised copies of the expert weights (caller-owned; refresh after every weight update):
+/* Quantised copies of the expert weights (caller-owned; refresh after every weight update), scales
+ * in the tiled layouts moe_grouped_gemm_mxfp8 reads (ROW_TILED / COL_TILED):
  *   W13q/W13s  ROW along d  [E*2F, d] / [E*2F, d/32]      (forward GEMM1)
  *   W13tq/W13ts COL along 2F [E*2F, d] / [d, E*2F/32]     (GEMM1 dgrad)
  *   W2q/W2s    ROW along F  [E*d, F] / [E*d, F/32]        (forward GEMM2)

@@ -462,7 +462,7 @@ int moe_quantize_weights_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
               MOE_ERR_INVALID_ARG);
   const int64_t E = cfg->E, d = cfg->d, F = cfg->F;
   cudaStream_t s = S(stream);
-  MOE_TRY(moe_quantize_mxfp8(w->W13, E * 2 * F, (int)d, MOE_QUANT_ROW_TILED_GATEUP, F, qw->W13q,
+  MOE_TRY(moe_quantize_mxfp8(w->W13, E * 2 * F, (int)d, MOE_QUANT_ROW_TILED, 0, qw->W13q,
                              qw->W13s, s));
   MOE_TRY(moe_quantize_mxfp8(w->W13, E * 2 * F, (int)d, MOE_QUANT_COL_TILED, 0, qw->W13tq, qw->W13ts, s));
   MOE_TRY(moe_quantize_mxfp8(w->W2, E * d, (int)F, MOE_QUANT_ROW_TILED, 0, qw->W2q, qw->W2s, s));

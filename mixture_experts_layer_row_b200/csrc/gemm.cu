@@ -64,7 +64,9 @@ struct Cfg {
   // accumulators in TMEM: two (the epilogue drains one while the MMA fills the other), or one for
   // MXFP8 tiles of 256 columns, whose per-stage scale columns leave no room for a second
   static constexpr int NACC = (MX && BN == 256) ? 1 : 2;
-  static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3 : (NACC == 1 ? 1 : 2);
+  static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3
+                              : (EPI == EPI_SWIGLU_BWD) ? 2  // one (gate, up) pair of boxes per warp
+                              : (NACC == 1 ? 1 : 2);
   static constexpr int STAGING_BYTES = 4 * NBUF * 4096;
   // MXFP8: per stage, one 512-byte scale chunk per 128 rows of A and of B (TMEM: 4 columns each)
   static constexpr int SF_BYTES = MX ? 512 + (BN / 128) * 512 : 0;
@@ -75,7 +77,6 @@ struct Cfg {
   static_assert(STAGES >= 2, "pipeline too shallow");
   static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;  // accumulators (+ scale columns)
   static_assert(!MX || NACC * BN + STAGES * SF_COLS <= 512, "TMEM overflow");
-  static_assert(!MX || EPI != EPI_SWIGLU_FWD || BN == 128, "MXFP8 gate/up tiles are 128 wide");
   static constexpr int BN_OUT = (EPI == EPI_SWIGLU_FWD) ? BN / 2 : BN;  // output columns per tile
   static constexpr uint32_t IDESC =
       MX ? instr_desc_mx(A_MN, B_MN, BM, BN) : instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, TILE_M, BN);
@@ -397,6 +398,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           const uint8_t* sf_a = nullptr;
           const uint8_t* sf_b = nullptr;
           uint8_t* sf_dst = nullptr;
+          int64_t b_chunk_step = 0;
           if constexpr (C::MX) {
             // this stage's scales: one 512-byte chunk for the 128 rows of A, one per 128 of B
             uint8_t* sf = sfs + (size_t)s * C::SF_BYTES;
@@ -408,7 +410,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
                 bmb = ti.n0 >> 7;
                 bkq = (int64_t)ti.e * (p.b_rows_per_group >> 7) + ks;
               } else if constexpr (EPI == EPI_SWIGLU_FWD) {
-                bmb = (int64_t)ti.e * (p.b_rows_per_group >> 7) + ti.n0 / (BN / 2);
+                bmb = ((int64_t)ti.e * p.b_rows_per_group + ti.n0) >> 7;  // gate rows n0..n0+BN/2-1
                 bkq = ks;
               } else {
                 bmb = ((int64_t)ti.e * p.b_rows_per_group + ti.n0) >> 7;
@@ -421,6 +423,9 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             }
             sf_a = p.sA + (amb * p.sA_ld + akq) * 512;
             sf_b = p.sB + (bmb * p.sB_ld + bkq) * 512;
+            // the tile's second 128 B rows: the next chunk row, or for the fused SwiGLU tile (gate
+            // rows, then the up rows F further down W13) the chunk row F/128 further
+            b_chunk_step = (EPI == EPI_SWIGLU_FWD ? (int64_t)(p.F >> 7) : 1) * p.sB_ld * 512;
             sf_dst = sf;
           }
           if constexpr (MODE == GROUP_M) {
@@ -429,8 +434,8 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             if constexpr (C::MX) {
               bulk_load(sf_dst, sf_a, 512, &full[s]);
 #pragma unroll
-              for (int c = 0; c < BN / 128; ++c)  // B: one chunk per 128 rows (chunk rows are sB_ld apart)
-                bulk_load(sf_dst + 512 * (c + 1), sf_b + (int64_t)c * p.sB_ld * 512, 512, &full[s]);
+              for (int c = 0; c < BN / 128; ++c)  // B: one chunk per 128 rows of the tile
+                bulk_load(sf_dst + 512 * (c + 1), sf_b + (int64_t)c * b_chunk_step, 512, &full[s]);
             }
             // A: K-major rows of the routed buffer (or the token matrix)
             tma_load_2d(a_dst, &tmA, &full[s], k0, ti.row_base + ti.m0);
@@ -469,8 +474,8 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             if constexpr (C::MX) {
               bulk_load(sf_dst, sf_a, 512, &full[s]);
 #pragma unroll
-              for (int c = 0; c < BN / 128; ++c)  // B: one chunk per 128 rows (chunk rows are sB_ld apart)
-                bulk_load(sf_dst + 512 * (c + 1), sf_b + (int64_t)c * p.sB_ld * 512, 512, &full[s]);
+              for (int c = 0; c < BN / 128; ++c)  // B: one chunk per 128 rows of the tile
+                bulk_load(sf_dst + 512 * (c + 1), sf_b + (int64_t)c * b_chunk_step, 512, &full[s]);
             }
             if (p.a_box3d) {
               tma_load_3d(a_dst, &tmA, &full[s], 0, krow0, ti.m0 / C::EPR);
@@ -978,16 +983,19 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
   } else if (es == 4) {
     MOE_GEMM_CASES(4)
   } else if (es == 1) {
-    // MXFP8: the SwiGLU GEMMs use 128-column tiles with two accumulators; the plain-store GEMMs use
-    // 256-column tiles (twice the work per block-scaled MMA) with one accumulator when N is a
-    // multiple of 256 (every B scale chunk a tile reads then exists).
+    // MXFP8: 256-column tiles (twice the work per block-scaled MMA) with one accumulator, since the
+    // per-stage scale columns leave no TMEM for a second; the SwiGLU forward tile is 128 gate + 128
+    // up rows of W13 (F is a multiple of 128); fwd2, dgrad1 and the wgrads take wide tiles when N
+    // is a multiple of 256 (every B scale chunk a tile reads then exists). The SwiGLU backward and
+    // narrow cases use 128-column tiles with two accumulators.
     const bool wide = p.N % 256 == 0;
     switch (kind) {
-      case GK_FWD1_SWIGLU: return launch_impl<1, false, false, 128, EPI_SWIGLU_FWD, GROUP_M, false>(A, B, p, s);
+      case GK_FWD1_SWIGLU: return launch_impl<1, false, false, 256, EPI_SWIGLU_FWD, GROUP_M, false>(A, B, p, s);
       case GK_FWD2:
         if (wide) return launch_impl<1, false, false, 256, EPI_STORE, GROUP_M, false>(A, B, p, s);
         return launch_impl<1, false, false, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);
-      case GK_DGRAD2_SWIGLU: return launch_impl<1, false, true, 128, EPI_SWIGLU_BWD, GROUP_M, false>(A, B, p, s);
+      case GK_DGRAD2_SWIGLU:  // epilogue-heavy: two accumulators overlap it with the next tile
+        return launch_impl<1, false, true, 128, EPI_SWIGLU_BWD, GROUP_M, false>(A, B, p, s);
       case GK_DGRAD1:
         if (wide) return launch_impl<1, false, true, 256, EPI_STORE, GROUP_M, false>(A, B, p, s);
         return launch_impl<1, false, true, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);

@@ -161,7 +161,7 @@ ROWQ, COLQ = O._mx_row, O._mx_col
 def test_mx_fwd1(shape):
     P = MxProblem(shape)
     X, W13 = P.rows(P.d), P.weights(P.E, 2 * P.F, P.d)
-    h13, a = P.run(P.L.GEMM_FWD1_SWIGLU, P.quant(X, 0), P.quant(W13.reshape(-1, P.d), 2, P.F),
+    h13, a = P.run(P.L.GEMM_FWD1_SWIGLU, P.quant(X, 0), P.quant(W13.reshape(-1, P.d), 0),
                    torch.zeros((P.R32, 2 * P.F), dtype=torch.bfloat16),
                    torch.zeros((P.R32, P.F), dtype=torch.bfloat16))
     Xn, Wn, H, A = np64(X), np64(W13), np64(h13), np64(a)
