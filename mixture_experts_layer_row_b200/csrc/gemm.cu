@@ -950,10 +950,11 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
 }  // namespace
 
 // Dispatch a GEMM request to its compiled variant. The caller (api.cu) has validated shapes.
-// The SwiGLU forward GEMM (bf16 / tf32) runs on CTA pairs: 256 x 256 tiles with cta_group::2 MMAs,
-// so each weight tile is fetched once per 256 routed rows. The other GEMMs are bound by their
-// epilogues, which a pair would couple (the MMA then waits for the slower CTA of the two), and run
-// on single CTAs with 128-row tiles, as do the router GEMM and MXFP8.
+// The ragged-row bf16 / tf32 GEMMs with light epilogues (fwd1 + SwiGLU, fwd2, dgrad1) run on CTA
+// pairs: 256 x 256 tiles with cta_group::2 MMAs, so each weight tile is fetched once per 256 routed
+// rows and each SM holds half of B. The SwiGLU backward and the wgrads are bound by their epilogues,
+// which a pair would couple (the MMA then waits for the slower CTA of the two): they run on single
+// CTAs with 128-row tiles, as do the router GEMM and MXFP8.
 int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
                 const GemmParams& p, cudaStream_t s) {
 #define MOE_GEMM_CASES(ES_)                                                                        \
@@ -961,14 +962,14 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
     case GK_FWD1_SWIGLU:                                                                           \
       return launch_impl<ES_, false, false, 256, EPI_SWIGLU_FWD, GROUP_M, true>(A, B, p, s);       \
     case GK_FWD2:                                                                                  \
-      if (bn == 256) return launch_impl<ES_, false, false, 256, EPI_STORE, GROUP_M, false>(A, B, p, s); \
+      if (bn == 256) return launch_impl<ES_, false, false, 256, EPI_STORE, GROUP_M, true>(A, B, p, s);  \
       return launch_impl<ES_, false, false, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);           \
     case GK_DGRAD2_SWIGLU:                                                                         \
       if (bn == 256)                                                                               \
         return launch_impl<ES_, false, true, 256, EPI_SWIGLU_BWD, GROUP_M, false>(A, B, p, s);     \
       return launch_impl<ES_, false, true, 128, EPI_SWIGLU_BWD, GROUP_M, false>(A, B, p, s);       \
     case GK_DGRAD1:                                                                                \
-      if (bn == 256) return launch_impl<ES_, false, true, 256, EPI_STORE, GROUP_M, false>(A, B, p, s); \
+      if (bn == 256) return launch_impl<ES_, false, true, 256, EPI_STORE, GROUP_M, true>(A, B, p, s);  \
       return launch_impl<ES_, false, true, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);            \
     case GK_WGRAD:                                                                                 \
       if (bn == 256) return launch_impl<ES_, true, true, 256, EPI_STORE, GROUP_K, false>(A, B, p, s); \
