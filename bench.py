@@ -56,6 +56,15 @@ def load_peaks():
 # algorithmic work per op (bytes moved once, flops of the definition); R = routed rows = T*k
 # ------------------------------------------------------------------------------------------------
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, from ncu captures of the
+# current kernels on the full-size workload (profiles/grouped_gemm_fwd1_e128_bf16.md,
+# profiles/grouped_gemm_wgrad1_e128_bf16.md). A kernel or workload not listed reports null.
+MEASURED_TRAFFIC = {
+    ("e128_bf16", "gemm_fwd1_swiglu"): 1.235260e9 + 0.198228e9,
+    ("e128_bf16", "gemm_wgrad1"): 0.286070e9 + 1.015937e9,
+}
+
+
 def op_work_mx(w):
     """Per-op algorithmic (bytes, flops) of the MXFP8 layer step: fp8 codes + 1/32 scale bytes for GEMM
     operands, bf16 for everything stored."""
@@ -521,12 +530,13 @@ def main():
     t_dom = per_op[dom] / 1e3
     if b / (bw * 1e9) >= f / (tc * 1e12) or f == 0:
         roof = {"kernel": dom, "bound": "hbm", "achieved": b / t_dom / 1e9, "peak": bw, "unit": "GB/s",
-                "frac": (b / t_dom / 1e9) / bw, "traffic": None,
+                "frac": (b / t_dom / 1e9) / bw, "traffic": MEASURED_TRAFFIC.get((w.name, dom)),
                 "algorithmic_bytes": b, "flops": f, "ms": per_op[dom],
                 "peak_source": f"{peaks['source']} hbm_gbs"}
     else:
         roof = {"kernel": dom, "bound": "tensor", "achieved": f / t_dom / 1e12, "peak": tc,
-                "unit": "TFLOP/s", "frac": (f / t_dom / 1e12) / tc, "traffic": None,
+                "unit": "TFLOP/s", "frac": (f / t_dom / 1e12) / tc,
+                "traffic": MEASURED_TRAFFIC.get((w.name, dom)),
                 "algorithmic_bytes": b, "flops": f, "ms": per_op[dom],
                 "peak_source": f"{peaks['source']} bf16_tflops (burst) x {ratio} ({w.dtype})"}
 

@@ -13,6 +13,9 @@ pytestmark = pytest.mark.gpu
 SHAPES = {
     # name: (T, d, F, E, k, counts or None for uniform routing)
     "ragged": (512, 128, 256, 8, 2, [0, 1, 31, 33, 129, 200, 300, 330]),
+    # d, F >= 256: fwd2 and dgrad1 run on CTA pairs (256-row tiles) over uneven groups, so tiles
+    # with an empty second half, single-row and empty experts all occur
+    "ragged_pairs": (512, 256, 256, 8, 2, [0, 1, 31, 33, 129, 200, 300, 330]),
     "edges": (400, 192, 384, 6, 2, [32, 127, 128, 0, 400, 113]),
     "one_expert": (300, 128, 128, 4, 1, [300, 0, 0, 0]),
     "wide": (2048, 2048, 1024, 16, 4, None),
