@@ -7,7 +7,8 @@ One step is the whole hot path over one batch: routing metadata, row-wise dispat
 SwiGLU, grouped GEMM2, combine, combine backward, GEMM2 dgrad + SwiGLU backward, GEMM2 wgrad, GEMM1
 dgrad, GEMM1 wgrad, token reduce (plus router scores / top-k / router backward for learned-router
 workloads). Inputs are resident in HBM when the timed region starts; the e2e figure repeats the
-measurement through the public layer API with host-resident inputs and outputs copied each step.
+measurement through the public layer API with host-resident inputs and outputs copied each step
+(on copy streams that overlap the neighbouring steps' compute).
 Rank 0 prints one JSON line.
 """
 from __future__ import annotations
@@ -554,49 +555,81 @@ def main():
               "tokens_per_s_including_it": world * w.T / ((ms_per_step + wq_ms) / 1e3),
               "note": "once per weight update (optimizer step), outside the timed layer step"}
 
-    # end to end through the public layer API: host inputs in, host results out, every step
+    # end to end through the public layer API: host inputs in, host results out, every step. The
+    # loop is the one a training job runs: step i+1's inputs are copied host -> device on one copy
+    # stream while step i computes (two device input buffers), and step i's out / dx are read back
+    # on another copy stream while the next step's work proceeds; the layer's own buffers are only
+    # rewritten after their read-back has finished.
     e2e = None
     if not args.no_e2e:
         hx = inp["x"].cpu().pin_memory()
         hd = inp["dout"].cpu().pin_memory()
         hi = inp["idx"].cpu().pin_memory() if not learned else None
         hg = inp["gates"].cpu().pin_memory() if not learned else None
-        dx_in = torch.empty_like(inp["x"])
-        dd_in = torch.empty_like(inp["dout"])
-        di = torch.empty_like(inp["idx"]) if not learned else None
-        dgt = torch.empty_like(inp["gates"]) if not learned else None
+        bx = [torch.empty_like(inp["x"]) for _ in range(2)]
+        bd = [torch.empty_like(inp["dout"]) for _ in range(2)]
+        bi = [torch.empty_like(inp["idx"]) for _ in range(2)] if not learned else [None, None]
+        bg = [torch.empty_like(inp["gates"]) for _ in range(2)] if not learned else [None, None]
         ho = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
         hdx = torch.empty(layer.dx.shape, dtype=layer.dx.dtype).pin_memory()
         h2d = hx.numel() * hx.element_size() + hd.numel() * hd.element_size()
         if not learned:
             h2d += hi.numel() * 4 + hg.numel() * 4
         d2h = ho.numel() * ho.element_size() + hdx.numel() * hdx.element_size()
+        comp = torch.cuda.current_stream()
+        up, down = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()
+        loaded, consumed = [ev(), ev()], [ev(), ev()]
+        out_read, dx_read, fwd_done, bwd_done = ev(), ev(), ev(), ev()
 
-        def e2e_step():
-            dx_in.copy_(hx, non_blocking=True)
-            dd_in.copy_(hd, non_blocking=True)
-            if not learned:
-                di.copy_(hi, non_blocking=True)
-                dgt.copy_(hg, non_blocking=True)
-            layer.forward(dx_in, bias=inp["bias"], idx=di, gates=dgt)
-            layer.backward(dd_in)
-            ho.copy_(layer.out, non_blocking=True)
-            hdx.copy_(layer.dx, non_blocking=True)
+        def upload(j):
+            with torch.cuda.stream(up):
+                up.wait_event(consumed[j])  # the step that last used buffer j has finished with it
+                bx[j].copy_(hx, non_blocking=True)
+                bd[j].copy_(hd, non_blocking=True)
+                if not learned:
+                    bi[j].copy_(hi, non_blocking=True)
+                    bg[j].copy_(hg, non_blocking=True)
+                loaded[j].record(up)
 
-        for _ in range(args.warmup):
-            e2e_step()
+        def e2e_run(n):
+            upload(0)
+            for i in range(n):
+                j = i % 2
+                comp.wait_event(loaded[j])
+                if i + 1 < n:
+                    upload(1 - j)
+                comp.wait_event(out_read)  # the previous step's out has been read back
+                layer.forward(bx[j], bias=inp["bias"], idx=bi[j], gates=bg[j])
+                fwd_done.record(comp)
+                with torch.cuda.stream(down):
+                    down.wait_event(fwd_done)
+                    ho.copy_(layer.out, non_blocking=True)
+                    out_read.record(down)
+                comp.wait_event(dx_read)
+                layer.backward(bd[j])
+                consumed[j].record(comp)
+                bwd_done.record(comp)
+                with torch.cuda.stream(down):
+                    down.wait_event(bwd_done)
+                    hdx.copy_(layer.dx, non_blocking=True)
+                    dx_read.record(down)
+            comp.wait_event(dx_read)  # the timed region ends with the last result on the host
+
+        e2e_run(args.warmup)
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record()
+        e0.record(comp)
+        e2e_run(args.steps)
+        e1.record(comp)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), "cuda")
         e2e = {"value": world * w.T / (ems / args.steps / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": ems / args.steps, "api": "MoELayer.forward/backward -> moe_layer_fwd/bwd"}
+               "ms_per_step": ems / args.steps,
+               "api": "MoELayer.forward/backward -> moe_layer_fwd/bwd; copies on two streams overlap "
+                      "the neighbouring steps' compute"}
         assert torch.equal(ho.cuda(), ref[0]) and torch.equal(hdx.cuda(), ref[1])
 
     cpu = None
