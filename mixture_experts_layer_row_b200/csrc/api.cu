@@ -41,8 +41,30 @@ inline int64_t max_rows_of(const moe_config_t* c) {
   return ((int64_t)c->T * c->k + (a - 1) * c->E + a - 1) / a * a;
 }
 
+// The router weight gradient dW_r = dlogits^T x has only ceil(E/128) x ceil(d/BN) output tiles, too
+// few to fill the GPU, so its contraction over the T tokens is split into `n` chunks of `rows` rows
+// (a multiple of 32, at least 256) that run as separate tiles; their fp32 partial products are then
+// summed in a fixed order. Aim: about one tile per SM of a 148-SM part.
+struct RouterSplit {
+  int n, rows;
+  int slab_rows;  // rows of one split's fp32 partial: E rounded up to the 32-row store box
+};
+
+RouterSplit router_split(const moe_config_t* c) {
+  const int bn = c->d >= 256 ? 256 : 128;
+  const int tiles = ((c->E + 127) / 128) * ((c->d + bn - 1) / bn);
+  int n = (148 + tiles - 1) / tiles;
+  const int max_n = c->T / 256;
+  if (n > max_n) n = max_n;
+  const int slab = (c->E + 31) / 32 * 32;
+  if (n < 2) return {1, c->T, slab};
+  int rows = (c->T + n - 1) / n;
+  rows = (rows + 31) / 32 * 32;
+  return {(c->T + rows - 1) / rows, rows, slab};
+}
+
 struct WsLayout {
-  size_t head, hist, dlsel, dlogits, total;
+  size_t head, hist, dlsel, dlogits, rpart, total;
 };
 
 WsLayout ws_layout(const moe_config_t* c) {
@@ -51,7 +73,9 @@ WsLayout ws_layout(const moe_config_t* c) {
   w.hist = kWsHeadBytes;
   w.dlsel = w.hist + round256(metadata_ws_bytes(c->T, c->E));
   w.dlogits = w.dlsel + round256((size_t)c->T * c->k * sizeof(float));
-  w.total = w.dlogits + round256((size_t)c->T * c->E * es_of(c));
+  w.rpart = w.dlogits + round256((size_t)c->T * c->E * es_of(c));
+  const RouterSplit rs = router_split(c);
+  w.total = w.rpart + (rs.n > 1 ? round256((size_t)rs.n * rs.slab_rows * c->d * sizeof(float)) : 0);
   return w;
 }
 
@@ -209,9 +233,21 @@ int router_wgrad_impl(const moe_config_t* c, const void* dlogits, const void* x,
   GemmParams p = base_params(c, ws);
   p.counts = nullptr;
   p.M = c->E; p.N = c->d; p.K = c->T;
-  p.C = dWr; p.ldc = c->d; p.c_group_stride = 0;
+  p.ldc = c->d; p.c_group_stride = 0;
   GemmOperand a{dlogits, c->T, c->E, c->E}, b{x, c->T, c->d, c->d};
-  return launch_gemm(GK_WGRAD, es_of(c), c->d >= 256 ? 256 : 128, a, b, p, s);
+  const int bn = c->d >= 256 ? 256 : 128;
+  const RouterSplit rs = router_split(c);
+  if (rs.n < 2) {
+    p.C = dWr;
+    return launch_gemm(GK_WGRAD, es_of(c), bn, a, b, p, s);
+  }
+  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + ws_layout(c).rpart);
+  p.C = part;
+  p.ksplit = rs.rows;
+  p.c_group_rows = rs.slab_rows;
+  MOE_TRY(launch_gemm(GK_WGRAD_SPLIT, es_of(c), bn, a, b, p, s));
+  return launch_split_reduce(part, rs.n, (int64_t)c->E * c->d, (int64_t)rs.slab_rows * c->d, dWr,
+                             es_of(c) == 2, s);
 }
 
 bool router_shape_ok(const moe_config_t* c) {

@@ -99,6 +99,13 @@ struct TileInfo {
   int row_base; // GROUP_M: poff[e]
 };
 
+// GROUP_K: number of output groups (experts, contraction splits, or one)
+__host__ __device__ __forceinline__ int k_groups(const GemmParams& p) {
+  if (p.counts) return p.E;
+  if (p.ksplit) return (p.K + p.ksplit - 1) / p.ksplit;
+  return 1;
+}
+
 template <class C, int MODE>
 __device__ __forceinline__ int num_kstages(const TileInfo& ti) {
   if constexpr (MODE == GROUP_M) return ti.nchunks;
@@ -140,6 +147,9 @@ __device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const i
     if (p.counts) {
       ti.kstart = p.poff[e];
       ti.nchunks = (p.poff[e + 1] - p.poff[e]) / 32;
+    } else if (p.ksplit) {
+      ti.kstart = e * p.ksplit;
+      ti.nchunks = (min(p.ksplit, p.K - ti.kstart) + 31) / 32;
     } else {
       ti.kstart = 0;
       ti.nchunks = (p.K + 31) / 32;
@@ -285,7 +295,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
   } else {
     n_tiles = (p.N + BN - 1) / BN;
     m_tiles_fixed = (p.M + C::TILE_M - 1) / C::TILE_M;
-    total = (p.counts ? p.E : 1) * m_tiles_fixed * n_tiles;
+    total = k_groups(p) * m_tiles_fixed * n_tiles;
   }
 
   if (threadIdx.x == 0) {
@@ -607,7 +617,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       const int m_cta = ti.m0 + (int)rank * BM;             // this CTA's first tile row
       const bool active = (m_cta + q * 32) < ti.rows;       // warp-uniform
       int c1;                                               // tensor row of this slab
-      if constexpr (MODE == GROUP_K) c1 = ti.e * p.M + m_cta + q * 32;
+      if constexpr (MODE == GROUP_K) c1 = ti.e * (p.c_group_rows ? p.c_group_rows : p.M) + m_cta + q * 32;
       else c1 = ti.row_base + m_cta + q * 32;
       // Every variant walks the accumulator in 32-column chunks and keeps the TMEM load of the next
       // chunk in flight while it converts and stages the current one; CPB chunks fill one box.
@@ -903,7 +913,8 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   }
   // outputs: 32-row x 128-byte boxes stored from the epilogue's swizzled staging
   CUtensorMap tc, tc2;
-  const int64_t out_rows = (MODE == GROUP_K) ? (int64_t)(p.counts ? p.E : 1) * p.M : A.rows;
+  const int64_t out_rows =
+      (MODE == GROUP_K) ? (int64_t)k_groups(p) * (p.c_group_rows ? p.c_group_rows : p.M) : A.rows;
   const int64_t out_cols = (EPI == EPI_SWIGLU_FWD || EPI == EPI_SWIGLU_BWD) ? 2 * (int64_t)p.F : p.N;
   if (!make_tmap(&tc, p.C, C::OES, out_rows, out_cols, p.ldc, C::OEPR, 32, 2)) return MOE_ERR_CUDA;
   tc2 = tc;
@@ -913,7 +924,7 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   // knows it (GROUP_K: fixed tiles per group)
   int64_t cap = 0;
   if (MODE == GROUP_K) {
-    cap = (int64_t)(p.counts ? p.E : 1) * ((p.M + C::TILE_M - 1) / C::TILE_M) * ((p.N + BN - 1) / BN);
+    cap = (int64_t)k_groups(p) * ((p.M + C::TILE_M - 1) / C::TILE_M) * ((p.N + BN - 1) / BN);
     if (cap < 1) cap = 1;
   }
   if constexpr (PAIR) {
@@ -978,6 +989,10 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
       if (bn == 256)                                                                               \
         return launch_impl<ES_, false, false, 256, EPI_STORE_F32_BIAS, GROUP_M, false>(A, B, p, s); \
       return launch_impl<ES_, false, false, 128, EPI_STORE_F32_BIAS, GROUP_M, false>(A, B, p, s);  \
+    case GK_WGRAD_SPLIT:  /* fp32 partial products, no bias */                                     \
+      if (bn == 256)                                                                               \
+        return launch_impl<ES_, true, true, 256, EPI_STORE_F32_BIAS, GROUP_K, false>(A, B, p, s);  \
+      return launch_impl<ES_, true, true, 128, EPI_STORE_F32_BIAS, GROUP_K, false>(A, B, p, s);    \
   }
   if (es == 2) {
     MOE_GEMM_CASES(2)
@@ -1008,6 +1023,34 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
   }
 #undef MOE_GEMM_CASES
   return MOE_ERR_UNSUPPORTED;
+}
+
+// Sum of the split-contraction partials (fp32, fixed order), rounded to the output dtype.
+__global__ void __launch_bounds__(256) split_reduce_kernel(const float4* __restrict__ part, int nsplit,
+                                                           int64_t n4, int64_t stride4,
+                                                           void* __restrict__ out, int bf16) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 acc = part[i];
+    for (int s = 1; s < nsplit; ++s) {
+      const float4 v = part[(int64_t)s * stride4 + i];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    if (bf16) reinterpret_cast<uint2*>(out)[i] = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+    else reinterpret_cast<float4*>(out)[i] = acc;
+  }
+}
+
+int launch_split_reduce(const float* part, int nsplit, int64_t n, int64_t stride, void* out, bool bf16,
+                        cudaStream_t s) {
+  if (n % 4 != 0 || stride % 4 != 0 || stride < n || nsplit < 1) return MOE_ERR_UNSUPPORTED;
+  const int64_t n4 = n / 4;
+  int64_t blocks = (n4 + 255) / 256;
+  if (blocks > 4 * (int64_t)sm_count()) blocks = 4 * (int64_t)sm_count();
+  split_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(part), nsplit, n4,
+                                                        stride / 4, out, bf16 ? 1 : 0);
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 // Bounded-wait self-test: wait on a barrier nobody arrives at.

@@ -9,7 +9,9 @@ namespace moe {
 enum { EPI_STORE = 0, EPI_SWIGLU_FWD = 1, EPI_SWIGLU_BWD = 2, EPI_STORE_F32_BIAS = 3 };
 enum { GROUP_M = 0, GROUP_K = 1 };
 
-enum GemmKind { GK_FWD1_SWIGLU, GK_FWD2, GK_DGRAD2_SWIGLU, GK_DGRAD1, GK_WGRAD, GK_ROUTER };
+// GK_WGRAD_SPLIT: single-group wgrad with the contraction split into chunks of ksplit rows, one fp32
+// partial product per chunk (summed afterwards by launch_split_reduce).
+enum GemmKind { GK_FWD1_SWIGLU, GK_FWD2, GK_DGRAD2_SWIGLU, GK_DGRAD1, GK_WGRAD, GK_ROUTER, GK_WGRAD_SPLIT };
 
 // A row-major 2-D operand as the TMA unit sees it.
 struct GemmOperand {
@@ -45,6 +47,11 @@ struct GemmParams {
   // MN-major operands whose column count is a whole number of 128-byte blocks are loaded as one
   // 3-D box per stage (set by the launcher); otherwise as 32-row x 128-byte 2-D boxes.
   int a_box3d, b_box3d;
+  // GROUP_K without groups: contraction rows per split (0 = one split); split s writes C rows
+  // [s*c_group_rows, s*c_group_rows + M). c_group_rows (0 = M) is M rounded up to the 32-row store
+  // box when M is not a multiple of 32, so a box never reaches into the next split's rows.
+  int ksplit;
+  int c_group_rows;
 };
 
 // Host-side count of kernels enqueued (every launcher adds the kernels it launched).
@@ -66,6 +73,9 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
 int launch_quantize(const void* src, int64_t rows, int cols, int mode, int64_t G, uint8_t* q,
                     uint8_t* s, cudaStream_t st);
 int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s);
+// out[i] = round_to_act(sum over s < nsplit of part[s*stride + i]) for i < n (fixed summation order).
+int launch_split_reduce(const float* part, int nsplit, int64_t n, int64_t stride, void* out, bool bf16,
+                        cudaStream_t s);
 
 int launch_topk(const float* logits, const float* bias, int T, int E, int k, int renorm, int32_t* idx,
                 float* gates, uint32_t* err, cudaStream_t s);

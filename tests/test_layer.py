@@ -128,6 +128,12 @@ def _sampled_full_size(w: Workload, n_tok=24, n_exp=2):
             assert_close_rel(g2, dW2, TOL_BF16, f"dW2[{e}]")
         else:
             assert np.all(g13 == 0) and np.all(g2 == 0)
+    if learned:
+        # the router weight gradient at full size (its contraction over T is split into token
+        # chunks on the GPU): dW_r = dlogits^T x, with dlogits from the GPU's gate gradients by the
+        # oracle's router backward
+        dl = O.router_bwd(layer.dgates.cpu().double().numpy(), gates_ref, idx, w.E)
+        assert_close_rel(np64(layer.dW_r), dl.T @ x64, TOL_BF16, "dW_r")
     return layer
 
 
