@@ -89,15 +89,30 @@ struct Cfg {
       STAGING_BYTES;
 };
 
+// One tile of the device schedule. lo / hi are the group's row range as read from the routing
+// metadata: GROUP_M the group's padded routed rows [lo, hi), GROUP_K its contraction rows [lo, hi).
+// They are kept raw, so that a role can fetch the next tile's entry while it works on the current
+// one and only use the loaded values a tile later (the loads then never stall the loop).
 struct TileInfo {
-  int e;        // group
-  int m0;       // GROUP_M: first row (relative to the group start); GROUP_K: first output row
-  int n0;       // first output column
-  int rows;     // GROUP_M: valid rows of the group (padded count); GROUP_K: M
-  int kstart;   // GROUP_M: unused; GROUP_K: first contraction row in the routed buffer
-  int nchunks;  // number of 32-row K chunks (GROUP_K) or K/BK stages (GROUP_M)
-  int row_base; // GROUP_M: poff[e]
+  int e;   // group
+  int m0;  // GROUP_M: first row relative to the group start; GROUP_K: first output row
+  int n0;  // first output column
+  int lo, hi;
 };
+
+template <int MODE>
+__device__ __forceinline__ int ti_rows(const TileInfo& ti, const GemmParams& p) {
+  return MODE == GROUP_M ? ti.hi - ti.lo : p.M;  // GROUP_M: padded rows of the group
+}
+__device__ __forceinline__ int ti_row_base(const TileInfo& ti) { return ti.lo; }  // GROUP_M
+__device__ __forceinline__ int ti_kstart(const TileInfo& ti) { return ti.lo; }    // GROUP_K
+
+// K stages of a tile: GROUP_M K/BK; GROUP_K the group's 32-row contraction chunks, CHUNKS per stage
+template <class C, int MODE>
+__device__ __forceinline__ int ti_nchunks(const TileInfo& ti, const GemmParams& p) {
+  if constexpr (MODE == GROUP_M) return p.K / C::BK;
+  else return (ti.hi - ti.lo + 31) / 32;
+}
 
 // GROUP_K: number of output groups (experts, contraction splits, or one)
 __host__ __device__ __forceinline__ int k_groups(const GemmParams& p) {
@@ -107,9 +122,14 @@ __host__ __device__ __forceinline__ int k_groups(const GemmParams& p) {
 }
 
 template <class C, int MODE>
-__device__ __forceinline__ int num_kstages(const TileInfo& ti) {
-  if constexpr (MODE == GROUP_M) return ti.nchunks;
-  else return (ti.nchunks + C::CHUNKS - 1) / C::CHUNKS;
+__device__ __forceinline__ int num_kstages(const TileInfo& ti, const GemmParams& p) {
+  if constexpr (MODE == GROUP_M) return ti_nchunks<C, MODE>(ti, p);
+  else return (ti_nchunks<C, MODE>(ti, p) + C::CHUNKS - 1) / C::CHUNKS;
+}
+
+// GROUP_M: m-tiles of group e, from the shared-memory tile prefix (no global load)
+__device__ __forceinline__ int prefix_m_tiles(const int* prefix, int e, int n_tiles) {
+  return (prefix[e + 1] - prefix[e]) / n_tiles;
 }
 
 template <class C, int EPI, int MODE>
@@ -126,15 +146,17 @@ __device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const i
       e = lo;
     }
     const int local = tile - prefix[e];
-    const int rows = p.counts ? (p.poff[e + 1] - p.poff[e]) : p.M;
-    const int mt = (rows + C::TILE_M - 1) / C::TILE_M;
+    const int mt = prefix_m_tiles(prefix, e, n_tiles);
     ti.e = e;
     ti.n0 = (local / mt) * C::BN_OUT;
     ti.m0 = (local % mt) * C::TILE_M;
-    ti.rows = rows;
-    ti.row_base = p.counts ? p.poff[e] : 0;
-    ti.kstart = 0;
-    ti.nchunks = p.K / C::BK;
+    if (p.counts) {
+      ti.lo = p.poff[e];
+      ti.hi = p.poff[e + 1];
+    } else {
+      ti.lo = 0;
+      ti.hi = p.M;
+    }
   } else {
     const int per = m_tiles_fixed * n_tiles;
     const int e = tile / per;
@@ -142,17 +164,15 @@ __device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const i
     ti.e = e;
     ti.m0 = (local / n_tiles) * C::TILE_M;
     ti.n0 = (local % n_tiles) * C::TILE_N;
-    ti.rows = p.M;
-    ti.row_base = 0;
     if (p.counts) {
-      ti.kstart = p.poff[e];
-      ti.nchunks = (p.poff[e + 1] - p.poff[e]) / 32;
+      ti.lo = p.poff[e];
+      ti.hi = p.poff[e + 1];
     } else if (p.ksplit) {
-      ti.kstart = e * p.ksplit;
-      ti.nchunks = (min(p.ksplit, p.K - ti.kstart) + 31) / 32;
+      ti.lo = e * p.ksplit;
+      ti.hi = min(p.K, ti.lo + p.ksplit);
     } else {
-      ti.kstart = 0;
-      ti.nchunks = (p.K + 31) / 32;
+      ti.lo = 0;
+      ti.hi = p.K;
     }
   }
 }
@@ -346,11 +366,13 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       // loaded (its accumulator rows are never stored).
       int it = 0;
       bool ok = true;
+      TileInfo nxt;  // the next tile's entry is fetched a tile ahead
+      if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, prefix, n_tiles, m_tiles_fixed, nxt);
       for (int tile = tile0; tile < total && ok; tile += tstep) {
-        TileInfo ti;
-        tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
-        const int nst = num_kstages<C, MODE>(ti);
-        const bool a0 = ti.m0 < ti.rows, a1 = ti.m0 + BM < ti.rows;
+        const TileInfo ti = nxt;
+        if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
+        const int nst = num_kstages<C, MODE>(ti, p);
+        const bool a0 = ti.m0 < ti_rows<MODE>(ti, p), a1 = ti.m0 + BM < ti_rows<MODE>(ti, p);
         const bool mine = rank == 0 ? a0 : a1;
         const uint32_t tx = (a0 ? C::A_BYTES : 0) + (a1 ? C::A_BYTES : 0) + 2 * C::B_BYTES;
         const int m_cta = ti.m0 + (int)rank * BM;
@@ -368,7 +390,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           if (rank == 0) mbar_arrive_expect_tx(&full[s], tx);
           if constexpr (MODE == GROUP_M) {
             const int k0 = ks * C::BK;
-            if (mine) tma_load_2d_pair(a_dst, &tmA, fb, k0, ti.row_base + m_cta);
+            if (mine) tma_load_2d_pair(a_dst, &tmA, fb, k0, ti_row_base(ti) + m_cta);
             const int brow = ti.e * p.b_rows_per_group;
             if constexpr (B_MN) {
               tma_load_3d_pair(b_dst, &tmB, fb, 0, brow + k0, n_cta / C::EPR);
@@ -379,7 +401,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               tma_load_2d_pair(b_dst, &tmB, fb, k0, brow + n_cta);
             }
           } else {
-            const int krow0 = ti.kstart + ks * C::CHUNKS * 32;
+            const int krow0 = ti_kstart(ti) + ks * C::CHUNKS * 32;
             if (mine) tma_load_3d_pair(a_dst, &tmA, fb, 0, krow0, m_cta / C::EPR);
             tma_load_3d_pair(b_dst, &tmB, fb, 0, krow0, n_cta / C::EPR);
           }
@@ -392,10 +414,12 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     } else if (lane == 0) {
       int it = 0;
       bool ok = true;
+      TileInfo nxt;  // the next tile's entry is fetched a tile ahead
+      if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, prefix, n_tiles, m_tiles_fixed, nxt);
       for (int tile = tile0; tile < total && ok; tile += tstep) {
-        TileInfo ti;
-        tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
-        const int nst = num_kstages<C, MODE>(ti);
+        const TileInfo ti = nxt;
+        if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
+        const int nst = num_kstages<C, MODE>(ti, p);
         for (int ks = 0; ks < nst; ++ks, ++it) {
           const int s = it % C::STAGES;
           if (!mbar_wait_bounded(&empty[s], ((it / C::STAGES) & 1) ^ 1, p.wait_limit_ns, abort_word,
@@ -414,7 +438,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             uint8_t* sf = sfs + (size_t)s * C::SF_BYTES;
             int64_t amb, akq, bmb, bkq;
             if constexpr (MODE == GROUP_M) {
-              amb = ((int64_t)ti.row_base + ti.m0) >> 7;
+              amb = ((int64_t)ti_row_base(ti) + ti.m0) >> 7;
               akq = ks;
               if constexpr (B_MN) {
                 bmb = ti.n0 >> 7;
@@ -429,7 +453,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             } else {
               amb = ti.m0 >> 7;
               bmb = ti.n0 >> 7;
-              akq = bkq = (ti.kstart >> 7) + ks;
+              akq = bkq = (ti_kstart(ti) >> 7) + ks;
             }
             sf_a = p.sA + (amb * p.sA_ld + akq) * 512;
             sf_b = p.sB + (bmb * p.sB_ld + bkq) * 512;
@@ -448,7 +472,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
                 bulk_load(sf_dst + 512 * (c + 1), sf_b + (int64_t)c * b_chunk_step, 512, &full[s]);
             }
             // A: K-major rows of the routed buffer (or the token matrix)
-            tma_load_2d(a_dst, &tmA, &full[s], k0, ti.row_base + ti.m0);
+            tma_load_2d(a_dst, &tmA, &full[s], k0, ti_row_base(ti) + ti.m0);
             if constexpr (!B_MN) {
               const int brow = ti.e * p.b_rows_per_group;
               if constexpr (EPI == EPI_SWIGLU_FWD) {
@@ -476,8 +500,8 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             // brings BK rows; in the group's last stage the rows past its end (the next group's, or
             // zero fill past the tensor) land in shared memory but the MMA loop stops before them.
             const int c0 = ks * C::CHUNKS;
-            const int nch = min(C::CHUNKS, ti.nchunks - c0);
-            const int krow0 = ti.kstart + c0 * 32;
+            const int nch = min(C::CHUNKS, ti_nchunks<C, MODE>(ti, p) - c0);
+            const int krow0 = ti_kstart(ti) + c0 * 32;
             const uint32_t a_bytes = p.a_box3d ? C::A_BYTES : nch * 32 * 128 * (BM / C::EPR);
             const uint32_t b_bytes = p.b_box3d ? C::B_BYTES : nch * 32 * 128 * (BN / C::EPR);
             mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes + C::SF_BYTES);
@@ -520,10 +544,12 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       int it = 0, local = 0;
       bool ok = true;
       bool issued = false;
+      TileInfo nxt;  // the next tile's entry is fetched a tile ahead
+      if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, prefix, n_tiles, m_tiles_fixed, nxt);
       for (int tile = tile0; tile < total && ok; tile += tstep, ++local) {
-        TileInfo ti;
-        tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
-        const int nst = num_kstages<C, MODE>(ti);
+        const TileInfo ti = nxt;
+        if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
+        const int nst = num_kstages<C, MODE>(ti, p);
         const int buf = local % C::NACC;
         const uint32_t use = (uint32_t)(local / C::NACC) & 1u;  // parity of this buffer's use
         const bool drained =
@@ -545,7 +571,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           const uint32_t a_addr = smem_u32(smA + (size_t)s * C::A_BYTES);
           const uint32_t b_addr = smem_u32(smB + (size_t)s * C::B_BYTES);
           int nk = C::KSTEPS;
-          if constexpr (MODE == GROUP_K) nk = min(C::CHUNKS, ti.nchunks - ks * C::CHUNKS) * (32 / C::UK);
+          if constexpr (MODE == GROUP_K) nk = min(C::CHUNKS, ti_nchunks<C, MODE>(ti, p) - ks * C::CHUNKS) * (32 / C::UK);
           uint32_t sf_col = 0;
           if constexpr (C::MX) {
             // this stage's scales: smem chunks -> TMEM columns after the two accumulators
@@ -601,10 +627,12 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     uint8_t* wstg = stg + (size_t)q * C::NBUF * 4096;
     int nb = 0;                           // next staging box (round robin)
     int local = 0;
+    TileInfo nxt;  // the next tile's entry is fetched a tile ahead
+    if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, prefix, n_tiles, m_tiles_fixed, nxt);
     for (int tile = tile0; tile < total; tile += tstep, ++local) {
-      TileInfo ti;
-      tile_info<C, EPI, MODE>(tile, p, prefix, n_tiles, m_tiles_fixed, ti);
-      const int nst = num_kstages<C, MODE>(ti);
+      const TileInfo ti = nxt;
+      if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
+      const int nst = num_kstages<C, MODE>(ti, p);
       const int buf = local % C::NACC;
       int ok = 1;
       if (lane == 0)
@@ -615,10 +643,10 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
       const int m_cta = ti.m0 + (int)rank * BM;             // this CTA's first tile row
-      const bool active = (m_cta + q * 32) < ti.rows;       // warp-uniform
+      const bool active = (m_cta + q * 32) < ti_rows<MODE>(ti, p);       // warp-uniform
       int c1;                                               // tensor row of this slab
       if constexpr (MODE == GROUP_K) c1 = ti.e * (p.c_group_rows ? p.c_group_rows : p.M) + m_cta + q * 32;
-      else c1 = ti.row_base + m_cta + q * 32;
+      else c1 = ti_row_base(ti) + m_cta + q * 32;
       // Every variant walks the accumulator in 32-column chunks and keeps the TMEM load of the next
       // chunk in flight while it converts and stages the current one; CPB chunks fill one box.
       constexpr int CPB = C::OEPR / 32;
@@ -672,7 +700,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
         constexpr int NCH = BN / 32;
         constexpr int RW = 2 * C::OES;  // 16-byte words per 32 stored values
         const char* hrow = reinterpret_cast<const char*>(p.aux) +
-                           ((size_t)ti.row_base + m_cta + q * 32 + lane) * p.ldaux * C::OES;
+                           ((size_t)ti_row_base(ti) + m_cta + q * 32 + lane) * p.ldaux * C::OES;
         if (active) {
           uint32_t da[32], db[32];
           uint4 gwa[RW], uwa[RW], gwb[RW], uwb[RW];
