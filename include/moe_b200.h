@@ -89,8 +89,8 @@ typedef struct {
  * Returns 0 for an invalid config. */
 MOE_API int64_t moe_max_rows(const moe_config_t* cfg);
 
-/* Bytes of scratch the layer-level calls need (routing histograms, router-gradient scratch and the
- * sticky error flag). The first call on a fresh workspace must be preceded by moe_clear_error (or a
+/* Bytes of scratch the layer-level calls need (routing histograms, router-gradient scratch incl.
+ * the router weight gradient's fp32 partials, and the sticky error flag). The first call on a fresh workspace must be preceded by moe_clear_error (or a
  * zero fill of the buffer) so that the flag starts at 0. Returns MOE_ERR_INVALID_ARG on a bad cfg. */
 MOE_API int moe_workspace_size(const moe_config_t* cfg, size_t* bytes /* host */);
 
@@ -209,7 +209,9 @@ MOE_API int moe_grouped_gemm(const moe_config_t* cfg, int op, const void* A, con
                      size_t ws_bytes, void* stream);
 
 /* Router weight gradient dW_r = dlogits^T x (act [E,d]) from the dense score gradient written by
- * moe_combine_bwd (act [T,E]); a single-group tensor-core GEMM contracting over tokens. */
+ * moe_combine_bwd (act [T,E]); a tensor-core GEMM contracting over tokens. When its output tiles are
+ * too few to fill the GPU, the token range is split into chunks whose fp32 partial products go to
+ * the workspace and are summed in a fixed order (deterministic). ws as for moe_workspace_size. */
 MOE_API int moe_router_wgrad(const moe_config_t* cfg, const void* dlogits, const void* x, void* dW_r,
                      void* ws, size_t ws_bytes, void* stream);
 

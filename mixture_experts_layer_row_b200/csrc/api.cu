@@ -104,7 +104,6 @@ GemmParams base_params(const moe_config_t* c, void* ws) {
   std::memset(&p, 0, sizeof(p));
   p.E = c->E;
   p.F = c->F;
-  p.vec_ok = 1;
   p.err = ws ? err_of(ws) : nullptr;
   p.wait_limit_ns = kWaitLimitNs;
   return p;
@@ -147,12 +146,12 @@ int gemm_op(const moe_config_t* c, int op, const void* A, const void* B, void* C
     case MOE_GEMM_WGRAD2:
       a = {A, R, d, d};
       b = {B, R, F, F};
-      p.M = d; p.N = F; p.ldc = F; p.c_group_stride = (int64_t)d * F;
+      p.M = d; p.N = F; p.ldc = F;
       return launch_gemm(GK_WGRAD, es, F >= 256 ? 256 : 128, a, b, p, s);
     case MOE_GEMM_WGRAD1:
       a = {A, R, 2 * F, 2 * F};
       b = {B, R, d, d};
-      p.M = 2 * F; p.N = d; p.ldc = d; p.c_group_stride = (int64_t)2 * F * d;
+      p.M = 2 * F; p.N = d; p.ldc = d;
       return launch_gemm(GK_WGRAD, es, d >= 256 ? 256 : 128, a, b, p, s);
     default:
       return MOE_ERR_INVALID_ARG;
@@ -203,13 +202,13 @@ int gemm_op_mx(const moe_config_t* c, int op, const uint8_t* Aq, const uint8_t* 
     case MOE_GEMM_WGRAD2:
       a = {Aq, R, d, d};
       b = {Bq, R, F, F};
-      p.M = d; p.N = F; p.ldc = F; p.c_group_stride = (int64_t)d * F;
+      p.M = d; p.N = F; p.ldc = F;
       p.sA_ld = R / 128; p.sB_ld = R / 128;
       return launch_gemm(GK_WGRAD, 1, 128, a, b, p, s);
     case MOE_GEMM_WGRAD1:
       a = {Aq, R, 2 * F, 2 * F};
       b = {Bq, R, d, d};
-      p.M = 2 * F; p.N = d; p.ldc = d; p.c_group_stride = (int64_t)2 * F * d;
+      p.M = 2 * F; p.N = d; p.ldc = d;
       p.sA_ld = R / 128; p.sB_ld = R / 128;
       return launch_gemm(GK_WGRAD, 1, 128, a, b, p, s);
     default:
@@ -223,7 +222,6 @@ int router_logits_impl(const moe_config_t* c, const void* x, const void* Wr, con
   p.counts = nullptr;
   p.M = c->T; p.K = c->d; p.N = c->E; p.b_rows_per_group = 0;
   p.C = logits; p.ldc = c->E; p.bias = bias;
-  p.vec_ok = (c->E % 4 == 0);
   GemmOperand a{x, c->T, c->d, c->d}, b{Wr, c->E, c->d, c->d};
   return launch_gemm(GK_ROUTER, es_of(c), c->E <= 128 ? 128 : 256, a, b, p, s);
 }
@@ -233,7 +231,7 @@ int router_wgrad_impl(const moe_config_t* c, const void* dlogits, const void* x,
   GemmParams p = base_params(c, ws);
   p.counts = nullptr;
   p.M = c->E; p.N = c->d; p.K = c->T;
-  p.ldc = c->d; p.c_group_stride = 0;
+  p.ldc = c->d;
   GemmOperand a{dlogits, c->T, c->E, c->E}, b{x, c->T, c->d, c->d};
   const int bn = c->d >= 256 ? 256 : 128;
   const RouterSplit rs = router_split(c);

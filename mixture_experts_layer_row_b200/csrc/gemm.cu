@@ -8,17 +8,19 @@
 //   warp 0      TMA producer: one elected thread streams A/B tiles into a STAGES-deep shared-memory
 //               ring (128-byte swizzle), completion counted on a "full" mbarrier per stage;
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, fp32 accumulate) into
-//               one of two TMEM accumulators and frees each ring stage with tcgen05.commit;
+//               one of NACC TMEM accumulators and frees each ring stage with tcgen05.commit;
 //   warps 2..5  epilogue: tcgen05.ld the finished accumulator (one row per thread), apply the fused
-//               op (store, SwiGLU forward, SwiGLU backward, fp32 + bias) and store to global memory,
-//               while the MMA thread already fills the other accumulator.
+//               op (store, SwiGLU forward, SwiGLU backward, fp32 + bias) and store to global memory
+//               with TMA, while the MMA thread already fills the other accumulator (NACC = 2; the
+//               256-column MXFP8 tiles have one, their scale columns filling the rest of TMEM).
 // The tile schedule is built on the device from the routing metadata (counts, padded offsets): the
 // host never learns the group sizes. Two grouping modes:
 //   GROUP_M  ragged rows per expert (forward and dgrad): tiles (expert, n-block, m-block), m fastest
 //            so CTAs running at the same time share the expert's weight block through L2;
 //   GROUP_K  ragged contraction per expert (wgrad): tiles (expert, m-block, n-block), the K loop runs
 //            over the expert's 32-aligned row range in 32-row chunks (zero pad rows make the tail
-//            exact); an expert with no rows writes a zero gradient.
+//            exact); an expert with no rows writes a zero gradient. Without experts, the same mode
+//            splits one long contraction into fixed chunks with one fp32 partial each (router dW_r).
 // CTA pairs (PAIR, a cluster of two CTAs on neighbouring SMs): a tile covers 256 rows; each CTA
 // loads its 128 rows of A and half of B's columns into its own shared memory (TMA with
 // .cta_group::2, completing on the leader's barrier, no multicast), the leader's MMA thread issues
@@ -574,7 +576,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           if constexpr (MODE == GROUP_K) nk = min(C::CHUNKS, ti_nchunks<C, MODE>(ti, p) - ks * C::CHUNKS) * (32 / C::UK);
           uint32_t sf_col = 0;
           if constexpr (C::MX) {
-            // this stage's scales: smem chunks -> TMEM columns after the two accumulators
+            // this stage's scales: smem chunks -> TMEM columns after the accumulator(s)
             sf_col = tmem_base + C::NACC * BN + s * C::SF_COLS;
             const uint32_t sf_smem = smem_u32(sfs + (size_t)s * C::SF_BYTES);
 #pragma unroll

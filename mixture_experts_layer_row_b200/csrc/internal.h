@@ -35,8 +35,6 @@ struct GemmParams {
   int64_t ldaux;
   const float* bias;
   int F;
-  int64_t c_group_stride;  // GROUP_K: elements between two groups' outputs
-  int vec_ok;              // output rows allow 16-byte vector stores
   // MXFP8 operands: UE8M0 scales in the tiled layout (512-byte chunks per 128 MN indices x 4
   // K-blocks); sA_ld / sB_ld = chunks per 128 MN indices (= K-blocks / 4 of that operand)
   const uint8_t* sA;
