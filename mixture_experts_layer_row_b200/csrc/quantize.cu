@@ -107,52 +107,44 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const uint4* __restrict_
   s[scale_index(layout, b / blocks_per_row, b % blocks_per_row, blocks_per_row, G)] = sb;
 }
 
-// One thread per (32-row block, 8 consecutive columns).
-__global__ void __launch_bounds__(256) quant_col_kernel(const uint4* __restrict__ src, int64_t rows,
-                                                        int cols, int layout, uint2* __restrict__ q,
+// One thread per (32-row block, 4 consecutive columns): the 32 8-byte row segments stay in registers
+// between the block-maximum pass and the conversion, so the source is read once (a warp covers 128
+// contiguous columns of each row).
+__global__ void __launch_bounds__(128) quant_col_kernel(const uint2* __restrict__ src, int64_t rows,
+                                                        int cols, int layout, uint32_t* __restrict__ q,
                                                         uint8_t* __restrict__ s) {
-  const int groups = cols / 8;
+  const int groups = cols / 4;
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t rblocks = rows / 32;
   if (t >= rblocks * groups) return;
   const int64_t rb = t / groups;
   const int cg = (int)(t % groups);
-  float amax[8];
+  const uint2* base = src + (rb * 32) * groups + cg;  // row stride = groups uint2
+  uint2 w[32];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) amax[j] = 0.f;
-  const uint4* base = src + (rb * 32) * groups + cg;  // row stride = groups uint4
-#pragma unroll 4
+  for (int r = 0; r < 32; ++r) w[r] = base[(int64_t)r * groups];
+  float amax[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
   for (int r = 0; r < 32; ++r) {
-    const uint4 w = base[(int64_t)r * groups];
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      amax[2 * j] = fmaxf(amax[2 * j], fabsf(bf16lo(u[j])));
-      amax[2 * j + 1] = fmaxf(amax[2 * j + 1], fabsf(bf16hi(u[j])));
-    }
+    amax[0] = fmaxf(amax[0], fabsf(bf16lo(w[r].x)));
+    amax[1] = fmaxf(amax[1], fabsf(bf16hi(w[r].x)));
+    amax[2] = fmaxf(amax[2], fabsf(bf16lo(w[r].y)));
+    amax[3] = fmaxf(amax[3], fabsf(bf16hi(w[r].y)));
   }
-  float inv[8];
+  float inv[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < 4; ++j) {
     uint8_t sb;
     const int e = block_exponent(amax[j], &sb);
     inv[j] = amax[j] > 0.f ? exp2_exact(-e) : 0.f;
-    s[scale_index(layout, (int64_t)cg * 8 + j, rb, rblocks, 0)] = sb;
+    s[scale_index(layout, (int64_t)cg * 4 + j, rb, rblocks, 0)] = sb;
   }
-  uint2* qb = q + (rb * 32) * groups + cg;
-#pragma unroll 4
-  for (int r = 0; r < 32; ++r) {
-    const uint4 w = base[(int64_t)r * groups];
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-    uint32_t c[2];
+  uint32_t* qb = q + (rb * 32) * groups + cg;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t lo = cvt_e4m3x2(bf16lo(u[2 * h]) * inv[4 * h], bf16hi(u[2 * h]) * inv[4 * h + 1]);
-      const uint32_t hi =
-          cvt_e4m3x2(bf16lo(u[2 * h + 1]) * inv[4 * h + 2], bf16hi(u[2 * h + 1]) * inv[4 * h + 3]);
-      c[h] = lo | (hi << 16);
-    }
-    qb[(int64_t)r * groups] = make_uint2(c[0], c[1]);
+  for (int r = 0; r < 32; ++r) {
+    const uint32_t lo = cvt_e4m3x2(bf16lo(w[r].x) * inv[0], bf16hi(w[r].x) * inv[1]);
+    const uint32_t hi = cvt_e4m3x2(bf16lo(w[r].y) * inv[2], bf16hi(w[r].y) * inv[3]);
+    qb[(int64_t)r * groups] = lo | (hi << 16);
   }
 }
 
@@ -172,10 +164,10 @@ int launch_quantize(const void* src, int64_t rows, int cols, int mode, int64_t G
     quant_row_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const uint4*>(src), nb, cols / 32,
                                                       layout, G, reinterpret_cast<uint4*>(q), s);
   } else {
-    const int64_t nt = (rows / 32) * (cols / 8);
-    const int64_t grid = (nt + 255) / 256;
-    quant_col_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const uint4*>(src), rows, cols,
-                                                      layout, reinterpret_cast<uint2*>(q), s);
+    const int64_t nt = (rows / 32) * (cols / 4);
+    const int64_t grid = (nt + 127) / 128;
+    quant_col_kernel<<<(unsigned)grid, 128, 0, st>>>(static_cast<const uint2*>(src), rows, cols,
+                                                      layout, reinterpret_cast<uint32_t*>(q), s);
   }
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
