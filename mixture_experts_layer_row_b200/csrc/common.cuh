@@ -265,6 +265,20 @@ __device__ __forceinline__ void tmem_regs_after(uint32_t (&r)[32]) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch. Every kernel of this library is launched with the stream's
+// programmatic serialisation allowed, so it may be scheduled while the previous kernel in the stream
+// is still finishing. pdl_trigger lets the next kernel be scheduled; pdl_wait blocks until the previous
+// kernel has completed and its memory is visible. Each kernel calls pdl_wait before its first global
+// memory access (read or write).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+  pdl_trigger();
+  pdl_wait();
+}
+
+// ---------------------------------------------------------------------------------------------
 // CTA pairs (thread-block cluster of 2, tcgen05 cta_group::2): the leader (rank 0) issues MMAs with
 // M = 256 whose A rows 0-127 and 128-255 and whose two halves of B sit in the two CTAs' shared
 // memory at the same offsets; each CTA's tensor memory holds its 128 accumulator rows.

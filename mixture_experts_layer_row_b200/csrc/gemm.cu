@@ -278,6 +278,41 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
   const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int tstep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  pdl_trigger();  // the next kernel may be scheduled as SMs free up
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      // single CTA: every epilogue thread arrives; pair: lane 0 of the 4 epilogue warps of each CTA
+      mbar_init(&tempty[b], PAIR ? 8 : kEpiThreads);
+    }
+    mbar_init(done, 1);
+    *abort_word = 0;
+    if constexpr (PAIR) fence_barrier_init_cluster();
+    else fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    prefetch_tensormap(&tmC);
+    if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmC2);
+  }
+  if (warp == 1) {
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
+  }
+  // Local setup above touches no global memory; wait here for the previous kernel in the stream
+  // (the routing metadata and operands it wrote) before building the schedule from it.
+  pdl_wait();
 
   // ---- device-side tile schedule ----
   int n_tiles, m_tiles_fixed = 0, total;
@@ -320,36 +355,6 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     total = k_groups(p) * m_tiles_fixed * n_tiles;
   }
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      // single CTA: every epilogue thread arrives; pair: lane 0 of the 4 epilogue warps of each CTA
-      mbar_init(&tempty[b], PAIR ? 8 : kEpiThreads);
-    }
-    mbar_init(done, 1);
-    *abort_word = 0;
-    if constexpr (PAIR) fence_barrier_init_cluster();
-    else fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&tmA);
-    prefetch_tensormap(&tmB);
-    prefetch_tensormap(&tmC);
-    if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmC2);
-  }
-  if (warp == 1) {
-    if constexpr (PAIR) {
-      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
-      tmem_relinquish_pair();
-    } else {
-      tmem_alloc(tmem_slot, C::TMEM_COLS);
-      tmem_relinquish();
-    }
-  }
   tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) cluster_sync();  // both CTAs' barriers exist before either signals the other
@@ -959,16 +964,18 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   }
   if constexpr (PAIR) {
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = 2;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = s;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1;  // occupancy query: cluster shape only
     if (!pair_slots[dev]) {
       cfg.gridDim = dim3(2 * (sm_count() / 2));
       int n = 0;
@@ -978,11 +985,12 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
     int64_t pairs = pair_slots[dev];
     if (cap > 0 && cap < pairs) pairs = cap;
     cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.numAttrs = 2;  // cluster shape + programmatic dependent launch
     if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tc2, q) != cudaSuccess) return MOE_ERR_CUDA;
   } else {
     int64_t grid = sm_count();
     if (cap > 0 && cap < grid) grid = cap;
-    kern<<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, tc, tc2, q);
+    MOE_LAUNCH(launch_pdl(kern, (unsigned)grid, C::THREADS, C::SMEM_BYTES, s, ta, tb, tc, tc2, q));
   }
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -1059,6 +1067,7 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
 __global__ void __launch_bounds__(256) split_reduce_kernel(const float4* __restrict__ part, int nsplit,
                                                            int64_t n4, int64_t stride4,
                                                            void* __restrict__ out, int bf16) {
+  pdl_enter();  // wait for the previous kernel before any global access
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (int64_t)gridDim.x * blockDim.x) {
     float4 acc = part[i];
@@ -1077,8 +1086,8 @@ int launch_split_reduce(const float* part, int nsplit, int64_t n, int64_t stride
   const int64_t n4 = n / 4;
   int64_t blocks = (n4 + 255) / 256;
   if (blocks > 4 * (int64_t)sm_count()) blocks = 4 * (int64_t)sm_count();
-  split_reduce_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(part), nsplit, n4,
-                                                        stride / 4, out, bf16 ? 1 : 0);
+  MOE_LAUNCH(launch_pdl(split_reduce_kernel, (unsigned)blocks, 256, 0, s, reinterpret_cast<const float4*>(part), nsplit, n4,
+                                                        stride / 4, out, bf16 ? 1 : 0));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -55,6 +55,29 @@ struct GemmParams {
 // Host-side count of kernels enqueued (every launcher adds the kernels it launched).
 void count_launches(int n);
 
+#define MOE_LAUNCH(call)                              \
+  do {                                                \
+    if ((call) != cudaSuccess) return MOE_ERR_CUDA;   \
+  } while (0)
+
+// Launch with programmatic dependent launch allowed (see pdl_enter): the kernel may be scheduled
+// while the previous kernel in the stream finishes; it waits for that kernel before touching memory.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Host helpers for TMA descriptors (swizzle: 2 = 128B, 1 = 128B with 32-byte atoms, 0 = none).
 bool make_tmap_nd(CUtensorMap* m, const void* ptr, int es, int rank, const uint64_t* dims,
                   const uint64_t* strides_bytes, const uint32_t* box, int swizzle);

@@ -70,6 +70,7 @@ __device__ __forceinline__ void zero_pad_rows(uint4* buf, int e, const int32_t* 
 __global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ prow, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ poff, uint4* __restrict__ xp, int T, int k, int vpr, int tok_blocks) {
+  pdl_enter();  // wait for the previous kernel before any global access
   if ((int)blockIdx.x >= tok_blocks) {
     zero_pad_rows(xp, blockIdx.x - tok_blocks, counts, poff, vpr);
     return;
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const uint4* __res
                                                               const int32_t* __restrict__ prow,
                                                               uint4* __restrict__ out, int T, int k,
                                                               int vpr) {
+  pdl_enter();  // wait for the previous kernel before any global access
   using V = Vec<BF16>;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -136,6 +138,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) combine_bwd_kernel(
     const int32_t* __restrict__ counts, const int32_t* __restrict__ poff, uint4* __restrict__ dy,
     float* __restrict__ dgates, float* __restrict__ dlsel, void* __restrict__ dlogits, int T, int k,
     int E, int vpr, int tok_blocks) {
+  pdl_enter();  // wait for the previous kernel before any global access
   using V = Vec<BF16>;
   if ((int)blockIdx.x >= tok_blocks) {
     zero_pad_rows(dy, blockIdx.x - tok_blocks, counts, poff, vpr);
@@ -219,6 +222,7 @@ __global__ void __launch_bounds__(kWarps * 32) token_reduce_kernel(
     const uint4* __restrict__ dxp, const int32_t* __restrict__ prow, const float* __restrict__ dlsel,
     const int32_t* __restrict__ idx, const uint4* __restrict__ Wr, uint4* __restrict__ dx, int T,
     int k, int E, int vpr) {
+  pdl_enter();  // wait for the previous kernel before any global access
   using V = Vec<BF16>;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
@@ -265,9 +269,9 @@ int launch_dispatch(const void* x, const int32_t* prow, const int32_t* counts, c
                     void* xp, int T, int k, int E, int row_bytes, cudaStream_t s) {
   const int vpr = row_bytes / 16;
   const int tok_blocks = (T + kWarps - 1) / kWarps;
-  dispatch_kernel<<<tok_blocks + E, kWarps * 32, 0, s>>>(
+  MOE_LAUNCH(launch_pdl(dispatch_kernel, tok_blocks + E, kWarps * 32, 0, s, 
       static_cast<const uint4*>(x), prow, counts, poff, static_cast<uint4*>(xp), T, k, vpr,
-      tok_blocks);
+      tok_blocks));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -277,11 +281,11 @@ int launch_combine(const void* y, const float* gates, const int32_t* prow, void*
   const int vpr = row_bytes / 16;
   const int blocks = (T + kWarps - 1) / kWarps;
   if (bf16)
-    combine_kernel<true><<<blocks, kWarps * 32, 0, s>>>(static_cast<const uint4*>(y), gates, prow,
-                                                        static_cast<uint4*>(out), T, k, vpr);
+    MOE_LAUNCH(launch_pdl(combine_kernel<true>, blocks, kWarps * 32, 0, s, static_cast<const uint4*>(y), gates, prow,
+                                                        static_cast<uint4*>(out), T, k, vpr));
   else
-    combine_kernel<false><<<blocks, kWarps * 32, 0, s>>>(static_cast<const uint4*>(y), gates, prow,
-                                                         static_cast<uint4*>(out), T, k, vpr);
+    MOE_LAUNCH(launch_pdl(combine_kernel<false>, blocks, kWarps * 32, 0, s, static_cast<const uint4*>(y), gates, prow,
+                                                         static_cast<uint4*>(out), T, k, vpr));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -293,13 +297,13 @@ int launch_combine_bwd(const void* dout, const void* y, const float* gates, cons
   const int vpr = row_bytes / 16;
   const int tok_blocks = (T + kWarps - 1) / kWarps;
   if (bf16)
-    combine_bwd_kernel<true><<<tok_blocks + E, kWarps * 32, 0, s>>>(
+    MOE_LAUNCH(launch_pdl(combine_bwd_kernel<true>, tok_blocks + E, kWarps * 32, 0, s, 
         static_cast<const uint4*>(dout), static_cast<const uint4*>(y), gates, prow, idx, counts,
-        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks);
+        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks));
   else
-    combine_bwd_kernel<false><<<tok_blocks + E, kWarps * 32, 0, s>>>(
+    MOE_LAUNCH(launch_pdl(combine_bwd_kernel<false>, tok_blocks + E, kWarps * 32, 0, s, 
         static_cast<const uint4*>(dout), static_cast<const uint4*>(y), gates, prow, idx, counts,
-        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks);
+        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -310,13 +314,13 @@ int launch_token_reduce(const void* dxp, const int32_t* prow, const float* dlsel
   const int vpr = row_bytes / 16;
   const int blocks = (T + kWarps - 1) / kWarps;
   if (bf16)
-    token_reduce_kernel<true><<<blocks, kWarps * 32, 0, s>>>(
+    MOE_LAUNCH(launch_pdl(token_reduce_kernel<true>, blocks, kWarps * 32, 0, s, 
         static_cast<const uint4*>(dxp), prow, dlsel, idx, static_cast<const uint4*>(Wr),
-        static_cast<uint4*>(dx), T, k, E, vpr);
+        static_cast<uint4*>(dx), T, k, E, vpr));
   else
-    token_reduce_kernel<false><<<blocks, kWarps * 32, 0, s>>>(
+    MOE_LAUNCH(launch_pdl(token_reduce_kernel<false>, blocks, kWarps * 32, 0, s, 
         static_cast<const uint4*>(dxp), prow, dlsel, idx, static_cast<const uint4*>(Wr),
-        static_cast<uint4*>(dx), T, k, E, vpr);
+        static_cast<uint4*>(dx), T, k, E, vpr));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

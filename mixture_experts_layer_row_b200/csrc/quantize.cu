@@ -74,6 +74,7 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const uint4* __restrict_
                                                         int blocks_per_row, int layout, int64_t G,
                                                         uint4* __restrict__ q,
                                                         uint8_t* __restrict__ s) {
+  pdl_enter();  // wait for the previous kernel before any global access
   const int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= nblocks) return;
   uint4 w[4];
@@ -113,6 +114,7 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const uint4* __restrict_
 __global__ void __launch_bounds__(128) quant_col_kernel(const uint2* __restrict__ src, int64_t rows,
                                                         int cols, int layout, uint32_t* __restrict__ q,
                                                         uint8_t* __restrict__ s) {
+  pdl_enter();  // wait for the previous kernel before any global access
   const int groups = cols / 4;
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t rblocks = rows / 32;
@@ -161,13 +163,13 @@ int launch_quantize(const void* src, int64_t rows, int cols, int mode, int64_t G
   if (row) {
     const int64_t nb = rows * (cols / 32);
     const int64_t grid = (nb + 255) / 256;
-    quant_row_kernel<<<(unsigned)grid, 256, 0, st>>>(static_cast<const uint4*>(src), nb, cols / 32,
-                                                      layout, G, reinterpret_cast<uint4*>(q), s);
+    MOE_LAUNCH(launch_pdl(quant_row_kernel, (unsigned)grid, 256, 0, st, static_cast<const uint4*>(src), nb, cols / 32,
+                                                      layout, G, reinterpret_cast<uint4*>(q), s));
   } else {
     const int64_t nt = (rows / 32) * (cols / 4);
     const int64_t grid = (nt + 127) / 128;
-    quant_col_kernel<<<(unsigned)grid, 128, 0, st>>>(static_cast<const uint2*>(src), rows, cols,
-                                                      layout, reinterpret_cast<uint32_t*>(q), s);
+    MOE_LAUNCH(launch_pdl(quant_col_kernel, (unsigned)grid, 128, 0, st, static_cast<const uint2*>(src), rows, cols,
+                                                      layout, reinterpret_cast<uint32_t*>(q), s));
   }
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

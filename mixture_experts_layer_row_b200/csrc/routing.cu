@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
                                                    const float* __restrict__ bias, int T, int E, int k,
                                                    int renorm, int32_t* __restrict__ idx,
                                                    float* __restrict__ gates, uint32_t* err) {
+  pdl_enter();  // wait for the previous kernel before any global access
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
@@ -102,6 +103,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 __global__ void __launch_bounds__(kChunk) hist_kernel(const int32_t* __restrict__ idx, int T, int E,
                                                       int k, int32_t* __restrict__ hist,
                                                       uint32_t* err) {
+  pdl_enter();  // wait for the previous kernel before any global access
   __shared__ int h[256];
   for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
   __syncthreads();
@@ -157,6 +159,7 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ hist, i
                                                    int32_t* __restrict__ offsets,
                                                    int32_t* __restrict__ poff,
                                                    int32_t* __restrict__ row_token, uint32_t* err) {
+  pdl_enter();  // wait for the previous kernel before any global access
   __shared__ int sw[32];
   const int e = threadIdx.x;
   int run = 0;
@@ -193,6 +196,7 @@ __global__ void __launch_bounds__(kChunk) rank_kernel(const int32_t* __restrict_
                                                       int32_t* __restrict__ perm,
                                                       int32_t* __restrict__ prow,
                                                       int32_t* __restrict__ row_token) {
+  pdl_enter();  // wait for the previous kernel before any global access
   __shared__ int wcnt[kChunk / 32][256];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < (kChunk / 32) * 256; i += blockDim.x) (&wcnt[0][0])[i] = 0;
@@ -253,7 +257,7 @@ int launch_topk(const float* logits, const float* bias, int T, int E, int k, int
   switch (vpl) {
 #define MOE_TOPK_CASE(V) \
   case V:                \
-    topk_kernel<V><<<blocks, threads, 0, s>>>(logits, bias, T, E, k, renorm, idx, gates, err); break;
+    MOE_LAUNCH(launch_pdl(topk_kernel<V>, blocks, threads, 0, s, logits, bias, T, E, k, renorm, idx, gates, err)); break;
     MOE_TOPK_CASE(1)
     MOE_TOPK_CASE(2)
     MOE_TOPK_CASE(3)
@@ -279,10 +283,10 @@ int launch_metadata(const int32_t* idx, int T, int E, int k, int align, int64_t 
                     int32_t* counts, int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
                     int32_t* row_token, int32_t* hist_ws, uint32_t* err, cudaStream_t s) {
   const int nchunks = (T + kChunk - 1) / kChunk;
-  hist_kernel<<<nchunks, kChunk, 0, s>>>(idx, T, E, k, hist_ws, err);
-  scan_kernel<<<1, 256, 0, s>>>(hist_ws, nchunks, T, E, k, align, max_rows, counts, offsets, poff,
-                                row_token, err);
-  rank_kernel<<<nchunks, kChunk, 0, s>>>(idx, T, E, k, hist_ws, offsets, poff, perm, prow, row_token);
+  MOE_LAUNCH(launch_pdl(hist_kernel, nchunks, kChunk, 0, s, idx, T, E, k, hist_ws, err));
+  MOE_LAUNCH(launch_pdl(scan_kernel, 1, 256, 0, s, hist_ws, nchunks, T, E, k, align, max_rows, counts, offsets, poff,
+                                row_token, err));
+  MOE_LAUNCH(launch_pdl(rank_kernel, nchunks, kChunk, 0, s, idx, T, E, k, hist_ws, offsets, poff, perm, prow, row_token));
   count_launches(3);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
