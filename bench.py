@@ -61,8 +61,8 @@ def load_peaks():
 # current kernels on the full-size workload (profiles/grouped_gemm_fwd1_e128_bf16.md,
 # profiles/grouped_gemm_wgrad1_e128_bf16.md). A kernel or workload not listed reports null.
 MEASURED_TRAFFIC = {
-    ("e128_bf16", "gemm_fwd1_swiglu"): 1.235260e9 + 0.198228e9,
-    ("e128_bf16", "gemm_wgrad1"): 0.286070e9 + 1.015937e9,
+    ("e128_bf16", "gemm_fwd1_swiglu"): 1.224964e9 + 0.199070e9,
+    ("e128_bf16", "gemm_wgrad1"): 0.286039e9 + 1.014497e9,
 }
 
 
