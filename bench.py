@@ -439,10 +439,14 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=256, help="oracle sample per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="expert-count sweep: the workload's shapes with E experts, uniform routing")
     args = ap.parse_args()
 
     from moe_workloads import WORKLOADS
     w = WORKLOADS[args.workload]
+    if args.experts:
+        w = w.scaled(E=args.experts, routing="uniform", skew=0.0, name=f"{w.name}_E{args.experts}")
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -504,6 +508,10 @@ def main():
     ms = max_over_ranks(t_start.elapsed_time(t_end), "cuda")
     ms_per_step = ms / args.steps
     value = world * w.T / (ms_per_step / 1e3)
+
+    # device memory high-water mark of the run so far: inputs, weights, gradients, the layer's saved
+    # activations and scratch (the MXFP8 path adds the quantised copies)
+    peak_mem_gb = torch.cuda.max_memory_allocated() / 1e9
 
     # per-op durations over the timed region
     per_op = {n: 0.0 for n in step.names}
@@ -654,6 +662,7 @@ def main():
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk,
+            "peak_mem_gb": round(peak_mem_gb, 2),
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -57,6 +57,8 @@ WORKLOADS = {
     "e128_bf16": Workload("e128_bf16", 8192, 2048, 1024, 128, 4, "bf16", "uniform"),
     "e128_skew": Workload("e128_skew", 16384, 2048, 1024, 128, 4, "bf16", "learned", skew=1.2),
     "e128_mxfp8": Workload("e128_mxfp8", 16384, 4096, 1536, 128, 4, "mxfp8", "uniform"),
+    # the MXFP8 workload's shapes in bf16, for the bf16 vs MXFP8 comparison
+    "e128_bf16_wide": Workload("e128_bf16_wide", 16384, 4096, 1536, 128, 4, "bf16", "uniform"),
 }
 
 
