@@ -101,7 +101,7 @@ def weight_quant_work(w):
     return 2 * (n * 2 + n + n // 32)            # two orientations: read bf16, write codes + scales
 
 
-def op_work(w, es=2):
+def op_work(w, es=2, recompute=False):
     if w.dtype == "mxfp8":
         return op_work_mx(w)
     T, d, F, E, k = w.T, w.d, w.F, w.E, w.k
@@ -113,10 +113,14 @@ def op_work(w, es=2):
         ops["route_topk"] = (T * E * 4 + T * k * 8, 0)
     ops["route_metadata"] = (T * k * 4 * 3 + Rp * 4, 0)
     ops["dispatch"] = ((T + R) * d * es, 0)
-    ops["gemm_fwd1_swiglu"] = ((R * d + E * 2 * F * d + R * 2 * F + R * F) * es, 2 * R * d * 2 * F)
+    fwd1 = ((R * d + E * 2 * F * d + R * 2 * F + R * F) * es, 2 * R * d * 2 * F)
+    # with activation recompute the forward's GEMM1 writes only a; the backward runs it again in full
+    ops["gemm_fwd1_swiglu"] = (fwd1[0] - R * 2 * F * es, fwd1[1]) if recompute else fwd1
     ops["gemm_fwd2"] = ((R * F + E * d * F + R * d) * es, 2 * R * F * d)
     ops["combine"] = ((R * d + T * d) * es + T * k * 8, 0)
     ops["combine_bwd"] = ((T * d + 2 * R * d) * es + T * k * 12, 0)
+    if recompute:
+        ops["gemm_fwd1_recompute"] = fwd1
     ops["gemm_dgrad2_swiglu"] = ((R * d + E * d * F + 2 * R * 2 * F) * es, 2 * R * d * F)
     ops["gemm_wgrad2"] = ((R * d + R * F + E * d * F) * es, 2 * R * d * F)
     ops["gemm_dgrad1"] = ((R * 2 * F + E * 2 * F * d + R * d) * es, 2 * R * 2 * F * d)
@@ -143,7 +147,7 @@ class Step:
         else:
             lay.idx.copy_(inp["idx"])
             lay.gates.copy_(inp["gates"])
-        self.names = list(op_work(w).keys())
+        self.names = list(op_work(w, recompute=layer.recompute).keys())
         self.ev = None
 
     def events(self, n_steps):
@@ -180,7 +184,12 @@ class Step:
         dlg = self.dlogits if self.learned else None
         mark(); L.combine_bwd(c, inp["dout"], lay.y, lay.gates, lay.prow, lay.idx, lay.counts, lay.poff,
                               lay.dy, lay.dgates, dls, dlg)
-        mark(); L.grouped_gemm(c, L.GEMM_DGRAD2_SWIGLU, lay.dy, inp["W2"], lay.dh13, None, lay.h13,
+        h13 = lay.h13
+        if lay.recompute:
+            mark(); L.grouped_gemm(c, L.GEMM_FWD1_SWIGLU, lay.x_perm, inp["W13"], lay.dh13, lay.a, None,
+                                   lay.counts, lay.poff, lay.ws)
+            h13 = lay.dh13
+        mark(); L.grouped_gemm(c, L.GEMM_DGRAD2_SWIGLU, lay.dy, inp["W2"], lay.dh13, None, h13,
                                lay.counts, lay.poff, lay.ws)
         mark(); L.grouped_gemm(c, L.GEMM_WGRAD2, lay.dy, lay.a, lay.dW2, None, None, lay.counts,
                                lay.poff, lay.ws)
@@ -441,6 +450,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
                     help="expert-count sweep: the workload's shapes with E experts, uniform routing")
+    ap.add_argument("--recompute", action="store_true",
+                    help="activation recompute: the layer keeps no h13 and the backward regenerates it; "
+                         "also times it against stored activations through the layer API")
     args = ap.parse_args()
 
     from moe_workloads import WORKLOADS
@@ -467,7 +479,10 @@ def main():
 
     inp = make_inputs(w, seed=0, device="cuda")
     learned = w.routing == "learned"
-    layer = MoELayer(w.T, w.d, w.F, w.E, w.k, dtype=w.dtype, learned_router=learned)
+    if args.recompute and w.dtype == "mxfp8":
+        raise SystemExit("--recompute: activation recompute is implemented for the bf16 / fp32 layer")
+    layer = MoELayer(w.T, w.d, w.F, w.E, w.k, dtype=w.dtype, learned_router=learned,
+                     recompute=args.recompute)
     layer.set_weights(inp["W13"], inp["W2"], inp["W_r"] if learned else None)
     step = Step(layer, w, inp)
 
@@ -522,7 +537,7 @@ def main():
     per_op = {n: v / args.steps for n, v in per_op.items()}
 
     peaks = load_peaks()
-    work = op_work(w, 4 if w.dtype == "fp32" else 2)
+    work = op_work(w, 4 if w.dtype == "fp32" else 2, recompute=layer.recompute)
     bw = peaks["hbm_gbs"]
     # tensor peak of the GEMMs' own dtype: the measured bf16 figure times the nominal dense ratio
     # (tf32 1.1 / bf16 2.25 PFLOP/s; fp8 4.5 / 2.25)
@@ -640,6 +655,51 @@ def main():
                       "the neighbouring steps' compute"}
         assert torch.equal(ho.cuda(), ref[0]) and torch.equal(hdx.cuda(), ref[1])
 
+    # activation recompute against stored activations, both through the public layer API on the
+    # same device-resident inputs, timed in alternation (so clock and power drift hit both alike),
+    # with the activation memory each keeps between the two passes
+    rc = None
+    if layer.recompute:
+        lay_st = MoELayer(w.T, w.d, w.F, w.E, w.k, dtype=w.dtype, learned_router=learned)
+        lay_st.set_weights(inp["W13"], inp["W2"], inp["W_r"] if learned else None)
+
+        def api_ms(lay):
+            def one():
+                lay.forward(inp["x"], bias=inp["bias"], idx=inp["idx"], gates=inp["gates"])
+                lay.backward(inp["dout"])
+            for _ in range(args.warmup):
+                one()
+            torch.cuda.synchronize()
+            barrier()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
+            for _ in range(args.steps):
+                one()
+            a1.record()
+            torch.cuda.synchronize()
+            return max_over_ranks(a0.elapsed_time(a1), "cuda") / args.steps
+
+        t_st, t_rc = [], []
+        for _ in range(3):
+            t_st.append(api_ms(lay_st))
+            t_rc.append(api_ms(layer))
+        ms_st, ms_rc = sorted(t_st)[1], sorted(t_rc)[1]
+        same = all(torch.equal(a, b) for a, b in zip(
+            (lay_st.out, lay_st.dx, lay_st.dW13, lay_st.dW2), (layer.out, layer.dx, layer.dW13, layer.dW2)))
+        assert same and layer.error_flags() == 0, "recompute differs from stored activations"
+        es, R = layer.act.itemsize, layer.R
+        # kept from forward to backward: x_perm and y, plus h13 and a when stored (with recompute a
+        # is scratch that the backward rewrites)
+        kept_st = R * (2 * w.d + 2 * w.F + w.F) * es
+        kept_rc = R * 2 * w.d * es
+        rc = {"ms_per_step_stored": ms_st, "ms_per_step_recompute": ms_rc,
+              "value_stored": world * w.T / (ms_st / 1e3), "value_recompute": world * w.T / (ms_rc / 1e3),
+              "throughput_ratio": ms_st / ms_rc,
+              "kept_activation_bytes": {"stored": kept_st, "recompute": kept_rc},
+              "kept_activation_ratio": kept_rc / kept_st, "bit_identical": same,
+              "timing": "layer API, device-resident inputs, median of 3 alternating runs of K steps"}
+        del lay_st
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, inp, min(args.cpu_tokens, w.T), w.name)
@@ -650,7 +710,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic (seeded; shapes and distributions of the workload)",
-            "config": dict(workload_config(w), parallelism=f"replicas x{world}"),
+            "config": dict(workload_config(w), parallelism=f"replicas x{world}",
+                           **({"activation_recompute": True} if layer.recompute else {})),
             "tflops": 18 * w.d * w.F * w.T * w.k * world / (ms_per_step / 1e3) / 1e12,
             "grouped_gemm_tensor_frac": (gemm_flops / (gemm_ms / 1e3) / 1e12) / tc,
             "layer_roofline": {"roofline_ms": roof_time * 1e3, "frac": roof_time * 1e3 / ms_per_step,
@@ -664,6 +725,8 @@ def main():
             "clocks": clk,
             "peak_mem_gb": round(peak_mem_gb, 2),
         }
+        if rc is not None:
+            line["recompute"] = rc
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

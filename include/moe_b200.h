@@ -183,13 +183,15 @@ MOE_API int moe_token_reduce(const moe_config_t* cfg, const void* dx_perm, const
 
 enum moe_gemm_op {
   /* h13 = X_e W13_e^T and a = silu(h13[:, :F]) * h13[:, F:] for every expert's rows.
-   * A = x_perm act [max_rows,d]; B = W13 [E,2F,d]; C = h13 act [max_rows,2F]; C2 = a act [max_rows,F]. */
+   * A = x_perm act [max_rows,d]; B = W13 [E,2F,d]; C = h13 act [max_rows,2F]; C2 = a act [max_rows,F].
+   * C may be NULL: only a is stored (the forward of a layer that recomputes h13 in its backward). */
   MOE_GEMM_FWD1_SWIGLU = 0,
   /* y = a_e W2_e^T.  A = a [max_rows,F]; B = W2 [E,d,F]; C = y [max_rows,d]. */
   MOE_GEMM_FWD2 = 1,
   /* da = dy_e W2_e, then the SwiGLU backward with the saved h13 (aux):
    * dh13[:, :F] = da * up * silu'(gate), dh13[:, F:] = da * silu(gate).
-   * A = dy [max_rows,d]; B = W2 [E,d,F]; aux = h13 [max_rows,2F]; C = dh13 [max_rows,2F]. */
+   * A = dy [max_rows,d]; B = W2 [E,d,F]; aux = h13 [max_rows,2F]; C = dh13 [max_rows,2F].
+   * aux may be C itself (dh13 overwrites h13 in place: each element is read before it is written). */
   MOE_GEMM_DGRAD2_SWIGLU = 2,
   /* dx_perm = dh13_e W13_e.  A = dh13 [max_rows,2F]; B = W13 [E,2F,d]; C = dx_perm [max_rows,d]. */
   MOE_GEMM_DGRAD1 = 3,
@@ -279,8 +281,8 @@ typedef struct {
   int32_t* prow;      /* [T*k] */
   int32_t* row_token; /* [max_rows] */
   void* x_perm;       /* act [max_rows,d] */
-  void* h13;          /* act [max_rows,2F] */
-  void* a;            /* act [max_rows,F] */
+  void* h13;          /* act [max_rows,2F]; NULL selects activation recompute (bf16 / fp32 layer) */
+  void* a;            /* act [max_rows,F]; with recompute, scratch between the two passes */
   void* y;            /* act [max_rows,d] */
 } moe_saved_t;
 
@@ -296,7 +298,12 @@ typedef struct {
 } moe_grads_t;
 
 /* Whole forward: [router scores -> top-k] -> metadata -> dispatch -> grouped GEMM1 + SwiGLU ->
- * grouped GEMM2 -> combine. x: act [T,d]; bias: fp32 [E] or NULL; out: act [T,d]. */
+ * grouped GEMM2 -> combine. x: act [T,d]; bias: fp32 [E] or NULL; out: act [T,d].
+ * Activation recompute (the memory-for-throughput trade of unite.ai "Parallelismo, precisione e
+ * tecniche di memoria"): with saved->h13 == NULL the forward stores no h13 and moe_layer_bwd recomputes h13 and
+ * a with one more GEMM1, writing h13 into grads->dh13 (which the SwiGLU backward then overwrites)
+ * and a into saved->a. The caller may reuse saved->a's memory between the two passes. Results are
+ * bit-identical to the stored-activation path. */
 MOE_API int moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* w, const void* x, const float* bias,
                   void* out, moe_saved_t* saved, void* ws, size_t ws_bytes, void* stream);
 

@@ -362,8 +362,8 @@ int moe_grouped_gemm(const moe_config_t* cfg, int op, const void* A, const void*
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws, ws_bytes));
   MOE_REQUIRE(cfg->dtype != MOE_DTYPE_MXFP8, MOE_ERR_UNSUPPORTED);
-  MOE_REQUIRE(A && B && C && counts && poff, MOE_ERR_INVALID_ARG);
-  MOE_REQUIRE(aligned16(A) && aligned16(B) && aligned16(C) && (!C2 || aligned16(C2)),
+  MOE_REQUIRE(A && B && (C || op == MOE_GEMM_FWD1_SWIGLU) && counts && poff, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(A) && aligned16(B) && (!C || aligned16(C)) && (!C2 || aligned16(C2)),
               MOE_ERR_INVALID_ARG);
   return gemm_op(cfg, op, A, B, C, C2, aux, counts, poff, ws, S(stream));
 }
@@ -418,11 +418,12 @@ int moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* w, const void* x
   MOE_TRY(check_ws(cfg, ws, ws_bytes));
   MOE_REQUIRE(cfg->dtype != MOE_DTYPE_MXFP8, MOE_ERR_UNSUPPORTED);
   MOE_REQUIRE(w && sv && x && out && w->W13 && w->W2, MOE_ERR_INVALID_ARG);
+  // sv->h13 == NULL selects activation recompute: h13 is not kept, the backward regenerates it
   MOE_REQUIRE(sv->idx && sv->gates && sv->counts && sv->offsets && sv->poff && sv->perm && sv->prow &&
-                  sv->row_token && sv->x_perm && sv->h13 && sv->a && sv->y,
+                  sv->row_token && sv->x_perm && sv->a && sv->y,
               MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(aligned16(x) && aligned16(out) && aligned16(w->W13) && aligned16(w->W2) &&
-                  aligned16(sv->x_perm) && aligned16(sv->h13) && aligned16(sv->a) &&
+                  aligned16(sv->x_perm) && (!sv->h13 || aligned16(sv->h13)) && aligned16(sv->a) &&
                   aligned16(sv->y),
               MOE_ERR_INVALID_ARG);
   cudaStream_t s = S(stream);
@@ -472,7 +473,16 @@ int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_sav
   const bool bf = es_of(cfg) == 2;
   MOE_TRY(launch_combine_bwd(dout, sv->y, sv->gates, sv->prow, sv->idx, sv->counts, sv->poff, g->dy,
                              g->dgates, dlsel, dlog, cfg->T, cfg->k, cfg->E, rb, bf, s));
-  MOE_TRY(gemm_op(cfg, MOE_GEMM_DGRAD2_SWIGLU, g->dy, w->W2, g->dh13, nullptr, sv->h13, sv->counts,
+  // Activation recompute (the forward kept no h13): GEMM1 regenerates h13 into the dh13 buffer and a
+  // into saved->a; the SwiGLU-backward GEMM then overwrites h13 with dh13 in place (each element is
+  // read and written by the same tile, the read first).
+  const void* h13 = sv->h13;
+  if (!h13) {
+    MOE_TRY(gemm_op(cfg, MOE_GEMM_FWD1_SWIGLU, sv->x_perm, w->W13, g->dh13, sv->a, nullptr, sv->counts,
+                    sv->poff, ws, s));
+    h13 = g->dh13;
+  }
+  MOE_TRY(gemm_op(cfg, MOE_GEMM_DGRAD2_SWIGLU, g->dy, w->W2, g->dh13, nullptr, h13, sv->counts,
                   sv->poff, ws, s));
   MOE_TRY(gemm_op(cfg, MOE_GEMM_WGRAD2, g->dy, sv->a, g->dW2, nullptr, nullptr, sv->counts, sv->poff,
                   ws, s));

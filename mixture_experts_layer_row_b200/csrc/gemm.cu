@@ -690,13 +690,17 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               a[i] = silu_f(g[i]) * u[i];
             }
             const int ch0 = ((j % CPB) * 32 * C::OES) >> 4;
-            stage_row32<C::OES>(bg, lane, ch0, g);
-            stage_row32<C::OES>(bu, lane, ch0, u);
+            if (p.C) {  // h13 kept for the backward (absent: the backward recomputes it)
+              stage_row32<C::OES>(bg, lane, ch0, g);
+              stage_row32<C::OES>(bu, lane, ch0, u);
+            }
             stage_row32<C::OES>(ba, lane, ch0, a);
             if (j % CPB == CPB - 1) {
               const int c = (j / CPB) * C::OEPR;
-              box_store(&tmC, bg, lane, ti.n0 + c, c1);
-              box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
+              if (p.C) {
+                box_store(&tmC, bg, lane, ti.n0 + c, c1);
+                box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
+              }
               box_store(&tmC2, ba, lane, ti.n0 + c, c1);
             }
           }
@@ -951,10 +955,16 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   const int64_t out_rows =
       (MODE == GROUP_K) ? (int64_t)k_groups(p) * (p.c_group_rows ? p.c_group_rows : p.M) : A.rows;
   const int64_t out_cols = (EPI == EPI_SWIGLU_FWD || EPI == EPI_SWIGLU_BWD) ? 2 * (int64_t)p.F : p.N;
-  if (!make_tmap(&tc, p.C, C::OES, out_rows, out_cols, p.ldc, C::OEPR, 32, 2)) return MOE_ERR_CUDA;
-  tc2 = tc;
   if (EPI == EPI_SWIGLU_FWD && !make_tmap(&tc2, p.C2, C::OES, out_rows, p.F, p.ldc2, C::OEPR, 32, 2))
     return MOE_ERR_CUDA;
+  if (p.C) {
+    if (!make_tmap(&tc, p.C, C::OES, out_rows, out_cols, p.ldc, C::OEPR, 32, 2)) return MOE_ERR_CUDA;
+  } else if (EPI == EPI_SWIGLU_FWD) {
+    tc = tc2;  // SwiGLU forward without h13: only a is stored, tc is never used
+  } else {
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (EPI != EPI_SWIGLU_FWD) tc2 = tc;
   // persistent grid: one CTA (pair) per SM (pair of SMs), capped by the tile count where the host
   // knows it (GROUP_K: fixed tiles per group)
   int64_t cap = 0;

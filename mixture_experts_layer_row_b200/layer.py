@@ -23,9 +23,14 @@ class MoELayer:
         learned_router: allocate router buffers (scores, score gradients, dW_r).
     """
 
-    def __init__(self, T, d, F, E, k, dtype="bf16", device="cuda", learned_router=True, renorm=True):
+    def __init__(self, T, d, F, E, k, dtype="bf16", device="cuda", learned_router=True, renorm=True,
+                 recompute=False):
+        """recompute: keep no h13 between the passes; the backward regenerates it with one more GEMM1
+        (bf16 / fp32 layers)."""
         if dtype not in _DT:
             raise ValueError(f"unsupported dtype {dtype}")
+        if recompute and dtype == "mxfp8":
+            raise ValueError("activation recompute is implemented for the bf16 / fp32 layer")
         code, self.act = _DT[dtype]
         self.cfg = L.make_config(T, d, F, E, k, code, 1 if renorm else 0)
         self.T, self.d, self.F, self.E, self.k = T, d, F, E, k
@@ -45,7 +50,9 @@ class MoELayer:
         self.idx, self.gates = z((T, k), i32), z((T, k), f32)
         self.counts, self.offsets, self.poff = z(E, i32), z(E + 1, i32), z(E + 1, i32)
         self.perm, self.prow, self.row_token = z(T * k, i32), z(T * k, i32), z(R, i32)
-        self.x_perm, self.h13, self.a, self.y = z((R, d), act), z((R, 2 * F), act), z((R, F), act), z((R, d), act)
+        self.recompute = recompute
+        self.x_perm, self.a, self.y = z((R, d), act), z((R, F), act), z((R, d), act)
+        self.h13 = None if recompute else z((R, 2 * F), act)
         self.out = z((T, d), act)
         self.dx = z((T, d), act)
         self.dW13, self.dW2 = z((E, 2 * F, d), act), z((E, d, F), act)

@@ -163,6 +163,27 @@ def test_wgrad(shape, dtype, which):
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("shape", ["ragged", "ragged_pairs", "wide"])
+def test_fwd1_without_h13_and_dgrad2_in_place(shape, dtype):
+    """The two GEMMs activation recompute relies on: GEMM1 with no h13 output stores the same a as
+    with it, and the SwiGLU-backward GEMM overwriting its h13 input in place gives the same dh13 as
+    with separate buffers."""
+    P = Problem(shape, dtype)
+    X, W13 = P.rows(P.d), P.weights(P.E, 2 * P.F, P.d)
+    h13, a = P.run(P.L.GEMM_FWD1_SWIGLU, X, W13, _sentinel(P.R, 2 * P.F, dtype), _sentinel(P.R, P.F, dtype))
+    _, a_only = P.run(P.L.GEMM_FWD1_SWIGLU, X, W13, None, _sentinel(P.R, P.F, dtype))
+    assert torch.equal(a_only, a)
+    dY, W2 = P.rows(P.d), P.weights(P.E, P.d, P.F)
+    dh, _ = P.run(P.L.GEMM_DGRAD2_SWIGLU, dY, W2, _sentinel(P.R, 2 * P.F, dtype), aux=h13)
+    buf = h13.clone()
+    P.L.grouped_gemm(P.cfg, P.L.GEMM_DGRAD2_SWIGLU, dY.to(dev()), W2.to(dev()), buf, None, buf,
+                     P.counts, P.poff, P.ws)
+    torch.cuda.synchronize()
+    assert P.L.get_error(P.ws) == 0
+    assert torch.equal(buf, dh)
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
 def test_gemm_is_deterministic(dtype):
     P = Problem("wide", dtype)
     G, X = P.rows(P.d), P.rows(P.F)

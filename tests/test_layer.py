@@ -176,6 +176,36 @@ def test_layer_back_to_back_matches_isolated_runs():
     assert layer.error_flags() == 0
 
 
+@pytest.mark.parametrize("name", ["e8_learned_small", "e128_uniform_ragged", "e32_skew_small"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_layer_recompute_matches_stored_activations(name, dtype):
+    """With activation recompute the forward keeps no h13 and the backward regenerates it with the
+    same GEMM1 kernel; every output and gradient must equal the stored-activation layer's bit for
+    bit."""
+    from mixture_experts_layer_row_b200 import MoELayer
+    w = SMALL[name]
+    w = Workload(w.name, w.T, w.d, w.F, w.E, w.k, dtype, w.routing, skew=w.skew)
+    inp = make_inputs(w, seed=11, device="cuda")
+    learned = w.routing == "learned"
+    res = []
+    for rc in (False, True):
+        layer = MoELayer(w.T, w.d, w.F, w.E, w.k, dtype=dtype, learned_router=learned, recompute=rc)
+        assert (layer.h13 is None) == rc
+        layer.set_weights(inp["W13"], inp["W2"], inp["W_r"] if learned else None)
+        layer.forward(inp["x"], bias=inp["bias"], idx=inp["idx"], gates=inp["gates"])
+        if rc:
+            layer.a.fill_(7.0)  # the forward's a is not needed by the backward's recompute path
+        layer.backward(inp["dout"])
+        torch.cuda.synchronize()
+        assert layer.error_flags() == 0
+        ts = [layer.out, layer.dx, layer.dW13, layer.dW2, layer.dgates]
+        if learned:
+            ts.append(layer.dW_r)
+        res.append([t.clone() for t in ts])
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
+
+
 def test_layer_twice_is_deterministic():
     w = SMALL["e32_uniform_small"]
     inp = make_inputs(w, seed=3, device="cuda")
