@@ -76,21 +76,18 @@ def op_work_mx(w):
     ops = {}
     ops["route_metadata"] = (T * k * 4 * 3 + Rp * 4, 0)
     ops["dispatch"] = ((T + R) * d * 2, 0)
-    ops["quant_x_row"] = (R * d * 2 + q(R * d), 0)
+    # each activation is quantised along rows and columns in one pass: one bf16 read, two fp8 writes
+    ops["quant_x"] = (R * d * 2 + 2 * q(R * d), 0)
     ops["gemm_fwd1_swiglu"] = (q(R * d) + q(E * 2 * F * d) + (R * 2 * F + R * F) * 2, 4 * R * d * F)
-    ops["quant_a_row"] = (R * F * 2 + q(R * F), 0)
+    ops["quant_a"] = (R * F * 2 + 2 * q(R * F), 0)
     ops["gemm_fwd2"] = (q(R * F) + q(E * d * F) + R * d * 2, 2 * R * F * d)
     ops["combine"] = ((R * d + T * d) * 2 + T * k * 8, 0)
     ops["combine_bwd"] = ((T * d + 2 * R * d) * 2 + T * k * 12, 0)
-    ops["quant_dy_row"] = (R * d * 2 + q(R * d), 0)
+    ops["quant_dy"] = (R * d * 2 + 2 * q(R * d), 0)
     ops["gemm_dgrad2_swiglu"] = (q(R * d) + q(E * d * F) + 2 * R * 2 * F * 2, 2 * R * d * F)
-    ops["quant_dy_col"] = (R * d * 2 + q(R * d), 0)
-    ops["quant_a_col"] = (R * F * 2 + q(R * F), 0)
     ops["gemm_wgrad2"] = (q(R * d) + q(R * F) + E * d * F * 2, 2 * R * d * F)
-    ops["quant_dh_row"] = (R * 2 * F * 2 + q(R * 2 * F), 0)
+    ops["quant_dh"] = (R * 2 * F * 2 + 2 * q(R * 2 * F), 0)
     ops["gemm_dgrad1"] = (q(R * 2 * F) + q(E * 2 * F * d) + R * d * 2, 4 * R * F * d)
-    ops["quant_dh_col"] = (R * 2 * F * 2 + q(R * 2 * F), 0)
-    ops["quant_x_col"] = (R * d * 2 + q(R * d), 0)
     ops["gemm_wgrad1"] = (q(R * 2 * F) + q(R * d) + E * 2 * F * d * 2, 4 * R * F * d)
     ops["token_reduce"] = ((R * d + T * d) * 2, 0)
     return ops
@@ -217,32 +214,29 @@ class Step:
                 ev[n].record()
             n += 1
 
-        R, ROW, COL = lay.R, L.QUANT_ROW_TILED, L.QUANT_COL_TILED
         cnt, po, ws = lay.counts, lay.poff, lay.ws
+        both = lambda src, n: L.quantize_mxfp8_rowcol(src, qa[n + "q"], qa[n + "s"], qa[n + "tq"],
+                                                      qa[n + "ts"])
         mark(); L.route_metadata(c, lay.idx, lay.counts, lay.offsets, lay.poff, lay.perm, lay.prow,
                                  lay.row_token, ws)
         mark(); L.dispatch(c, inp["x"], lay.prow, cnt, po, lay.x_perm)
-        mark(); L.quantize_mxfp8(lay.x_perm, qa["xq"], qa["xs"], ROW)
+        mark(); both(lay.x_perm, "x")
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_FWD1_SWIGLU, qa["xq"], qa["xs"], qw["W13q"], qw["W13s"],
                                      lay.h13, lay.a, None, cnt, po, ws)
-        mark(); L.quantize_mxfp8(lay.a, qa["aq"], qa["as"], ROW)
+        mark(); both(lay.a, "a")
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_FWD2, qa["aq"], qa["as"], qw["W2q"], qw["W2s"], lay.y,
                                      None, None, cnt, po, ws)
         mark(); L.combine(c, lay.y, lay.gates, lay.prow, lay.out)
         mark(); L.combine_bwd(c, inp["dout"], lay.y, lay.gates, lay.prow, lay.idx, cnt, po, lay.dy,
                               lay.dgates)
-        mark(); L.quantize_mxfp8(lay.dy, qa["dyq"], qa["dys"], ROW)
+        mark(); both(lay.dy, "dy")
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_DGRAD2_SWIGLU, qa["dyq"], qa["dys"], qw["W2tq"],
                                      qw["W2ts"], lay.dh13, None, lay.h13, cnt, po, ws)
-        mark(); L.quantize_mxfp8(lay.dy, qa["dytq"], qa["dyts"], COL)
-        mark(); L.quantize_mxfp8(lay.a, qa["atq"], qa["ats"], COL)
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_WGRAD2, qa["dytq"], qa["dyts"], qa["atq"], qa["ats"],
                                      lay.dW2, None, None, cnt, po, ws)
-        mark(); L.quantize_mxfp8(lay.dh13, qa["dhq"], qa["dhs"], ROW)
+        mark(); both(lay.dh13, "dh")
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_DGRAD1, qa["dhq"], qa["dhs"], qw["W13tq"], qw["W13ts"],
                                      lay.dx_perm, None, None, cnt, po, ws)
-        mark(); L.quantize_mxfp8(lay.dh13, qa["dhtq"], qa["dhts"], COL)
-        mark(); L.quantize_mxfp8(lay.x_perm, qa["xtq"], qa["xts"], COL)
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_WGRAD1, qa["dhtq"], qa["dhts"], qa["xtq"], qa["xts"],
                                      lay.dW13, None, None, cnt, po, ws)
         mark(); L.token_reduce(c, lay.dx_perm, lay.prow, lay.dx)

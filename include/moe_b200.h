@@ -244,6 +244,14 @@ MOE_API int moe_router_wgrad(const moe_config_t* cfg, const void* dlogits, const
 MOE_API int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode, int64_t G, uint8_t* q,
                                uint8_t* s, void* stream);
 
+/* Both tiled quantisations of one operand from a single read of src: MOE_QUANT_ROW_TILED into
+ * (q_row, s_row) and MOE_QUANT_COL_TILED into (q_col, s_col), bit-identical to two moe_quantize_mxfp8
+ * calls. For an activation that one GEMM contracts along its columns and another along its rows
+ * (x_perm, a, dy, dh13 of the layer). rows % 128 == 0, cols % 128 == 0; src and q_col 16-byte
+ * aligned, q_row 8-byte aligned; the four outputs must not overlap. */
+MOE_API int moe_quantize_mxfp8_rowcol(const void* src, int64_t rows, int cols, uint8_t* q_row,
+                                      uint8_t* s_row, uint8_t* q_col, uint8_t* s_col, void* stream);
+
 /* The grouped GEMM of moe_grouped_gemm with MXFP8 operands (tcgen05 kind::mxf8f6f4.block_scale, fp32
  * accumulation, bf16 outputs). Each operand is E4M3 codes in the layout its bf16 counterpart has in
  * moe_grouped_gemm plus UE8M0 scales, tiled, along that GEMM's contraction axis:
@@ -328,9 +336,13 @@ typedef struct {
   uint8_t *W2q, *W2s, *W2tq, *W2ts;
 } moe_mxfp8_weights_t;
 
-/* Quantised routed activations (caller-owned scratch), R32 = moe_max_rows(cfg):
+/* Quantised routed activations (caller-owned), R32 = moe_max_rows(cfg):
  *   x*: x_perm [R32, d]   a*: a [R32, F]   dy*: dy [R32, d]   dh*: dh13 [R32, 2F]
- *   ?q/?s ROW (scales [R32, cols/32]);  ?tq/?ts COL (scales [cols, R32/32]). */
+ *   ?q/?s ROW_TILED (codes [R32, cols], scales R32*cols/32 bytes);
+ *   ?tq/?ts COL_TILED (codes [R32, cols], scales cols*R32/32 bytes).
+ * Each activation is quantised both ways in one pass (moe_quantize_mxfp8_rowcol). The forward writes
+ * x* and a* (both orientations) and the backward reads them, so they are state kept between the two
+ * passes like moe_saved_t; dy* and dh* are backward scratch. */
 typedef struct {
   uint8_t *xq, *xs, *xtq, *xts;
   uint8_t *aq, *as, *atq, *ats;
@@ -342,16 +354,18 @@ typedef struct {
 MOE_API int moe_quantize_weights_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
                                        const moe_mxfp8_weights_t* qw, void* stream);
 
-/* moe_layer_fwd with MXFP8 expert GEMMs (cfg->dtype == MOE_DTYPE_MXFP8, bf16 storage): the routed
- * activations are quantised along each GEMM's contraction axis right before it; SwiGLU, combine and
- * all stored activations stay bf16. A learned router runs in bf16. */
+/* moe_layer_fwd with MXFP8 expert GEMMs (cfg->dtype == MOE_DTYPE_MXFP8, bf16 storage): x_perm and a
+ * are quantised along both axes right after they are written (the row copy feeds the next forward
+ * GEMM, the column copy the backward's weight gradient); SwiGLU, combine and all stored activations
+ * stay bf16. A learned router runs in bf16. Needs all of qa's x* and a* buffers. */
 MOE_API int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
                                 const moe_mxfp8_weights_t* qw, const void* x, const float* bias,
                                 void* out, moe_saved_t* saved, const moe_mxfp8_acts_t* qa, void* ws,
                                 size_t ws_bytes, void* stream);
 
 /* moe_layer_bwd with MXFP8 expert GEMMs (dgrad operands ROW/COL as listed above, wgrad operands COL
- * along the expert's rows, in 32-row blocks of its zero-padded group). */
+ * along the expert's rows, in 32-row blocks of its zero-padded group). Reads qa's x* and a* as the
+ * forward left them; quantises dy and dh13 both ways in one pass each. */
 MOE_API int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
                                 const moe_mxfp8_weights_t* qw, const moe_saved_t* saved,
                                 const moe_mxfp8_acts_t* qa, const void* x, const void* dout, void* dx,

@@ -26,7 +26,7 @@ EXPORTS = [
     "moe_route_topk", "moe_route_metadata", "moe_dispatch", "moe_combine", "moe_combine_bwd",
     "moe_token_reduce", "moe_grouped_gemm", "moe_router_wgrad", "moe_layer_fwd", "moe_layer_bwd",
     "moe_test_bounded_wait", "moe_version", "moe_launch_count", "moe_route_metadata_noalloc",
-    "moe_quantize_mxfp8", "moe_grouped_gemm_mxfp8", "moe_quantize_weights_mxfp8",
+    "moe_quantize_mxfp8", "moe_quantize_mxfp8_rowcol", "moe_grouped_gemm_mxfp8", "moe_quantize_weights_mxfp8",
     "moe_layer_fwd_mxfp8", "moe_layer_bwd_mxfp8",
 ]
 
@@ -96,6 +96,7 @@ def _load():
         "moe_launch_count": ([], ctypes.c_uint64),
         "moe_route_metadata_noalloc": ([cfgp, vp, vp, vp, vp, vp, vp, vp, vp], i),
         "moe_quantize_mxfp8": ([vp, ctypes.c_int64, i, i, ctypes.c_int64, vp, vp, vp], i),
+        "moe_quantize_mxfp8_rowcol": ([vp, ctypes.c_int64, i, vp, vp, vp, vp, vp], i),
         "moe_grouped_gemm_mxfp8": ([cfgp, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], i),
         "moe_quantize_weights_mxfp8": ([cfgp, ctypes.POINTER(Weights), ctypes.POINTER(MxWeights), vp], i),
         "moe_layer_fwd_mxfp8": ([cfgp, ctypes.POINTER(Weights), ctypes.POINTER(MxWeights), vp, vp, vp,
@@ -248,6 +249,13 @@ def quantize_mxfp8(src, q, s, mode, G=0, stream=None):
     rows, cols = src.shape
     check(lib.moe_quantize_mxfp8(ptr(src), rows, cols, mode, int(G), ptr(q), ptr(s),
                                  stream_handle(stream)), "moe_quantize_mxfp8")
+
+
+def quantize_mxfp8_rowcol(src, q_row, s_row, q_col, s_col, stream=None):
+    """Row-block and column-block tiled MXFP8 quantisations of src [rows, cols] in one pass."""
+    rows, cols = src.shape
+    check(lib.moe_quantize_mxfp8_rowcol(ptr(src), rows, cols, ptr(q_row), ptr(s_row), ptr(q_col),
+                                        ptr(s_col), stream_handle(stream)), "moe_quantize_mxfp8_rowcol")
 
 
 def grouped_gemm_mxfp8(cfg, op, Aq, As, Bq, Bs, C, C2, aux, counts, poff, ws, stream=None):

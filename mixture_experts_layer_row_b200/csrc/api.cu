@@ -387,6 +387,15 @@ int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode, int64_
   return launch_quantize(src, rows, cols, mode, G, q, s, S(stream));
 }
 
+int moe_quantize_mxfp8_rowcol(const void* src, int64_t rows, int cols, uint8_t* q_row, uint8_t* s_row,
+                              uint8_t* q_col, uint8_t* s_col, void* stream) {
+  MOE_REQUIRE(src && q_row && s_row && q_col && s_col && rows >= 1 && cols >= 1, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(rows % 128 == 0 && cols % 128 == 0, MOE_ERR_INVALID_ARG);
+  const auto a8 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 7u) == 0; };
+  MOE_REQUIRE(aligned16(src) && a8(q_row) && aligned16(q_col), MOE_ERR_INVALID_ARG);
+  return launch_quantize_rowcol(src, rows, cols, q_row, s_row, q_col, s_col, S(stream));
+}
+
 int moe_grouped_gemm_mxfp8(const moe_config_t* cfg, int op, const uint8_t* Aq, const uint8_t* As,
                            const uint8_t* Bq, const uint8_t* Bs, void* C, void* C2, const void* aux,
                            const int32_t* counts, const int32_t* poff, void* ws, size_t ws_bytes,
@@ -524,7 +533,8 @@ int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
   MOE_REQUIRE(sv->idx && sv->gates && sv->counts && sv->offsets && sv->poff && sv->perm && sv->prow &&
                   sv->row_token && sv->x_perm && sv->h13 && sv->a && sv->y,
               MOE_ERR_INVALID_ARG);
-  MOE_REQUIRE(qa->xq && qa->xs && qa->aq && qa->as, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(qa->xq && qa->xs && qa->xtq && qa->xts && qa->aq && qa->as && qa->atq && qa->ats,
+              MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(aligned16(x) && aligned16(out) && aligned16(sv->x_perm) && aligned16(sv->h13) &&
                   aligned16(sv->a) && aligned16(sv->y),
               MOE_ERR_INVALID_ARG);
@@ -546,10 +556,10 @@ int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
                           s));
   MOE_TRY(launch_dispatch(x, sv->prow, sv->counts, sv->poff, sv->x_perm, cfg->T, cfg->k, cfg->E, d * 2,
                           s));
-  MOE_TRY(launch_quantize(sv->x_perm, R, d, MOE_QUANT_ROW_TILED, 0, qa->xq, qa->xs, s));
+  MOE_TRY(launch_quantize_rowcol(sv->x_perm, R, d, qa->xq, qa->xs, qa->xtq, qa->xts, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_FWD1_SWIGLU, qa->xq, qa->xs, qw->W13q, qw->W13s, sv->h13, sv->a,
                      nullptr, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize(sv->a, R, F, MOE_QUANT_ROW_TILED, 0, qa->aq, qa->as, s));
+  MOE_TRY(launch_quantize_rowcol(sv->a, R, F, qa->aq, qa->as, qa->atq, qa->ats, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_FWD2, qa->aq, qa->as, qw->W2q, qw->W2s, sv->y, nullptr, nullptr,
                      sv->counts, sv->poff, ws, s));
   return launch_combine(sv->y, sv->gates, sv->prow, out, cfg->T, cfg->k, d * 2, true, s);
@@ -587,18 +597,15 @@ int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
   void* dlog = router ? static_cast<void*>(static_cast<char*>(ws) + L.dlogits) : nullptr;
   MOE_TRY(launch_combine_bwd(dout, sv->y, sv->gates, sv->prow, sv->idx, sv->counts, sv->poff, g->dy,
                              g->dgates, dlsel, dlog, cfg->T, cfg->k, cfg->E, d * 2, true, s));
-  MOE_TRY(launch_quantize(g->dy, R, d, MOE_QUANT_ROW_TILED, 0, qa->dyq, qa->dys, s));
+  // dy and dh13: both orientations from one read; x_perm's and a's column copies come from the forward
+  MOE_TRY(launch_quantize_rowcol(g->dy, R, d, qa->dyq, qa->dys, qa->dytq, qa->dyts, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_DGRAD2_SWIGLU, qa->dyq, qa->dys, qw->W2tq, qw->W2ts, g->dh13,
                      nullptr, sv->h13, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize(g->dy, R, d, MOE_QUANT_COL_TILED, 0, qa->dytq, qa->dyts, s));
-  MOE_TRY(launch_quantize(sv->a, R, F, MOE_QUANT_COL_TILED, 0, qa->atq, qa->ats, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD2, qa->dytq, qa->dyts, qa->atq, qa->ats, g->dW2, nullptr,
                      nullptr, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize(g->dh13, R, 2 * F, MOE_QUANT_ROW_TILED, 0, qa->dhq, qa->dhs, s));
+  MOE_TRY(launch_quantize_rowcol(g->dh13, R, 2 * F, qa->dhq, qa->dhs, qa->dhtq, qa->dhts, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_DGRAD1, qa->dhq, qa->dhs, qw->W13tq, qw->W13ts, g->dx_perm, nullptr,
                      nullptr, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize(g->dh13, R, 2 * F, MOE_QUANT_COL_TILED, 0, qa->dhtq, qa->dhts, s));
-  MOE_TRY(launch_quantize(sv->x_perm, R, d, MOE_QUANT_COL_TILED, 0, qa->xtq, qa->xts, s));
   MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD1, qa->dhtq, qa->dhts, qa->xtq, qa->xts, g->dW13, nullptr,
                      nullptr, sv->counts, sv->poff, ws, s));
   MOE_TRY(launch_token_reduce(g->dx_perm, sv->prow, dlsel, router ? sv->idx : nullptr, w->W_r, dx,

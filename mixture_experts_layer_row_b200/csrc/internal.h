@@ -93,6 +93,8 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
                 const GemmParams& p, cudaStream_t s);
 int launch_quantize(const void* src, int64_t rows, int cols, int mode, int64_t G, uint8_t* q,
                     uint8_t* s, cudaStream_t st);
+int launch_quantize_rowcol(const void* src, int64_t rows, int cols, uint8_t* qr, uint8_t* sr,
+                           uint8_t* qc, uint8_t* sc, cudaStream_t st);
 int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s);
 // out[i] = round_to_act(sum over s < nsplit of part[s*stride + i]) for i < n (fixed summation order).
 int launch_split_reduce(const float* part, int nsplit, int64_t n, int64_t stride, void* out, bool bf16,

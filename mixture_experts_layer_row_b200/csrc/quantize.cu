@@ -56,6 +56,13 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Byte mask over four packed column codes that clears the codes of all-zero column blocks (whose
+// values, +0 or -0, would otherwise convert to +0 or -0 codes; an all-zero block has zero codes).
+__device__ __forceinline__ uint32_t zero_block_mask(const float (&amax)[4]) {
+  return (amax[0] > 0.f ? 0x000000FFu : 0u) | (amax[1] > 0.f ? 0x0000FF00u : 0u) |
+         (amax[2] > 0.f ? 0x00FF0000u : 0u) | (amax[3] > 0.f ? 0xFF000000u : 0u);
+}
+
 // Byte offset of the scale of (MN index i, K-block b) in the tiled layout with KB K-blocks per MN index.
 __device__ __forceinline__ int64_t tiled_sf_offset(int64_t i, int64_t b, int64_t KB) {
   return ((i >> 7) * (KB >> 2) + (b >> 2)) * 512 + (i & 31) * 16 + ((i >> 5) & 3) * 4 + (b & 3);
@@ -141,16 +148,118 @@ __global__ void __launch_bounds__(128) quant_col_kernel(const uint2* __restrict_
     inv[j] = amax[j] > 0.f ? exp2_exact(-e) : 0.f;
     s[scale_index(layout, (int64_t)cg * 4 + j, rb, rblocks, 0)] = sb;
   }
+  const uint32_t keep = zero_block_mask(amax);
   uint32_t* qb = q + (rb * 32) * groups + cg;
 #pragma unroll
   for (int r = 0; r < 32; ++r) {
     const uint32_t lo = cvt_e4m3x2(bf16lo(w[r].x) * inv[0], bf16hi(w[r].x) * inv[1]);
     const uint32_t hi = cvt_e4m3x2(bf16lo(w[r].y) * inv[2], bf16hi(w[r].y) * inv[3]);
-    qb[(int64_t)r * groups] = lo | (hi << 16);
+    qb[(int64_t)r * groups] = (lo | (hi << 16)) & keep;
+  }
+}
+
+// Both tiled quantisations of one operand in a single read. A CTA of 128 threads takes a 32-row x
+// 128-column tile: coalesced 16-byte loads into registers and shared memory; row blocks (4 lanes hold
+// one 32-column block) are converted from registers and stored as 8-byte groups; column blocks (one
+// thread per column) are read back from shared memory, converted into a shared code tile and stored
+// as 16-byte rows. Codes and scales are bit-identical to quant_row_kernel / quant_col_kernel with the
+// tiled layout.
+constexpr int kRcRows = 32, kRcCols = 128, kRcThreads = 128;
+
+__global__ void __launch_bounds__(kRcThreads) quant_rowcol_kernel(const uint4* __restrict__ src,
+                                                                  int64_t rows, int cols,
+                                                                  uint2* __restrict__ qr,
+                                                                  uint8_t* __restrict__ sr,
+                                                                  uint4* __restrict__ qc,
+                                                                  uint8_t* __restrict__ sc) {
+  __shared__ __align__(16) uint4 tile[kRcRows * kRcCols / 8];      // bf16 [32][128]
+  __shared__ __align__(16) uint8_t codes[kRcRows * kRcCols];        // column-block codes [32][128]
+  pdl_enter();  // wait for the previous kernel before any global access
+  const int ctiles = cols / kRcCols;
+  const int64_t rb = blockIdx.x / ctiles;
+  const int cb = (int)(blockIdx.x % ctiles);
+  const int t = threadIdx.x;
+  const int64_t row0 = rb * kRcRows;
+  const int64_t w16 = cols / 8;  // 16-byte words per row
+  const int c16 = t & 15;        // this thread's 16-byte column word inside the tile
+  uint4 v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = (t >> 4) + 8 * i;
+    v[i] = src[(row0 + r) * w16 + cb * 16 + c16];
+    tile[r * 16 + c16] = v[i];
+  }
+  // row blocks: lanes 4j..4j+3 hold the 32 columns of one block of one row
+  const int kb = cols / 32;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = (t >> 4) + 8 * i;
+    const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[2 * j] = bf16lo(u[j]);
+      f[2 * j + 1] = bf16hi(u[j]);
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(f[j]));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    uint8_t sb;
+    const float ir = exp2_exact(-block_exponent(m, &sb));
+    uint2 c;
+    c.x = cvt_e4m3x2(f[0] * ir, f[1] * ir) | ((uint32_t)cvt_e4m3x2(f[2] * ir, f[3] * ir) << 16);
+    c.y = cvt_e4m3x2(f[4] * ir, f[5] * ir) | ((uint32_t)cvt_e4m3x2(f[6] * ir, f[7] * ir) << 16);
+    if (!(m > 0.f)) c = make_uint2(0u, 0u);
+    qr[(row0 + r) * w16 + cb * 16 + c16] = c;
+    if ((t & 3) == 0) sr[tiled_sf_offset(row0 + r, (int64_t)cb * 4 + (c16 >> 2), kb)] = sb;
+  }
+  __syncthreads();
+  // column blocks: thread t owns column t of the tile (32 rows)
+  {
+    const __nv_bfloat16* tb = reinterpret_cast<const __nv_bfloat16*>(tile);
+    float f[kRcRows];
+    float amax = 0.f;
+#pragma unroll
+    for (int r = 0; r < kRcRows; ++r) {
+      f[r] = __bfloat162float(tb[r * kRcCols + t]);
+      amax = fmaxf(amax, fabsf(f[r]));
+    }
+    uint8_t sb;
+    const int e = block_exponent(amax, &sb);
+    const float inv = amax > 0.f ? exp2_exact(-e) : 0.f;
+    sc[tiled_sf_offset((int64_t)cb * kRcCols + t, rb, rows / 32)] = sb;
+#pragma unroll
+    for (int r = 0; r < kRcRows; r += 2) {
+      const uint32_t c2 = amax > 0.f ? cvt_e4m3x2(f[r] * inv, f[r + 1] * inv) : 0u;
+      codes[r * kRcCols + t] = (uint8_t)(c2 & 0xFFu);
+      codes[(r + 1) * kRcCols + t] = (uint8_t)(c2 >> 8);
+    }
+  }
+  __syncthreads();
+  const uint4* cw = reinterpret_cast<const uint4*>(codes);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int idx = t + kRcThreads * j;  // 16-byte word of the code tile: 8 per row
+    const int r = idx >> 3, c = idx & 7;
+    qc[((row0 + r) * cols + (int64_t)cb * kRcCols) / 16 + c] = cw[idx];
   }
 }
 
 }  // namespace
+
+// Row-block and column-block tiled quantisations (MOE_QUANT_ROW_TILED into qr/sr, MOE_QUANT_COL_TILED
+// into qc/sc) of one [rows, cols] operand in one pass; rows % 128 == 0, cols % 128 == 0.
+int launch_quantize_rowcol(const void* src, int64_t rows, int cols, uint8_t* qr, uint8_t* sr,
+                           uint8_t* qc, uint8_t* sc, cudaStream_t st) {
+  const int64_t grid = (rows / kRcRows) * (cols / kRcCols);
+  MOE_LAUNCH(launch_pdl(quant_rowcol_kernel, (unsigned)grid, kRcThreads, 0, st,
+                        static_cast<const uint4*>(src), rows, cols, reinterpret_cast<uint2*>(qr), sr,
+                        reinterpret_cast<uint4*>(qc), sc));
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
 // mode: MOE_QUANT_ROW / COL / ROW_TILED / COL_TILED / ROW_TILED_GATEUP (G = gate rows per stack)
 int launch_quantize(const void* src, int64_t rows, int cols, int mode, int64_t G, uint8_t* q,

@@ -46,6 +46,7 @@ def test_quantize_row_bitexact(rows, cols):
 def test_quantize_col_bitexact(rows, cols):
     L = _lib()
     x = _bf16_matrix(rows, cols, 3 * rows + cols)
+    x[:32, 4:8] = -0.0  # an all-zero column block of negative zeros: zero codes
     q = torch.zeros((rows, cols), dtype=torch.uint8, device=dev())
     s = torch.zeros((cols, rows // 32), dtype=torch.uint8, device=dev())
     L.quantize_mxfp8(x.to(dev()), q, s, L.QUANT_COL)
@@ -91,6 +92,34 @@ def test_quantize_tiled_bitexact(rows, cols, mode):
         ref_s = tiled(rs, G)
     assert np.array_equal(q.cpu().numpy(), rq)
     assert np.array_equal(s.cpu().numpy(), ref_s)
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 128), (384, 256), (1024, 2048), (2048, 1536)])
+def test_quantize_rowcol_bitexact(rows, cols):
+    """One pass writing both tiled orientations equals the oracle's row and column quantisers (and
+    so the two single-orientation launches)."""
+    L = _lib()
+    x = _bf16_matrix(rows, cols, 7 * rows + cols)
+    x[5::17, :] = -0.0                                   # negative zeros: all-zero row blocks
+    x[32:64, :4] = -0.0                                  # and all-zero column blocks
+    z = lambda *sh: torch.full(sh, 0xAB, dtype=torch.uint8, device=dev())
+    qr, sr, qc, sc = z(rows, cols), z(rows * cols // 32), z(rows, cols), z(rows * cols // 32)
+    L.quantize_mxfp8_rowcol(x.to(dev()), qr, sr, qc, sc)
+    torch.cuda.synchronize()
+    xn = x.double().numpy()
+    rq, rs = MX.quantize_rows(xn)
+    cq, cs = MX.quantize_cols(xn)
+    assert np.array_equal(qr.cpu().numpy(), rq)
+    assert np.array_equal(sr.cpu().numpy(), tiled(rs))
+    assert np.array_equal(qc.cpu().numpy(), cq)
+    assert np.array_equal(sc.cpu().numpy(), tiled(cs.T))
+    # and the single-orientation kernels agree byte for byte (negative zeros included)
+    q1, s1 = z(rows, cols), z(rows * cols // 32)
+    L.quantize_mxfp8(x.to(dev()), q1, s1, L.QUANT_COL_TILED)
+    q2, s2 = z(rows, cols), z(rows * cols // 32)
+    L.quantize_mxfp8(x.to(dev()), q2, s2, L.QUANT_ROW_TILED)
+    torch.cuda.synchronize()
+    assert torch.equal(q1, qc) and torch.equal(s1, sc) and torch.equal(q2, qr) and torch.equal(s2, sr)
 
 
 SHAPES = {
