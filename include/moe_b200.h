@@ -154,7 +154,7 @@ MOE_API int moe_route_metadata_noalloc(const moe_config_t* cfg, const int32_t* i
 /* Row-wise dispatch (unite.ai, "Parallelismo, precisione e tecniche di memoria": each routed token is
  * written directly into its expert's input buffer): x_perm[prow[t*k+j]] = x[t] for all j, and every
  * pad row [poff[e]+counts[e], poff[e+1]) is zeroed. x: act [T,d]; x_perm: act [max_rows,d] (bf16 in
- * MXFP8 mode, quantised afterwards with moe_quantize_mxfp8). */
+ * MXFP8 mode, quantised afterwards with moe_quantize_mxfp8_rowcol). */
 MOE_API int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* prow, const int32_t* counts,
                  const int32_t* poff, void* x_perm, void* stream);
 
