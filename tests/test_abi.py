@@ -97,6 +97,14 @@ def test_host_validation_before_any_launch(L):
                                   10 ** 9, None) == -1  # unknown op
     assert L.lib.moe_grouped_gemm(c, 0, fake, fake, fake, None, None, fake, fake, fake,
                                   10 ** 9, None) == -1  # SwiGLU forward needs its second output
+    assert L.lib.moe_grouped_gemm(c, 1, fake, fake, None, None, None, fake, fake, fake,
+                                  10 ** 9, None) == -1  # only the SwiGLU forward may omit C
+    rc = L.lib.moe_quantize_mxfp8_rowcol
+    assert rc(fake, 96, 128, fake, fake, fake, fake, None) == -1    # rows % 128
+    assert rc(fake, 128, 96, fake, fake, fake, fake, None) == -1    # cols % 128
+    assert rc(fake, 128, 128, fake, fake, fake + 8, fake, None) == -1  # column codes 16-byte aligned
+    assert rc(fake, 128, 128, fake + 4, fake, fake, fake, None) == -1  # row codes 8-byte aligned
+    assert rc(fake, 128, 128, None, fake, fake, fake, None) == -1
     assert L.lib.moe_get_error(None, None, None) == -1
     mx = L.make_config(64, 64, 128, 8, 2, L.DTYPE_MXFP8)
     # the router GEMM and the bf16/fp32 grouped GEMM entry points do not take MXFP8 configs

@@ -1,0 +1,51 @@
+"""The benchmark's per-op work model (algorithmic bytes and flops behind every roofline figure),
+checked against plain counts on CPU: the op list follows the layer's launch order, the recompute
+variant adds exactly one GEMM1 and drops the h13 store from the forward one, and the MXFP8 step
+counts one read and two quantised writes per activation."""
+import bench
+from moe_workloads import WORKLOADS
+
+
+def test_bf16_op_order_is_the_launch_order():
+    w = WORKLOADS["e128_bf16"]
+    assert list(bench.op_work(w)) == [
+        "route_metadata", "dispatch", "gemm_fwd1_swiglu", "gemm_fwd2", "combine", "combine_bwd",
+        "gemm_dgrad2_swiglu", "gemm_wgrad2", "gemm_dgrad1", "gemm_wgrad1", "token_reduce"]
+
+
+def test_recompute_adds_one_gemm1_and_drops_the_h13_store():
+    w = WORKLOADS["e128_bf16"]
+    R, d, F, E = w.T * w.k, w.d, w.F, w.E
+    st, rc = bench.op_work(w), bench.op_work(w, recompute=True)
+    names = list(rc)
+    assert names.index("gemm_fwd1_recompute") == names.index("combine_bwd") + 1
+    assert names.index("gemm_dgrad2_swiglu") == names.index("gemm_fwd1_recompute") + 1
+    assert rc["gemm_fwd1_recompute"] == st["gemm_fwd1_swiglu"]
+    assert st["gemm_fwd1_swiglu"][0] - rc["gemm_fwd1_swiglu"][0] == R * 2 * F * 2
+    assert rc["gemm_fwd1_swiglu"][1] == st["gemm_fwd1_swiglu"][1] == 2 * R * d * 2 * F
+    # every other op is unchanged
+    for n in st:
+        if n != "gemm_fwd1_swiglu":
+            assert rc[n] == st[n], n
+    # GEMM1 stored: x_perm and W13 read, h13 and a written, all bf16
+    assert st["gemm_fwd1_swiglu"][0] == (R * d + E * 2 * F * d + R * 2 * F + R * F) * 2
+
+
+def test_total_flops_are_the_layer_count():
+    """Six expert GEMMs: 3 forward-equivalents of 2 R d (3F) flops (GEMM1 2F wide, GEMM2 F)."""
+    w = WORKLOADS["e128_bf16"]
+    R = w.T * w.k
+    gemm = sum(f for n, (b, f) in bench.op_work(w).items() if n.startswith("gemm_"))
+    assert gemm == 3 * 2 * R * w.d * 3 * w.F
+
+
+def test_mxfp8_quantisation_counts_one_read_two_writes():
+    w = WORKLOADS["e128_mxfp8"]
+    R, d, F = w.T * w.k, w.d, w.F
+    ops = bench.op_work(w)
+    q = lambda n: n + n // 32
+    assert ops["quant_x"] == (R * d * 2 + 2 * q(R * d), 0)
+    assert ops["quant_a"] == (R * F * 2 + 2 * q(R * F), 0)
+    assert ops["quant_dy"] == (R * d * 2 + 2 * q(R * d), 0)
+    assert ops["quant_dh"] == (R * 2 * F * 2 + 2 * q(R * 2 * F), 0)
+    assert not any(n.endswith("_row") or n.endswith("_col") for n in ops)
