@@ -57,13 +57,11 @@ def load_peaks():
 # algorithmic work per op (bytes moved once, flops of the definition); R = routed rows = T*k
 # ------------------------------------------------------------------------------------------------
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, from ncu captures of the
-# current kernels on the full-size workload (profiles/grouped_gemm_fwd1_e128_bf16.md,
-# profiles/grouped_gemm_wgrad1_e128_bf16.md). A kernel or workload not listed reports null.
-MEASURED_TRAFFIC = {
-    ("e128_bf16", "gemm_fwd1_swiglu"): 1.224964e9 + 0.199070e9,
-    ("e128_bf16", "gemm_wgrad1"): 0.286039e9 + 1.014497e9,
-}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, taken from a committed ncu
+# capture of the kernel as it is now; an entry is removed whenever its kernel changes, so a kernel or
+# workload not listed reports null.
+MEASURED_TRAFFIC = {}
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
 
 
 def op_work_mx(w):
@@ -75,18 +73,17 @@ def op_work_mx(w):
     q = lambda n: n + n // 32          # codes + scales of n elements
     ops = {}
     ops["route_metadata"] = (T * k * 4 * 3 + Rp * 4, 0)
-    ops["dispatch"] = ((T + R) * d * 2, 0)
-    # each activation is quantised along rows and columns in one pass: one bf16 read, two fp8 writes
-    ops["quant_x"] = (R * d * 2 + 2 * q(R * d), 0)
-    ops["gemm_fwd1_swiglu"] = (q(R * d) + q(E * 2 * F * d) + (R * 2 * F + R * F) * 2, 4 * R * d * F)
-    ops["quant_a"] = (R * F * 2 + 2 * q(R * F), 0)
+    # the routed input, a, dy and dh13 exist only in their two quantised forms: their producers read
+    # bf16 once and write the row-block and the column-block codes + scales
+    ops["dispatch_quant"] = (T * d * 2 + R * 4 + 2 * q(R * d), 0)
+    ops["gemm_fwd1_swiglu_quant"] = (q(R * d) + q(E * 2 * F * d) + R * 2 * F * 2 + 2 * q(R * F),
+                                     4 * R * d * F)
     ops["gemm_fwd2"] = (q(R * F) + q(E * d * F) + R * d * 2, 2 * R * F * d)
     ops["combine"] = ((R * d + T * d) * 2 + T * k * 8, 0)
-    ops["combine_bwd"] = ((T * d + 2 * R * d) * 2 + T * k * 12, 0)
-    ops["quant_dy"] = (R * d * 2 + 2 * q(R * d), 0)
-    ops["gemm_dgrad2_swiglu"] = (q(R * d) + q(E * d * F) + 2 * R * 2 * F * 2, 2 * R * d * F)
+    ops["combine_bwd_quant"] = ((T * d + R * d) * 2 + T * k * 8 + R * 4 + 2 * q(R * d), 0)
+    ops["gemm_dgrad2_swiglu_quant"] = (q(R * d) + q(E * d * F) + R * 2 * F * 2 + 2 * q(R * 2 * F),
+                                       2 * R * d * F)
     ops["gemm_wgrad2"] = (q(R * d) + q(R * F) + E * d * F * 2, 2 * R * d * F)
-    ops["quant_dh"] = (R * 2 * F * 2 + 2 * q(R * 2 * F), 0)
     ops["gemm_dgrad1"] = (q(R * 2 * F) + q(E * 2 * F * d) + R * d * 2, 4 * R * F * d)
     ops["gemm_wgrad1"] = (q(R * 2 * F) + q(R * d) + E * 2 * F * d * 2, 4 * R * F * d)
     ops["token_reduce"] = ((R * d + T * d) * 2, 0)
@@ -146,11 +143,25 @@ class Step:
             lay.gates.copy_(inp["gates"])
         self.names = list(op_work(w, recompute=layer.recompute).keys())
         self.ev = None
+        self.only = None  # record only the boundaries of this op (None: every op boundary)
 
-    def events(self, n_steps):
+    def events(self, n_steps, only=None):
+        """Events for the next n_steps runs: at every op boundary (the per-op breakdown), or only
+        around op `only` (every other boundary is left free, so consecutive kernels overlap their
+        launch and prologue through programmatic dependent launch)."""
         import torch
+        self.only = only
         self.ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(self.names) + 1)]
                    for _ in range(n_steps)]
+
+    def op_ms(self, i, name):
+        j = self.names.index(name)
+        return self.ev[i][j].elapsed_time(self.ev[i][j + 1])
+
+    @property
+    def only_idx(self):
+        j = self.names.index(self.only)
+        return (j, j + 1)
 
     def run(self, i=None):
         if self.layer.mx:
@@ -162,7 +173,7 @@ class Step:
 
         def mark():
             nonlocal n
-            if ev is not None:
+            if ev is not None and (self.only is None or n in self.only_idx):
                 ev[n].record()
             n += 1
 
@@ -202,7 +213,8 @@ class Step:
 
 
     def run_mx(self, i=None):
-        """The kernels of moe_layer_fwd_mxfp8 / moe_layer_bwd_mxfp8, op by op (uniform routing)."""
+        """The kernels of moe_layer_fwd_mxfp8 / moe_layer_bwd_mxfp8, op by op (uniform routing): the
+        routed input, a, dy and dh13 leave their producers only as their two quantised forms."""
         L, lay, w, inp = self.L, self.layer, self.w, self.inp
         ev = self.ev[i] if (i is not None and self.ev is not None) else None
         c, qa, qw = lay.cfg, lay.qa_t, lay.qw_t
@@ -210,31 +222,25 @@ class Step:
 
         def mark():
             nonlocal n
-            if ev is not None:
+            if ev is not None and (self.only is None or n in self.only_idx):
                 ev[n].record()
             n += 1
 
-        cnt, po, ws = lay.counts, lay.poff, lay.ws
-        both = lambda src, n: L.quantize_mxfp8_rowcol(src, qa[n + "q"], qa[n + "s"], qa[n + "tq"],
-                                                      qa[n + "ts"])
+        cnt, po, ws, ops = lay.counts, lay.poff, lay.ws, lay.q_ops
         mark(); L.route_metadata(c, lay.idx, lay.counts, lay.offsets, lay.poff, lay.perm, lay.prow,
                                  lay.row_token, ws)
-        mark(); L.dispatch(c, inp["x"], lay.prow, cnt, po, lay.x_perm)
-        mark(); both(lay.x_perm, "x")
-        mark(); L.grouped_gemm_mxfp8(c, L.GEMM_FWD1_SWIGLU, qa["xq"], qa["xs"], qw["W13q"], qw["W13s"],
-                                     lay.h13, lay.a, None, cnt, po, ws)
-        mark(); both(lay.a, "a")
+        mark(); L.dispatch_mxfp8(c, inp["x"], lay.row_token, po, ops["x"])
+        mark(); L.grouped_gemm_mxfp8_quant(c, L.GEMM_FWD1_SWIGLU, qa["xq"], qa["xs"], qw["W13q"],
+                                           qw["W13s"], lay.h13, None, ops["a"], cnt, po, ws)
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_FWD2, qa["aq"], qa["as"], qw["W2q"], qw["W2s"], lay.y,
                                      None, None, cnt, po, ws)
         mark(); L.combine(c, lay.y, lay.gates, lay.prow, lay.out)
-        mark(); L.combine_bwd(c, inp["dout"], lay.y, lay.gates, lay.prow, lay.idx, cnt, po, lay.dy,
-                              lay.dgates)
-        mark(); both(lay.dy, "dy")
-        mark(); L.grouped_gemm_mxfp8(c, L.GEMM_DGRAD2_SWIGLU, qa["dyq"], qa["dys"], qw["W2tq"],
-                                     qw["W2ts"], lay.dh13, None, lay.h13, cnt, po, ws)
+        mark(); L.combine_bwd_mxfp8(c, inp["dout"], lay.y, lay.gates, lay.row_token, po, lay.dgates,
+                                    ops["dy"])
+        mark(); L.grouped_gemm_mxfp8_quant(c, L.GEMM_DGRAD2_SWIGLU, qa["dyq"], qa["dys"], qw["W2tq"],
+                                           qw["W2ts"], None, lay.h13, ops["dh"], cnt, po, ws)
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_WGRAD2, qa["dytq"], qa["dyts"], qa["atq"], qa["ats"],
                                      lay.dW2, None, None, cnt, po, ws)
-        mark(); both(lay.dh13, "dh")
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_DGRAD1, qa["dhq"], qa["dhs"], qw["W13tq"], qw["W13ts"],
                                      lay.dx_perm, None, None, cnt, po, ws)
         mark(); L.grouped_gemm_mxfp8(c, L.GEMM_WGRAD1, qa["dhtq"], qa["dhts"], qa["xtq"], qa["xts"],
@@ -413,12 +419,63 @@ def run_reference(args, w):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(w),
+            "data": "synthetic", "config": dict(workload_config(w), parallelism=f"replicas x{args.gpus}"),
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": blas_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def gemm_peak(args):
+    """Dense throughput of this library's own tcgen05 grouped GEMM on one square problem (one expert
+    holding every row: M = N = K = 8192), forward GEMM2 op (K-major operands, plain bf16 store): bf16
+    on CTA pairs, or MXFP8 block-scaled (E4M3 operands, UE8M0 scales). CUDA events around 20 launches
+    after 5 warm-up launches, nvidia-smi clocks sampled meanwhile. Prints one JSON line."""
+    import torch
+    from mixture_experts_layer_row_b200 import _lib as L
+    torch.cuda.set_device(0)
+    n = 8192
+    mx = args.gemm_peak == "mxfp8"
+    cfg = L.make_config(n, n, n, 1, 1, L.DTYPE_MXFP8 if mx else L.DTYPE_BF16)
+    R = L.max_rows(cfg)
+    dev = torch.device("cuda", 0)
+    ws = torch.zeros(L.workspace_size(cfg), dtype=torch.uint8, device=dev)
+    counts = torch.tensor([n], dtype=torch.int32, device=dev)
+    poff = torch.tensor([0, n], dtype=torch.int32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(0)
+    A = torch.zeros((R, n), dtype=torch.bfloat16, device=dev)
+    A[:n] = torch.randn((n, n), generator=g, device=dev).to(torch.bfloat16)
+    B = (torch.randn((n, n), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    C = torch.empty((R, n), dtype=torch.bfloat16, device=dev)
+    if mx:
+        q = lambda t: (torch.empty(t.shape, dtype=torch.uint8, device=dev),
+                       torch.empty(t.numel() // 32, dtype=torch.uint8, device=dev))
+        (Aq, As), (Bq, Bs) = q(A), q(B)
+        L.quantize_mxfp8(A, Aq, As, L.QUANT_ROW_TILED)
+        L.quantize_mxfp8(B, Bq, Bs, L.QUANT_ROW_TILED)
+        run = lambda: L.grouped_gemm_mxfp8(cfg, L.GEMM_FWD2, Aq, As, Bq, Bs, C, None, None, counts, poff, ws)
+    else:
+        run = lambda: L.grouped_gemm(cfg, L.GEMM_FWD2, A, B, C, None, None, counts, poff, ws)
+    for _ in range(5):
+        run()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(20):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / 20
+    flops = 2.0 * n * n * n
+    print(json.dumps({"gemm_peak": args.gemm_peak, "M": n, "N": n, "K": n, "ms": ms,
+                      "tflops": flops / (ms / 1e3) / 1e12, "clocks": clk,
+                      "error_flags": L.get_error(ws)}), flush=True)
     return 0
 
 
@@ -444,6 +501,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--experts", type=int, default=0,
                     help="expert-count sweep: the workload's shapes with E experts, uniform routing")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="the workload's shapes with T tokens (smaller cases for ncu captures)")
+    ap.add_argument("--gemm-peak", default="",
+                    choices=["", "bf16", "mxfp8"],
+                    help="time this library's grouped GEMM on one large square group (E=1) and print its "
+                         "TFLOP/s instead of the layer step")
     ap.add_argument("--recompute", action="store_true",
                     help="activation recompute: the layer keeps no h13 and the backward regenerates it; "
                          "also times it against stored activations through the layer API")
@@ -453,6 +516,10 @@ def main():
     w = WORKLOADS[args.workload]
     if args.experts:
         w = w.scaled(E=args.experts, routing="uniform", skew=0.0, name=f"{w.name}_E{args.experts}")
+    if args.tokens:
+        w = w.scaled(T=args.tokens, name=f"{w.name}_T{args.tokens}")
+    if args.gemm_peak:
+        return gemm_peak(args)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -497,7 +564,21 @@ def main():
 
     for _ in range(args.warmup):
         step.run()
+    # per-op breakdown: an instrumented pass of K steps with an event at every op boundary (each event
+    # also serialises the two kernels around it, so these per-op times include launch gaps)
     step.events(args.steps)
+    for i in range(args.steps):
+        step.run(i)
+    torch.cuda.synchronize()
+    per_op = {n: 0.0 for n in step.names}
+    for i in range(args.steps):
+        for n in step.names:
+            per_op[n] += step.op_ms(i, n)
+    per_op = {n: v / args.steps for n, v in per_op.items()}
+    dom = max(per_op, key=lambda n: per_op[n])
+    # timed region: K steps issued back to back as the layer API issues them, with events only around
+    # the dominant kernel (its duration for the roofline)
+    step.events(args.steps, only=dom)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -522,13 +603,8 @@ def main():
     # activations and scratch (the MXFP8 path adds the quantised copies)
     peak_mem_gb = torch.cuda.max_memory_allocated() / 1e9
 
-    # per-op durations over the timed region
-    per_op = {n: 0.0 for n in step.names}
-    for i in range(args.steps):
-        ev = step.ev[i]
-        for j, n in enumerate(step.names):
-            per_op[n] += ev[j].elapsed_time(ev[j + 1])
-    per_op = {n: v / args.steps for n, v in per_op.items()}
+    # the dominant kernel's duration inside the timed region
+    dom_ms = sum(step.op_ms(i, dom) for i in range(args.steps)) / args.steps
 
     peaks = load_peaks()
     work = op_work(w, 4 if w.dtype == "fp32" else 2, recompute=layer.recompute)
@@ -540,22 +616,28 @@ def main():
     roof_time = 0.0
     for n, (b, f) in work.items():
         roof_time += max(b / (bw * 1e9), f / (tc * 1e12))
+    # every HBM-bound kernel's achieved bandwidth against the measured copy peak and the nominal 8 TB/s
+    hbm_ops = {}
+    for n, (b, f) in work.items():
+        if b / (bw * 1e9) >= f / (tc * 1e12):
+            gbs = b / (per_op[n] / 1e3) / 1e9
+            hbm_ops[n] = {"GB/s": round(gbs, 1), "frac_measured": round(gbs / bw, 3),
+                          "frac_nominal": round(gbs / NOMINAL_HBM_GBS, 3)}
     gemm_ops = [n for n in work if n.startswith("gemm_")]
     gemm_flops = sum(work[n][1] for n in gemm_ops)
     gemm_ms = sum(per_op[n] for n in gemm_ops)
-    dom = max(per_op, key=lambda n: per_op[n])
     b, f = work[dom]
-    t_dom = per_op[dom] / 1e3
+    t_dom = dom_ms / 1e3
     if b / (bw * 1e9) >= f / (tc * 1e12) or f == 0:
         roof = {"kernel": dom, "bound": "hbm", "achieved": b / t_dom / 1e9, "peak": bw, "unit": "GB/s",
                 "frac": (b / t_dom / 1e9) / bw, "traffic": MEASURED_TRAFFIC.get((w.name, dom)),
-                "algorithmic_bytes": b, "flops": f, "ms": per_op[dom],
+                "algorithmic_bytes": b, "flops": f, "ms": dom_ms,
                 "peak_source": f"{peaks['source']} hbm_gbs"}
     else:
         roof = {"kernel": dom, "bound": "tensor", "achieved": f / t_dom / 1e12, "peak": tc,
                 "unit": "TFLOP/s", "frac": (f / t_dom / 1e12) / tc,
                 "traffic": MEASURED_TRAFFIC.get((w.name, dom)),
-                "algorithmic_bytes": b, "flops": f, "ms": per_op[dom],
+                "algorithmic_bytes": b, "flops": f, "ms": dom_ms,
                 "peak_source": f"{peaks['source']} bf16_tflops (burst) x {ratio} ({w.dtype})"}
 
     wq = None
@@ -712,6 +794,9 @@ def main():
                                "peaks": peaks},
             "roofline": roof,
             "per_op_ms": {n: round(v, 4) for n, v in per_op.items()},
+            "per_op_note": "instrumented pass of K steps with an event at every op boundary, run before "
+                           "the timed region (each event serialises the kernels around it)",
+            "per_op_hbm": hbm_ops,
             "weight_quantisation": wq,
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -125,7 +125,9 @@ MOE_API int moe_route_topk(const moe_config_t* cfg, const float* logits, const f
  *                  expert (a stable counting sort; deterministic, no atomics in the ordering);
  *   prow[T*k]      padded row of entry t*k+j: poff[e] + perm - offsets[e];
  *   row_token[max_rows]  entry t*k+j held by each padded row, -1 for pad rows and unused rows.
- * An expert id outside [0,E) sets MOE_DEVERR_ROUTING; such entries are skipped. */
+ * An expert id outside [0,E) sets MOE_DEVERR_ROUTING; such an entry gets no row (perm = prow = -1),
+ * and dispatch, combine, combine_bwd and the token reduce skip every entry whose prow lies outside
+ * [0, max_rows): nothing is read or written through it. */
 MOE_API int moe_route_metadata(const moe_config_t* cfg, const int32_t* idx, int32_t* counts,
                        int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
                        int32_t* row_token, void* ws, size_t ws_bytes, void* stream);
@@ -140,11 +142,13 @@ MOE_API int moe_route_metadata(const moe_config_t* cfg, const int32_t* idx, int3
  *   - Limit: ceil(T/256) * E <= 65536 (e.g. T = 131072 at E = 128); larger requests return
  *     MOE_ERR_WORKSPACE and enqueue nothing.
  *   - The first call on a device looks up the scratch's device address (cudaGetSymbolAddress, with
- *     that device current); make that first call before any stream capture.
+ *     that device current), and so does the first call after the device's context has been
+ *     re-created (cudaDeviceReset); make such a call before any stream capture.
  *   - Every call on a device shares the one array: calls that overlap on the GPU (other streams, other
  *     host threads) race and corrupt each other's results. Order them on one stream.
  *   - Nothing in the scratch needs clearing (each call writes all it reads). Device-side routing
- *     errors (expert ids outside [0,E)) are skipped but not reported: there is no error flag. */
+ *     errors (expert ids outside [0,E)) are not reported, since there is no error flag; such entries
+ *     get perm = prow = -1 as in moe_route_metadata. */
 MOE_API int moe_route_metadata_noalloc(const moe_config_t* cfg, const int32_t* idx, int32_t* counts,
                                        int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
                                        int32_t* row_token, void* stream);
@@ -158,12 +162,15 @@ MOE_API int moe_route_metadata_noalloc(const moe_config_t* cfg, const int32_t* i
 MOE_API int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* prow, const int32_t* counts,
                  const int32_t* poff, void* x_perm, void* stream);
 
-/* Gate-weighted combine: out[t] = sum_j gates[t,j] * y[prow[t*k+j]] (fp32 accumulation, a gather:
+/* Gate-weighted combine (the pages are silent on the combine; this is the gate-weighted sum over the
+ * token's k experts that the layer's definition gives): out[t] = sum_j gates[t,j] * y[prow[t*k+j]]
+ * (fp32 accumulation, a gather:
  * deterministic, no atomics). y: act [max_rows,d]; out: act [T,d]. */
 MOE_API int moe_combine(const moe_config_t* cfg, const void* y, const float* gates, const int32_t* prow,
                 void* out, void* stream);
 
-/* Backward of the combine: dy[prow[t*k+j]] = gates[t,j] * dout[t]; dgates[t,j] = <dout[t], y[row]>.
+/* Backward of the combine (pages silent; the exact derivative of moe_combine):
+ * dy[prow[t*k+j]] = gates[t,j] * dout[t]; dgates[t,j] = <dout[t], y[row]>.
  * Pad rows of dy are zeroed. When dlsel is non-NULL (learned router, renormalised gates) it also
  * writes dlsel[t,j] = g_j (dg_j - sum_i g_i dg_i), the score gradient of the chosen experts, and,
  * when dlogits is non-NULL, the dense score gradient dlogits[t,e] (act [T,E], zero for experts
@@ -173,7 +180,8 @@ MOE_API int moe_combine_bwd(const moe_config_t* cfg, const void* dout, const voi
                     const int32_t* poff, void* dy, float* dgates, float* dlsel, void* dlogits,
                     void* stream);
 
-/* Scatter-add of routed-row gradients back to tokens, done as a deterministic gather-sum:
+/* Scatter-add of routed-row gradients back to tokens (pages silent; the exact derivative of the
+ * dispatch), done as a deterministic gather-sum:
  * dx[t] = sum_j dx_perm[prow[t*k+j]] (+ sum_j dlsel[t,j] * W_r[idx[t,j]] when dlsel, idx and W_r
  * are all non-NULL: the router's input gradient). dx_perm: act [max_rows,d]; dx: act [T,d]. */
 MOE_API int moe_token_reduce(const moe_config_t* cfg, const void* dx_perm, const int32_t* prow,
@@ -252,6 +260,37 @@ MOE_API int moe_quantize_mxfp8(const void* src, int64_t rows, int cols, int mode
 MOE_API int moe_quantize_mxfp8_rowcol(const void* src, int64_t rows, int cols, uint8_t* q_row,
                                       uint8_t* s_row, uint8_t* q_col, uint8_t* s_col, void* stream);
 
+/* One MXFP8 operand in both tiled orientations (caller-owned), for a routed-row activation [R, cols]
+ * with R = moe_max_rows(cfg): row-block codes q_row [R, cols] + scales s_row (MOE_QUANT_ROW_TILED,
+ * R*cols/32 bytes; 4-byte aligned) for the GEMM that contracts along the columns, and column-block
+ * codes q_col [R, cols] + scales s_col (MOE_QUANT_COL_TILED over 32-row blocks of the expert groups,
+ * cols*R/32 bytes) for the weight gradient that contracts over the expert's rows. Code arrays are
+ * 16-byte aligned. */
+typedef struct {
+  uint8_t *q_row, *s_row, *q_col, *s_col;
+} moe_mxfp8_operand_t;
+
+/* Row-wise dispatch straight into MXFP8 expert buffers (unite.ai, "Parallelismo, precisione e
+ * tecniche di memoria": tokens are written directly into their experts' buffers, and MXFP8 cuts the
+ * expert data moved): the routed buffer x_perm[r] = x[row_token[r] / k] (zero for pad rows) is formed
+ * and quantised in one pass -- no bf16 x_perm is written. Codes and scales are bit-identical to
+ * moe_dispatch followed by moe_quantize_mxfp8_rowcol on rows [0, poff[E]); rows at or past poff[E] are
+ * not written (no GEMM reads them). x: bf16 [T,d] (16-byte aligned); row_token, poff: from
+ * moe_route_metadata; out: [R, d] operand. cfg->dtype must be MOE_DTYPE_MXFP8, d % 128 == 0. */
+MOE_API int moe_dispatch_mxfp8(const moe_config_t* cfg, const void* x, const int32_t* row_token,
+                               const int32_t* poff, const moe_mxfp8_operand_t* out, void* stream);
+
+/* Backward of the combine straight into MXFP8 (the pages are silent on the backward's formulas; this
+ * is the exact derivative of the combine): dy[r] = bf16(gates[n] * dout[n / k]) with n = row_token[r]
+ * (zero for pad rows) is formed and quantised in one pass -- no bf16 dy is written -- and
+ * dgates[n] = <dout[n / k], y[r]> (fp32, fixed summation order). Codes and scales are bit-identical to
+ * quantising the bf16 dy that moe_combine_bwd writes. dout: bf16 [T,d]; y: bf16 [R,d]; gates, dgates:
+ * fp32 [T,k]; dy: [R, d] operand. Score gradients of a learned router are not computed here
+ * (moe_layer_bwd_mxfp8 adds them). cfg->dtype must be MOE_DTYPE_MXFP8, d % 128 == 0. */
+MOE_API int moe_combine_bwd_mxfp8(const moe_config_t* cfg, const void* dout, const void* y,
+                                  const float* gates, const int32_t* row_token, const int32_t* poff,
+                                  float* dgates, const moe_mxfp8_operand_t* dy, void* stream);
+
 /* The grouped GEMM of moe_grouped_gemm with MXFP8 operands (tcgen05 kind::mxf8f6f4.block_scale, fp32
  * accumulation, bf16 outputs). Each operand is E4M3 codes in the layout its bf16 counterpart has in
  * moe_grouped_gemm plus UE8M0 scales, tiled, along that GEMM's contraction axis:
@@ -268,6 +307,19 @@ MOE_API int moe_grouped_gemm_mxfp8(const moe_config_t* cfg, int op, const uint8_
                                    const uint8_t* Bq, const uint8_t* Bs, void* C, void* C2,
                                    const void* aux, const int32_t* counts, const int32_t* poff,
                                    void* ws, size_t ws_bytes, void* stream);
+
+/* The two MXFP8 SwiGLU GEMMs with their activation output quantised in the epilogue (both tiled
+ * orientations of its bf16 value; no bf16 copy of it is written). Operands as for
+ * moe_grouped_gemm_mxfp8:
+ *   MOE_GEMM_FWD1_SWIGLU   C = h13 bf16 [R,2F] (kept for the backward), out = a [R, F];
+ *   MOE_GEMM_DGRAD2_SWIGLU aux = h13 bf16, C unused (may be NULL), out = dh13 [R, 2F].
+ * Codes and scales are bit-identical to moe_quantize_mxfp8_rowcol of the bf16 output that
+ * moe_grouped_gemm_mxfp8 writes for the same op. Other ops: MOE_ERR_INVALID_ARG. */
+MOE_API int moe_grouped_gemm_mxfp8_quant(const moe_config_t* cfg, int op, const uint8_t* Aq,
+                                         const uint8_t* As, const uint8_t* Bq, const uint8_t* Bs,
+                                         void* C, const void* aux, const moe_mxfp8_operand_t* out,
+                                         const int32_t* counts, const int32_t* poff, void* ws,
+                                         size_t ws_bytes, void* stream);
 
 /* ---- whole layer ------------------------------------------------------------------------------------ */
 
@@ -340,9 +392,9 @@ typedef struct {
  *   x*: x_perm [R32, d]   a*: a [R32, F]   dy*: dy [R32, d]   dh*: dh13 [R32, 2F]
  *   ?q/?s ROW_TILED (codes [R32, cols], scales R32*cols/32 bytes);
  *   ?tq/?ts COL_TILED (codes [R32, cols], scales cols*R32/32 bytes).
- * Each activation is quantised both ways in one pass (moe_quantize_mxfp8_rowcol). The forward writes
- * x* and a* (both orientations) and the backward reads them, so they are state kept between the two
- * passes like moe_saved_t; dy* and dh* are backward scratch. */
+ * Each activation exists only in these two quantised forms (see moe_layer_fwd_mxfp8). Kept from the
+ * forward to the backward: the column forms xtq/xts and atq/ats (the weight gradients' operands).
+ * xq/xs and aq/as are forward scratch, dy* and dh* backward scratch. */
 typedef struct {
   uint8_t *xq, *xs, *xtq, *xts;
   uint8_t *aq, *as, *atq, *ats;
@@ -354,18 +406,21 @@ typedef struct {
 MOE_API int moe_quantize_weights_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
                                        const moe_mxfp8_weights_t* qw, void* stream);
 
-/* moe_layer_fwd with MXFP8 expert GEMMs (cfg->dtype == MOE_DTYPE_MXFP8, bf16 storage): x_perm and a
- * are quantised along both axes right after they are written (the row copy feeds the next forward
- * GEMM, the column copy the backward's weight gradient); SwiGLU, combine and all stored activations
- * stay bf16. A learned router runs in bf16. Needs all of qa's x* and a* buffers. */
+/* moe_layer_fwd with MXFP8 expert GEMMs (cfg->dtype == MOE_DTYPE_MXFP8): the dispatch writes the
+ * routed input only in its two quantised forms (moe_dispatch_mxfp8) and GEMM1's epilogue writes a only
+ * in its two quantised forms (moe_grouped_gemm_mxfp8_quant); h13 and y are kept in bf16, SwiGLU and the
+ * combine run on bf16 values. saved->x_perm and saved->a are not used (may be NULL). A learned router
+ * runs in bf16. Needs all of qa's x* and a* buffers. */
 MOE_API int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
                                 const moe_mxfp8_weights_t* qw, const void* x, const float* bias,
                                 void* out, moe_saved_t* saved, const moe_mxfp8_acts_t* qa, void* ws,
                                 size_t ws_bytes, void* stream);
 
 /* moe_layer_bwd with MXFP8 expert GEMMs (dgrad operands ROW/COL as listed above, wgrad operands COL
- * along the expert's rows, in 32-row blocks of its zero-padded group). Reads qa's x* and a* as the
- * forward left them; quantises dy and dh13 both ways in one pass each. */
+ * along the expert's rows, in 32-row blocks of its zero-padded group). Reads qa's column forms of x and
+ * a as the forward left them; dy comes straight out of the combine backward and dh13 out of the
+ * SwiGLU-backward epilogue in their two quantised forms only (moe_combine_bwd_mxfp8,
+ * moe_grouped_gemm_mxfp8_quant). grads->dy and grads->dh13 are not used (may be NULL). */
 MOE_API int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
                                 const moe_mxfp8_weights_t* qw, const moe_saved_t* saved,
                                 const moe_mxfp8_acts_t* qa, const void* x, const void* dout, void* dx,

@@ -27,7 +27,8 @@ EXPORTS = [
     "moe_token_reduce", "moe_grouped_gemm", "moe_router_wgrad", "moe_layer_fwd", "moe_layer_bwd",
     "moe_test_bounded_wait", "moe_version", "moe_launch_count", "moe_route_metadata_noalloc",
     "moe_quantize_mxfp8", "moe_quantize_mxfp8_rowcol", "moe_grouped_gemm_mxfp8", "moe_quantize_weights_mxfp8",
-    "moe_layer_fwd_mxfp8", "moe_layer_bwd_mxfp8",
+    "moe_layer_fwd_mxfp8", "moe_layer_bwd_mxfp8", "moe_dispatch_mxfp8", "moe_combine_bwd_mxfp8",
+    "moe_grouped_gemm_mxfp8_quant",
 ]
 
 
@@ -58,6 +59,10 @@ class Grads(ctypes.Structure):
 class MxWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("W13q", "W13s", "W13tq", "W13ts", "W2q", "W2s", "W2tq", "W2ts")]
+
+
+class MxOperand(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("q_row", "s_row", "q_col", "s_col")]
 
 
 class MxActs(ctypes.Structure):
@@ -104,6 +109,10 @@ def _load():
         "moe_layer_bwd_mxfp8": ([cfgp, ctypes.POINTER(Weights), ctypes.POINTER(MxWeights),
                                  ctypes.POINTER(Saved), ctypes.POINTER(MxActs), vp, vp, vp,
                                  ctypes.POINTER(Grads), vp, sz, vp], i),
+        "moe_dispatch_mxfp8": ([cfgp, vp, vp, vp, ctypes.POINTER(MxOperand), vp], i),
+        "moe_combine_bwd_mxfp8": ([cfgp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(MxOperand), vp], i),
+        "moe_grouped_gemm_mxfp8_quant": ([cfgp, i, vp, vp, vp, vp, vp, vp, ctypes.POINTER(MxOperand),
+                                          vp, vp, vp, sz, vp], i),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -263,6 +272,34 @@ def grouped_gemm_mxfp8(cfg, op, Aq, As, Bq, Bs, C, C2, aux, counts, poff, ws, st
     check(lib.moe_grouped_gemm_mxfp8(ctypes.byref(cfg), int(op), ptr(Aq), ptr(As), ptr(Bq), ptr(Bs),
                                      ptr(C), ptr(C2), ptr(aux), ptr(counts), ptr(poff), w, n,
                                      stream_handle(stream)), "moe_grouped_gemm_mxfp8")
+
+
+def mx_operand(q_row, s_row, q_col, s_col) -> MxOperand:
+    """Both tiled MXFP8 forms of one routed-row activation (device buffers)."""
+    return MxOperand(ptr(q_row), ptr(s_row), ptr(q_col), ptr(s_col))
+
+
+def dispatch_mxfp8(cfg, x, row_token, poff, out: MxOperand, stream=None):
+    """Row-wise dispatch of x into the routed buffer's two MXFP8 forms (no bf16 copy)."""
+    check(lib.moe_dispatch_mxfp8(ctypes.byref(cfg), ptr(x), ptr(row_token), ptr(poff), ctypes.byref(out),
+                                 stream_handle(stream)), "moe_dispatch_mxfp8")
+
+
+def combine_bwd_mxfp8(cfg, dout, y, gates, row_token, poff, dgates, dy: MxOperand, stream=None):
+    """Combine backward into dy's two MXFP8 forms (no bf16 dy) and the gate gradients."""
+    check(lib.moe_combine_bwd_mxfp8(ctypes.byref(cfg), ptr(dout), ptr(y), ptr(gates), ptr(row_token),
+                                    ptr(poff), ptr(dgates), ctypes.byref(dy), stream_handle(stream)),
+          "moe_combine_bwd_mxfp8")
+
+
+def grouped_gemm_mxfp8_quant(cfg, op, Aq, As, Bq, Bs, C, aux, out: MxOperand, counts, poff, ws,
+                             stream=None):
+    """The MXFP8 SwiGLU GEMMs with their activation output quantised in the epilogue."""
+    w, n = _ws(ws)
+    check(lib.moe_grouped_gemm_mxfp8_quant(ctypes.byref(cfg), int(op), ptr(Aq), ptr(As), ptr(Bq),
+                                           ptr(Bs), ptr(C), ptr(aux), ctypes.byref(out), ptr(counts),
+                                           ptr(poff), w, n, stream_handle(stream)),
+          "moe_grouped_gemm_mxfp8_quant")
 
 
 def quantize_weights_mxfp8(cfg, weights: Weights, qw: MxWeights, stream=None):

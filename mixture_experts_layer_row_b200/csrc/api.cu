@@ -216,6 +216,53 @@ int gemm_op_mx(const moe_config_t* c, int op, const uint8_t* Aq, const uint8_t* 
   }
 }
 
+// The MXFP8 SwiGLU GEMMs whose activation output leaves quantised (row-block codes for the next
+// GEMM, column-block codes for a weight gradient): FWD1_SWIGLU (C = h13, bf16; out = a) and
+// DGRAD2_SWIGLU (aux = h13; out = dh13, no bf16 copy).
+int gemm_op_mx_quant(const moe_config_t* c, int op, const uint8_t* Aq, const uint8_t* As,
+                     const uint8_t* Bq, const uint8_t* Bs, void* Cout, const void* aux,
+                     const moe_mxfp8_operand_t* out, const int32_t* counts, const int32_t* poff,
+                     void* ws, cudaStream_t s) {
+  const int64_t R = r32_of(c);
+  const int d = c->d, F = c->F, E = c->E;
+  GemmParams p = base_params(c, ws);
+  p.counts = counts;
+  p.poff = poff;
+  p.C = Cout;
+  p.sA = As;
+  p.sB = Bs;
+  p.q_qr = out->q_row;
+  p.q_sr = out->s_row;
+  p.q_qc = out->q_col;
+  p.q_sc = out->s_col;
+  p.q_kb_col = R / 32;
+  GemmOperand a{Aq, 0, 0, 0}, b{Bq, 0, 0, 0};
+  switch (op) {
+    case MOE_GEMM_FWD1_SWIGLU:
+      a = {Aq, R, d, d};
+      b = {Bq, (int64_t)E * 2 * F, d, d};
+      p.K = d; p.N = F; p.b_rows_per_group = 2 * F; p.ldc = 2 * F;
+      p.sA_ld = d / 128; p.sB_ld = d / 128;
+      p.q_kb_row = F / 32;
+      return launch_gemm(GK_FWD1_SWIGLU_Q, 1, 128, a, b, p, s);
+    case MOE_GEMM_DGRAD2_SWIGLU:
+      MOE_REQUIRE(aux && aligned16(aux), MOE_ERR_INVALID_ARG);
+      a = {Aq, R, d, d};
+      b = {Bq, (int64_t)E * d, F, F};
+      p.K = d; p.N = F; p.b_rows_per_group = d; p.aux = aux; p.ldaux = 2 * F; p.ldc = 2 * F;
+      p.sA_ld = d / 128; p.sB_ld = (int64_t)E * d / 128;
+      p.q_kb_row = 2 * F / 32;
+      return launch_gemm(GK_DGRAD2_SWIGLU_Q, 1, 128, a, b, p, s);
+    default:
+      return MOE_ERR_INVALID_ARG;
+  }
+}
+
+bool operand_ok(const moe_mxfp8_operand_t* o) {
+  return o && o->q_row && o->s_row && o->q_col && o->s_col && aligned16(o->q_row) &&
+         aligned16(o->q_col) && ((reinterpret_cast<uintptr_t>(o->s_row) & 3u) == 0);
+}
+
 int router_logits_impl(const moe_config_t* c, const void* x, const void* Wr, const float* bias,
                        float* logits, void* ws, cudaStream_t s) {
   GemmParams p = base_params(c, ws);
@@ -322,7 +369,7 @@ int moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* prow, co
   MOE_REQUIRE(x && prow && counts && poff && x_perm, MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(aligned16(x) && aligned16(x_perm), MOE_ERR_INVALID_ARG);
   return launch_dispatch(x, prow, counts, poff, x_perm, cfg->T, cfg->k, cfg->E, cfg->d * es_of(cfg),
-                         S(stream));
+                         max_rows_of(cfg), S(stream));
 }
 
 int moe_combine(const moe_config_t* cfg, const void* y, const float* gates, const int32_t* prow,
@@ -331,7 +378,7 @@ int moe_combine(const moe_config_t* cfg, const void* y, const float* gates, cons
   MOE_REQUIRE(y && gates && prow && out, MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(aligned16(y) && aligned16(out), MOE_ERR_INVALID_ARG);
   return launch_combine(y, gates, prow, out, cfg->T, cfg->k, cfg->d * es_of(cfg), es_of(cfg) == 2,
-                        S(stream));
+                        max_rows_of(cfg), S(stream));
 }
 
 int moe_combine_bwd(const moe_config_t* cfg, const void* dout, const void* y, const float* gates,
@@ -344,7 +391,8 @@ int moe_combine_bwd(const moe_config_t* cfg, const void* dout, const void* y, co
   MOE_REQUIRE(!dlogits || (dlsel && idx), MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(!dlsel || cfg->renorm == 1, MOE_ERR_UNSUPPORTED);
   return launch_combine_bwd(dout, y, gates, prow, idx, counts, poff, dy, dgates, dlsel, dlogits,
-                            cfg->T, cfg->k, cfg->E, cfg->d * es_of(cfg), es_of(cfg) == 2, S(stream));
+                            cfg->T, cfg->k, cfg->E, cfg->d * es_of(cfg), es_of(cfg) == 2,
+                            max_rows_of(cfg), S(stream));
 }
 
 int moe_token_reduce(const moe_config_t* cfg, const void* dx_perm, const int32_t* prow,
@@ -353,7 +401,7 @@ int moe_token_reduce(const moe_config_t* cfg, const void* dx_perm, const int32_t
   MOE_REQUIRE(dx_perm && prow && dx, MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(aligned16(dx_perm) && aligned16(dx) && (!W_r || aligned16(W_r)), MOE_ERR_INVALID_ARG);
   return launch_token_reduce(dx_perm, prow, dlsel, idx, W_r, dx, cfg->T, cfg->k, cfg->E,
-                             cfg->d * es_of(cfg), es_of(cfg) == 2, S(stream));
+                             cfg->d * es_of(cfg), es_of(cfg) == 2, max_rows_of(cfg), S(stream));
 }
 
 int moe_grouped_gemm(const moe_config_t* cfg, int op, const void* A, const void* B, void* C, void* C2,
@@ -410,6 +458,45 @@ int moe_grouped_gemm_mxfp8(const moe_config_t* cfg, int op, const uint8_t* Aq, c
   return gemm_op_mx(cfg, op, Aq, As, Bq, Bs, C, C2, aux, counts, poff, ws, S(stream));
 }
 
+int moe_dispatch_mxfp8(const moe_config_t* cfg, const void* x, const int32_t* row_token,
+                       const int32_t* poff, const moe_mxfp8_operand_t* out, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(cfg->dtype == MOE_DTYPE_MXFP8, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(cfg->d % 128 == 0, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(x && row_token && poff && operand_ok(out) && aligned16(x), MOE_ERR_INVALID_ARG);
+  return launch_dispatch_quant(x, row_token, poff + cfg->E, cfg->k, max_rows_of(cfg), cfg->d,
+                               out->q_row, out->s_row, out->q_col, out->s_col, S(stream));
+}
+
+int moe_combine_bwd_mxfp8(const moe_config_t* cfg, const void* dout, const void* y, const float* gates,
+                          const int32_t* row_token, const int32_t* poff, float* dgates,
+                          const moe_mxfp8_operand_t* dy, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(cfg->dtype == MOE_DTYPE_MXFP8, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(cfg->d % 128 == 0, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(dout && y && gates && row_token && poff && dgates && operand_ok(dy), MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(dout) && aligned16(y), MOE_ERR_INVALID_ARG);
+  return launch_combine_bwd_quant(dout, y, gates, row_token, poff + cfg->E, cfg->k, max_rows_of(cfg),
+                                  cfg->d, dgates, dy->q_row, dy->s_row, dy->q_col, dy->s_col,
+                                  S(stream));
+}
+
+int moe_grouped_gemm_mxfp8_quant(const moe_config_t* cfg, int op, const uint8_t* Aq, const uint8_t* As,
+                                 const uint8_t* Bq, const uint8_t* Bs, void* C, const void* aux,
+                                 const moe_mxfp8_operand_t* out, const int32_t* counts,
+                                 const int32_t* poff, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  MOE_REQUIRE(cfg->dtype == MOE_DTYPE_MXFP8, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(cfg->d % 128 == 0, MOE_ERR_UNSUPPORTED);
+  MOE_REQUIRE(op == MOE_GEMM_FWD1_SWIGLU || op == MOE_GEMM_DGRAD2_SWIGLU, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(Aq && As && Bq && Bs && counts && poff && operand_ok(out), MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(op != MOE_GEMM_FWD1_SWIGLU || (C && aligned16(C)), MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(Aq) && aligned16(Bq), MOE_ERR_INVALID_ARG);
+  return gemm_op_mx_quant(cfg, op, Aq, As, Bq, Bs, op == MOE_GEMM_FWD1_SWIGLU ? C : nullptr, aux, out,
+                          counts, poff, ws, S(stream));
+}
+
 int moe_router_wgrad(const moe_config_t* cfg, const void* dlogits, const void* x, void* dW_r, void* ws,
                      size_t ws_bytes, void* stream) {
   MOE_TRY(check_cfg(cfg));
@@ -448,13 +535,13 @@ int moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* w, const void* x
                           sv->counts, sv->offsets, sv->poff, sv->perm, sv->prow, sv->row_token, hist,
                           err_of(ws), s));
   MOE_TRY(launch_dispatch(x, sv->prow, sv->counts, sv->poff, sv->x_perm, cfg->T, cfg->k, cfg->E,
-                          cfg->d * es_of(cfg), s));
+                          cfg->d * es_of(cfg), max_rows_of(cfg), s));
   MOE_TRY(gemm_op(cfg, MOE_GEMM_FWD1_SWIGLU, sv->x_perm, w->W13, sv->h13, sv->a, nullptr, sv->counts,
                   sv->poff, ws, s));
   MOE_TRY(gemm_op(cfg, MOE_GEMM_FWD2, sv->a, w->W2, sv->y, nullptr, nullptr, sv->counts, sv->poff, ws,
                   s));
   return launch_combine(sv->y, sv->gates, sv->prow, out, cfg->T, cfg->k, cfg->d * es_of(cfg),
-                        es_of(cfg) == 2, s);
+                        es_of(cfg) == 2, max_rows_of(cfg), s);
 }
 
 int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_saved_t* sv,
@@ -481,7 +568,8 @@ int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_sav
   const int rb = cfg->d * es_of(cfg);
   const bool bf = es_of(cfg) == 2;
   MOE_TRY(launch_combine_bwd(dout, sv->y, sv->gates, sv->prow, sv->idx, sv->counts, sv->poff, g->dy,
-                             g->dgates, dlsel, dlog, cfg->T, cfg->k, cfg->E, rb, bf, s));
+                             g->dgates, dlsel, dlog, cfg->T, cfg->k, cfg->E, rb, bf, max_rows_of(cfg),
+                             s));
   // Activation recompute (the forward kept no h13): GEMM1 regenerates h13 into the dh13 buffer and a
   // into saved->a; the SwiGLU-backward GEMM then overwrites h13 with dh13 in place (each element is
   // read and written by the same tile, the read first).
@@ -500,7 +588,7 @@ int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_sav
   MOE_TRY(gemm_op(cfg, MOE_GEMM_WGRAD1, g->dh13, sv->x_perm, g->dW13, nullptr, nullptr, sv->counts,
                   sv->poff, ws, s));
   MOE_TRY(launch_token_reduce(g->dx_perm, sv->prow, dlsel, router ? sv->idx : nullptr, w->W_r, dx,
-                              cfg->T, cfg->k, cfg->E, rb, bf, s));
+                              cfg->T, cfg->k, cfg->E, rb, bf, max_rows_of(cfg), s));
   if (router) MOE_TRY(router_wgrad_impl(cfg, dlog, x, g->dW_r, ws, s));
   return MOE_OK;
 }
@@ -531,16 +619,16 @@ int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
   MOE_REQUIRE(cfg->d % 128 == 0, MOE_ERR_UNSUPPORTED);
   MOE_REQUIRE(w && qw && qa && sv && x && out, MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(sv->idx && sv->gates && sv->counts && sv->offsets && sv->poff && sv->perm && sv->prow &&
-                  sv->row_token && sv->x_perm && sv->h13 && sv->a && sv->y,
+                  sv->row_token && sv->h13 && sv->y,
               MOE_ERR_INVALID_ARG);
-  MOE_REQUIRE(qa->xq && qa->xs && qa->xtq && qa->xts && qa->aq && qa->as && qa->atq && qa->ats,
-              MOE_ERR_INVALID_ARG);
-  MOE_REQUIRE(aligned16(x) && aligned16(out) && aligned16(sv->x_perm) && aligned16(sv->h13) &&
-                  aligned16(sv->a) && aligned16(sv->y),
+  const moe_mxfp8_operand_t xo{qa->xq, qa->xs, qa->xtq, qa->xts};
+  const moe_mxfp8_operand_t ao{qa->aq, qa->as, qa->atq, qa->ats};
+  MOE_REQUIRE(operand_ok(&xo) && operand_ok(&ao), MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(aligned16(x) && aligned16(out) && aligned16(sv->h13) && aligned16(sv->y),
               MOE_ERR_INVALID_ARG);
   cudaStream_t s = S(stream);
   const int64_t R = max_rows_of(cfg);
-  const int d = cfg->d, F = cfg->F;
+  const int d = cfg->d;
   if (w->W_r) {
     MOE_REQUIRE(sv->logits && aligned16(w->W_r) && aligned16(sv->logits), MOE_ERR_INVALID_ARG);
     moe_config_t rc = *cfg;
@@ -554,15 +642,15 @@ int moe_layer_fwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
   MOE_TRY(launch_metadata(sv->idx, cfg->T, cfg->E, cfg->k, group_align(cfg->dtype), R, sv->counts,
                           sv->offsets, sv->poff, sv->perm, sv->prow, sv->row_token, hist, err_of(ws),
                           s));
-  MOE_TRY(launch_dispatch(x, sv->prow, sv->counts, sv->poff, sv->x_perm, cfg->T, cfg->k, cfg->E, d * 2,
-                          s));
-  MOE_TRY(launch_quantize_rowcol(sv->x_perm, R, d, qa->xq, qa->xs, qa->xtq, qa->xts, s));
-  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_FWD1_SWIGLU, qa->xq, qa->xs, qw->W13q, qw->W13s, sv->h13, sv->a,
-                     nullptr, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize_rowcol(sv->a, R, F, qa->aq, qa->as, qa->atq, qa->ats, s));
-  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_FWD2, qa->aq, qa->as, qw->W2q, qw->W2s, sv->y, nullptr, nullptr,
+  // row-wise dispatch straight into the quantised expert buffers (no bf16 x_perm)
+  MOE_TRY(launch_dispatch_quant(x, sv->row_token, sv->poff + cfg->E, cfg->k, R, d, xo.q_row, xo.s_row,
+                                xo.q_col, xo.s_col, s));
+  // GEMM1 + SwiGLU: h13 in bf16 for the backward, a only as its two quantised forms
+  MOE_TRY(gemm_op_mx_quant(cfg, MOE_GEMM_FWD1_SWIGLU, xo.q_row, xo.s_row, qw->W13q, qw->W13s, sv->h13,
+                           nullptr, &ao, sv->counts, sv->poff, ws, s));
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_FWD2, ao.q_row, ao.s_row, qw->W2q, qw->W2s, sv->y, nullptr, nullptr,
                      sv->counts, sv->poff, ws, s));
-  return launch_combine(sv->y, sv->gates, sv->prow, out, cfg->T, cfg->k, d * 2, true, s);
+  return launch_combine(sv->y, sv->gates, sv->prow, out, cfg->T, cfg->k, d * 2, true, R, s);
 }
 
 int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const moe_mxfp8_weights_t* qw,
@@ -574,12 +662,13 @@ int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
   MOE_REQUIRE(cfg->dtype == MOE_DTYPE_MXFP8, MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(cfg->d % 128 == 0, MOE_ERR_UNSUPPORTED);
   MOE_REQUIRE(w && qw && qa && sv && g && x && dout && dx, MOE_ERR_INVALID_ARG);
-  MOE_REQUIRE(g->dW13 && g->dW2 && g->dgates && g->dy && g->dh13 && g->dx_perm, MOE_ERR_INVALID_ARG);
-  MOE_REQUIRE(qa->xtq && qa->xts && qa->atq && qa->ats && qa->dyq && qa->dys && qa->dytq && qa->dyts &&
-                  qa->dhq && qa->dhs && qa->dhtq && qa->dhts,
+  MOE_REQUIRE(g->dW13 && g->dW2 && g->dgates && g->dx_perm, MOE_ERR_INVALID_ARG);
+  const moe_mxfp8_operand_t dyo{qa->dyq, qa->dys, qa->dytq, qa->dyts};
+  const moe_mxfp8_operand_t dho{qa->dhq, qa->dhs, qa->dhtq, qa->dhts};
+  MOE_REQUIRE(operand_ok(&dyo) && operand_ok(&dho) && qa->xtq && qa->xts && qa->atq && qa->ats,
               MOE_ERR_INVALID_ARG);
   MOE_REQUIRE(aligned16(dout) && aligned16(dx) && aligned16(g->dW13) && aligned16(g->dW2) &&
-                  aligned16(g->dy) && aligned16(g->dh13) && aligned16(g->dx_perm),
+                  aligned16(g->dx_perm) && aligned16(sv->h13) && aligned16(sv->y),
               MOE_ERR_INVALID_ARG);
   const bool router = w->W_r != nullptr;
   moe_config_t rc = *cfg;
@@ -591,25 +680,27 @@ int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
   }
   cudaStream_t s = S(stream);
   const int64_t R = max_rows_of(cfg);
-  const int d = cfg->d, F = cfg->F;
+  const int d = cfg->d;
   const WsLayout L = ws_layout(cfg);
   float* dlsel = router ? reinterpret_cast<float*>(static_cast<char*>(ws) + L.dlsel) : nullptr;
   void* dlog = router ? static_cast<void*>(static_cast<char*>(ws) + L.dlogits) : nullptr;
-  MOE_TRY(launch_combine_bwd(dout, sv->y, sv->gates, sv->prow, sv->idx, sv->counts, sv->poff, g->dy,
-                             g->dgates, dlsel, dlog, cfg->T, cfg->k, cfg->E, d * 2, true, s));
-  // dy and dh13: both orientations from one read; x_perm's and a's column copies come from the forward
-  MOE_TRY(launch_quantize_rowcol(g->dy, R, d, qa->dyq, qa->dys, qa->dytq, qa->dyts, s));
-  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_DGRAD2_SWIGLU, qa->dyq, qa->dys, qw->W2tq, qw->W2ts, g->dh13,
-                     nullptr, sv->h13, sv->counts, sv->poff, ws, s));
-  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD2, qa->dytq, qa->dyts, qa->atq, qa->ats, g->dW2, nullptr,
+  // combine backward straight into dy's quantised forms (no bf16 dy), and the gate gradients
+  MOE_TRY(launch_combine_bwd_quant(dout, sv->y, sv->gates, sv->row_token, sv->poff + cfg->E, cfg->k, R,
+                                   d, g->dgates, dyo.q_row, dyo.s_row, dyo.q_col, dyo.s_col, s));
+  if (router)
+    MOE_TRY(launch_score_grad(sv->gates, g->dgates, sv->idx, dlsel, dlog, cfg->T, cfg->k, cfg->E,
+                              true, s));
+  // GEMM2 dgrad + SwiGLU backward: dh13 only as its two quantised forms
+  MOE_TRY(gemm_op_mx_quant(cfg, MOE_GEMM_DGRAD2_SWIGLU, dyo.q_row, dyo.s_row, qw->W2tq, qw->W2ts,
+                           nullptr, sv->h13, &dho, sv->counts, sv->poff, ws, s));
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD2, dyo.q_col, dyo.s_col, qa->atq, qa->ats, g->dW2, nullptr,
                      nullptr, sv->counts, sv->poff, ws, s));
-  MOE_TRY(launch_quantize_rowcol(g->dh13, R, 2 * F, qa->dhq, qa->dhs, qa->dhtq, qa->dhts, s));
-  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_DGRAD1, qa->dhq, qa->dhs, qw->W13tq, qw->W13ts, g->dx_perm, nullptr,
-                     nullptr, sv->counts, sv->poff, ws, s));
-  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD1, qa->dhtq, qa->dhts, qa->xtq, qa->xts, g->dW13, nullptr,
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_DGRAD1, dho.q_row, dho.s_row, qw->W13tq, qw->W13ts, g->dx_perm,
+                     nullptr, nullptr, sv->counts, sv->poff, ws, s));
+  MOE_TRY(gemm_op_mx(cfg, MOE_GEMM_WGRAD1, dho.q_col, dho.s_col, qa->xtq, qa->xts, g->dW13, nullptr,
                      nullptr, sv->counts, sv->poff, ws, s));
   MOE_TRY(launch_token_reduce(g->dx_perm, sv->prow, dlsel, router ? sv->idx : nullptr, w->W_r, dx,
-                              cfg->T, cfg->k, cfg->E, d * 2, true, s));
+                              cfg->T, cfg->k, cfg->E, d * 2, true, R, s));
   if (router) MOE_TRY(router_wgrad_impl(&rc, dlog, x, g->dW_r, ws, s));
   return MOE_OK;
 }

@@ -426,4 +426,105 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+
+// ---------------------------------------------------------------------------------------------
+// MXFP8 encoding (OCP Microscaling Formats v1.0: E4M3 elements, one UE8M0 scale per 32-element block)
+//   block exponent e = floor(log2(amax)) - 8 (8 = E4M3's largest exponent), clamped to [-127, 127];
+//   scale byte = e + 127; code = round-to-nearest-even(x * 2^-e) saturated to +-448;
+//   an all-zero block gets scale byte 0 and zero codes.
+// ---------------------------------------------------------------------------------------------
+// floor(log2(a)) for a finite a > 0 given as fp32 bits.
+__device__ __forceinline__ int floor_log2_bits(uint32_t bits) {
+  const int ex = (int)((bits >> 23) & 0xFFu);
+  if (ex != 0) return ex - 127;
+  const uint32_t man = bits & 0x7FFFFFu;  // subnormal: man * 2^-149
+  return -149 + (31 - __clz(man));
+}
+
+// 2^k as an fp32 value for k in [-127, 127] (2^-127 is subnormal, still exact).
+__device__ __forceinline__ float exp2_exact(int k) {
+  return k >= -126 ? __int_as_float((k + 127) << 23) : __int_as_float(1 << (k + 149));
+}
+
+// Block exponent and scale byte for a block with maximum magnitude amax (>= 0).
+__device__ __forceinline__ int block_exponent(float amax, uint8_t* scale_byte) {
+  if (!(amax > 0.f)) {
+    *scale_byte = 0;
+    return 127;  // unused: all codes are zero
+  }
+  int e = floor_log2_bits(__float_as_uint(amax)) - 8;
+  e = e < -127 ? -127 : (e > 127 ? 127 : e);
+  *scale_byte = (uint8_t)(e + 127);
+  return e;
+}
+
+// Two floats -> two E4M3 codes (round to nearest even, saturate to finite), packed lo | hi << 8.
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Byte mask over four packed column codes that clears the codes of all-zero column blocks (whose
+// values, +0 or -0, would otherwise convert to +0 or -0 codes; an all-zero block has zero codes).
+__device__ __forceinline__ uint32_t zero_block_mask(const float (&amax)[4]) {
+  return (amax[0] > 0.f ? 0x000000FFu : 0u) | (amax[1] > 0.f ? 0x0000FF00u : 0u) |
+         (amax[2] > 0.f ? 0x00FF0000u : 0u) | (amax[3] > 0.f ? 0xFF000000u : 0u);
+}
+
+// Byte offset of the scale of (MN index i, K-block b) in the tiled layout with KB K-blocks per MN index.
+__device__ __forceinline__ int64_t tiled_sf_offset(int64_t i, int64_t b, int64_t KB) {
+  return ((i >> 7) * (KB >> 2) + (b >> 2)) * 512 + (i & 31) * 16 + ((i >> 5) & 3) * 4 + (b & 3);
+}
+
+// The MXFP8 quantisations of a warp's 32 rows x 32 columns, one row per lane (v = this lane's row,
+// already rounded to the stored precision).
+// Row block: the lane's 32 values -> 32 codes (8 words, column order) and the block's scale byte.
+__device__ __forceinline__ uint8_t mx_row_block(const float (&v)[32], uint32_t (&c)[8]) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(v[i]));
+  uint8_t sb;
+  const float ir = exp2_exact(-block_exponent(m, &sb));
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    c[i] = m > 0.f ? ((uint32_t)cvt_e4m3x2(v[4 * i] * ir, v[4 * i + 1] * ir) |
+                      ((uint32_t)cvt_e4m3x2(v[4 * i + 2] * ir, v[4 * i + 3] * ir) << 16))
+                   : 0u;
+  return sb;
+}
+// Column blocks: column j of the warp's 32 rows is one block. The 32 column maxima come out of a
+// transposing butterfly (lane L ends with column L's maximum), the scales are broadcast back, and
+// each lane converts its own row; returns the scale byte of column `lane`.
+__device__ __forceinline__ uint8_t mx_col_blocks(const float (&v)[32], int lane, uint32_t (&c)[8]) {
+  float m[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) m[i] = fabsf(v[i]);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;  // keep columns [off, 2off) of the current range, else [0, off)
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? m[i] : m[i + off];
+      const float keep = upper ? m[i + off] : m[i];
+      m[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
+    }
+  }
+  uint8_t sb;
+  const int e = block_exponent(m[0], &sb);
+  const float inv_mine = m[0] > 0.f ? exp2_exact(-e) : 0.f;
+  const uint32_t nz = __ballot_sync(0xffffffffu, m[0] > 0.f);  // columns whose block is not all zero
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = v[4 * i + q] * __shfl_sync(0xffffffffu, inv_mine, 4 * i + q);
+    uint32_t word = (uint32_t)cvt_e4m3x2(w[0], w[1]) | ((uint32_t)cvt_e4m3x2(w[2], w[3]) << 16);
+    const uint32_t keep = ((nz >> (4 * i)) & 1u ? 0x000000FFu : 0u) | ((nz >> (4 * i + 1)) & 1u ? 0x0000FF00u : 0u) |
+                          ((nz >> (4 * i + 2)) & 1u ? 0x00FF0000u : 0u) | ((nz >> (4 * i + 3)) & 1u ? 0xFF000000u : 0u);
+    c[i] = word & keep;
+  }
+  return sb;
+}
+
 }  // namespace moe

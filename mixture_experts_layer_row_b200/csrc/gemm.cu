@@ -27,6 +27,10 @@
 // tcgen05.mma.cta_group::2 (M=256) that reads both CTAs' shared memory and writes each CTA's 128
 // accumulator rows into that CTA's TMEM, and its commits arrive on both CTAs' barriers. Each CTA's
 // epilogue drains its own rows and releases the accumulator with a remote arrive on the leader.
+// A pair tile with at most 128 of its group's rows left (an expert's ragged tail) runs as an M = 128
+// pair MMA instead: each CTA holds 64 rows of A, and its accumulator keeps those 64 rows with output
+// columns [0, BN/2) in TMEM lanes 0-63 and [BN/2, BN) in lanes 64-127, so no tensor work goes to
+// rows past the group.
 // Every mbarrier wait is bounded; on a timeout the CTA raises MOE_DEVERR_TIMEOUT, drains what it has
 // in flight (bounded), frees TMEM and returns.
 #include "internal.h"
@@ -41,6 +45,10 @@ constexpr int kEpiThreads = 128;
 
 constexpr int kSmemBudget = 232448;  // 227 KB of opt-in shared memory per CTA
 constexpr int kCtrlBytes = 2048;      // mbarriers, TMEM slot, abort word, tile prefix [<=257 ints]
+
+constexpr bool epi_swiglu_fwd(int e) { return e == EPI_SWIGLU_FWD || e == EPI_SWIGLU_FWD_Q; }
+constexpr bool epi_swiglu_bwd(int e) { return e == EPI_SWIGLU_BWD || e == EPI_SWIGLU_BWD_Q; }
+constexpr bool epi_quant(int e) { return e == EPI_SWIGLU_FWD_Q || e == EPI_SWIGLU_BWD_Q; }
 
 template <int ES, bool A_MN, bool B_MN, int BN, int EPI, int MODE, bool PAIR>
 struct Cfg {
@@ -66,8 +74,13 @@ struct Cfg {
   // accumulators in TMEM: two (the epilogue drains one while the MMA fills the other), or one for
   // MXFP8 tiles of 256 columns, whose per-stage scale columns leave no room for a second
   static constexpr int NACC = (MX && BN == 256) ? 1 : 2;
+  static_assert(!epi_quant(EPI) || (MX && !PAIR), "quantising epilogues are MXFP8-only");
+  // staging boxes per epilogue warp: SwiGLU forward h13 gate + up + a (quantising: gate + up + a's row
+  // codes + a's column codes); SwiGLU backward dh13 gate + up (quantising: row and column codes of
+  // each); stores round robin over NBUF boxes
   static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3
-                              : (EPI == EPI_SWIGLU_BWD) ? 2  // one (gate, up) pair of boxes per warp
+                              : epi_quant(EPI)        ? 4
+                              : (EPI == EPI_SWIGLU_BWD) ? 2
                               : (NACC == 1 ? 1 : 2);
   static constexpr int STAGING_BYTES = 4 * NBUF * 4096;
   // MXFP8: per stage, one 512-byte scale chunk per 128 rows of A and of B (TMEM: 4 columns each)
@@ -79,9 +92,12 @@ struct Cfg {
   static_assert(STAGES >= 2, "pipeline too shallow");
   static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;  // accumulators (+ scale columns)
   static_assert(!MX || NACC * BN + STAGES * SF_COLS <= 512, "TMEM overflow");
-  static constexpr int BN_OUT = (EPI == EPI_SWIGLU_FWD) ? BN / 2 : BN;  // output columns per tile
+  static constexpr int BN_OUT = epi_swiglu_fwd(EPI) ? BN / 2 : BN;  // output columns per tile
   static constexpr uint32_t IDESC =
       MX ? instr_desc_mx(A_MN, B_MN, BM, BN) : instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, TILE_M, BN);
+  // pair tail tile: M = 128 over the pair, HALF_M rows of A per CTA
+  static constexpr int HALF_M = BM / 2;
+  static constexpr uint32_t IDESC_HALF = PAIR ? instr_desc(ES == 2 ? 1u : 2u, A_MN, B_MN, BM, BN) : IDESC;
   // MN-major operands: 16-bit types use the plain 128B swizzle (8-row atoms of 1 KB); 32-bit (tf32)
   // operands need the 128B swizzle with 32-byte chunks (4-row atoms of 512 B).
   static constexpr uint32_t MN_LAYOUT = ES == 4 ? kLayoutSW128Atom32 : kLayoutSW128;
@@ -108,6 +124,13 @@ __device__ __forceinline__ int ti_rows(const TileInfo& ti, const GemmParams& p) 
 }
 __device__ __forceinline__ int ti_row_base(const TileInfo& ti) { return ti.lo; }  // GROUP_M
 __device__ __forceinline__ int ti_kstart(const TileInfo& ti) { return ti.lo; }    // GROUP_K
+
+// A pair tile with at most BM of its group's rows left runs as an M = 128 pair MMA (64 rows per CTA).
+template <bool PAIR, int MODE>
+__device__ __forceinline__ bool ti_half(const TileInfo& ti, const GemmParams& p) {
+  if constexpr (PAIR && MODE == GROUP_M) return ti_rows<MODE>(ti, p) - ti.m0 <= BM;
+  else return false;
+}
 
 // K stages of a tile: GROUP_M K/BK; GROUP_K the group's 32-row contraction chunks, CHUNKS per stage
 template <class C, int MODE>
@@ -211,6 +234,14 @@ __device__ __forceinline__ void stage_row32(uint8_t* box, int lane, int ch0, con
   }
 }
 
+// Write 32 one-byte codes (8 words, column order) of this thread's row into a staged 32-row x 128-byte
+// box (128B swizzle) at 32-byte position `pos` (0..3).
+__device__ __forceinline__ void stage_codes32(uint8_t* box, int lane, int pos, const uint32_t (&c)[8]) {
+  uint8_t* row = box + lane * 128;
+  st_shared_v4(row + (((2 * pos) ^ (lane & 7)) << 4), make_uint4(c[0], c[1], c[2], c[3]));
+  st_shared_v4(row + (((2 * pos + 1) ^ (lane & 7)) << 4), make_uint4(c[4], c[5], c[6], c[7]));
+}
+
 // Hand a fully written box to the TMA unit: every lane fences its writes, lane 0 stores the box.
 __device__ __forceinline__ void box_store(const CUtensorMap* map, const uint8_t* box, int lane, int c0,
                                           int c1) {
@@ -253,7 +284,13 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmC,
-                        const __grid_constant__ CUtensorMap tmC2, const GemmParams p) {
+                        const __grid_constant__ CUtensorMap tmC2,
+                        const __grid_constant__ CUtensorMap tmX1,
+                        const __grid_constant__ CUtensorMap tmX2, const GemmParams p) {
+  // tmX1 / tmX2: pair tail tiles -- 64-row boxes of A / of B (SwiGLU forward); quantising epilogues --
+  // the row-block / column-block code outputs
+  const CUtensorMap& tmA64 = tmX1;
+  const CUtensorMap& tmB64 = tmX2;
   using C = Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>;
   static_assert(MODE == GROUP_M || (A_MN && B_MN), "wgrad mode needs MN-major operands");
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -300,6 +337,14 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     prefetch_tensormap(&tmB);
     prefetch_tensormap(&tmC);
     if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmC2);
+    if constexpr (epi_quant(EPI)) {
+      prefetch_tensormap(&tmX1);
+      prefetch_tensormap(&tmX2);
+    }
+    if constexpr (PAIR && MODE == GROUP_M) {
+      prefetch_tensormap(&tmA64);
+      if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmB64);
+    }
   }
   if (warp == 1) {
     if constexpr (PAIR) {
@@ -379,10 +424,14 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
         const TileInfo ti = nxt;
         if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
         const int nst = num_kstages<C, MODE>(ti, p);
-        const bool a0 = ti.m0 < ti_rows<MODE>(ti, p), a1 = ti.m0 + BM < ti_rows<MODE>(ti, p);
+        // tail tile (<= BM rows left): 64 rows of A per CTA for an M = 128 pair MMA
+        const bool half = ti_half<PAIR, MODE>(ti, p);
+        const int cta_rows = half ? C::HALF_M : BM;
+        const uint32_t a_bytes = (uint32_t)cta_rows * 128;
+        const bool a0 = ti.m0 < ti_rows<MODE>(ti, p), a1 = ti.m0 + cta_rows < ti_rows<MODE>(ti, p);
         const bool mine = rank == 0 ? a0 : a1;
-        const uint32_t tx = (a0 ? C::A_BYTES : 0) + (a1 ? C::A_BYTES : 0) + 2 * C::B_BYTES;
-        const int m_cta = ti.m0 + (int)rank * BM;
+        const uint32_t tx = (a0 ? a_bytes : 0) + (a1 ? a_bytes : 0) + 2 * C::B_BYTES;
+        const int m_cta = ti.m0 + (int)rank * cta_rows;
         const int n_cta = ti.n0 + (int)rank * C::BN_CTA;
         for (int ks = 0; ks < nst; ++ks, ++it) {
           const int s = it % C::STAGES;
@@ -397,13 +446,22 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           if (rank == 0) mbar_arrive_expect_tx(&full[s], tx);
           if constexpr (MODE == GROUP_M) {
             const int k0 = ks * C::BK;
-            if (mine) tma_load_2d_pair(a_dst, &tmA, fb, k0, ti_row_base(ti) + m_cta);
+            if (mine) tma_load_2d_pair(a_dst, half ? &tmA64 : &tmA, fb, k0, ti_row_base(ti) + m_cta);
             const int brow = ti.e * p.b_rows_per_group;
             if constexpr (B_MN) {
               tma_load_3d_pair(b_dst, &tmB, fb, 0, brow + k0, n_cta / C::EPR);
-            } else if constexpr (EPI == EPI_SWIGLU_FWD) {
-              // leader: the gate rows of the tile's outputs; peer: the matching up rows
-              tma_load_2d_pair(b_dst, &tmB, fb, k0, brow + (rank ? p.F : 0) + ti.n0);
+            } else if constexpr (epi_swiglu_fwd(EPI)) {
+              if (!half) {
+                // leader: the gate rows of the tile's outputs; peer: the matching up rows
+                tma_load_2d_pair(b_dst, &tmB, fb, k0, brow + (rank ? p.F : 0) + ti.n0);
+              } else {
+                // M = 128: the accumulator's lanes 0-63 take B columns [0, BN/2) (the leader's half),
+                // lanes 64-127 columns [BN/2, BN) (the peer's). Each CTA loads 64 gate rows and the
+                // 64 matching up rows, so each lane holds gate and up for the same output columns.
+                const int g0 = brow + ti.n0 + (int)rank * (BN / 4);
+                tma_load_2d_pair(b_dst, &tmB64, fb, k0, g0);
+                tma_load_2d_pair(b_dst + (BN / 4) * 128, &tmB64, fb, k0, g0 + p.F);
+              }
             } else {
               tma_load_2d_pair(b_dst, &tmB, fb, k0, brow + n_cta);
             }
@@ -450,7 +508,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               if constexpr (B_MN) {
                 bmb = ti.n0 >> 7;
                 bkq = (int64_t)ti.e * (p.b_rows_per_group >> 7) + ks;
-              } else if constexpr (EPI == EPI_SWIGLU_FWD) {
+              } else if constexpr (epi_swiglu_fwd(EPI)) {
                 bmb = ((int64_t)ti.e * p.b_rows_per_group + ti.n0) >> 7;  // gate rows n0..n0+BN/2-1
                 bkq = ks;
               } else {
@@ -466,7 +524,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             sf_b = p.sB + (bmb * p.sB_ld + bkq) * 512;
             // the tile's second 128 B rows: the next chunk row, or for the fused SwiGLU tile (gate
             // rows, then the up rows F further down W13) the chunk row F/128 further
-            b_chunk_step = (EPI == EPI_SWIGLU_FWD ? (int64_t)(p.F >> 7) : 1) * p.sB_ld * 512;
+            b_chunk_step = (epi_swiglu_fwd(EPI) ? (int64_t)(p.F >> 7) : 1) * p.sB_ld * 512;
             sf_dst = sf;
           }
           if constexpr (MODE == GROUP_M) {
@@ -482,7 +540,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             tma_load_2d(a_dst, &tmA, &full[s], k0, ti_row_base(ti) + ti.m0);
             if constexpr (!B_MN) {
               const int brow = ti.e * p.b_rows_per_group;
-              if constexpr (EPI == EPI_SWIGLU_FWD) {
+              if constexpr (epi_swiglu_fwd(EPI)) {
                 tma_load_2d(b_dst, &tmB, &full[s], k0, brow + ti.n0);                       // gate
                 tma_load_2d(b_dst + (BN / 2) * 128, &tmB, &full[s], k0, brow + p.F + ti.n0);  // up
               } else {
@@ -557,6 +615,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
         const TileInfo ti = nxt;
         if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
         const int nst = num_kstages<C, MODE>(ti, p);
+        const uint32_t idesc = ti_half<PAIR, MODE>(ti, p) ? C::IDESC_HALF : C::IDESC;
         const int buf = local % C::NACC;
         const uint32_t use = (uint32_t)(local / C::NACC) & 1u;  // parity of this buffer's use
         const bool drained =
@@ -599,7 +658,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               umma_mx(d_tmem, ad, bd, id, sf_col | ((uint32_t)kk << 30),
                       (sf_col + 4) | ((uint32_t)kk << 30), (ks > 0 || kk > 0) ? 1u : 0u);
             } else if constexpr (PAIR) {
-              umma_pair<ES == 2 ? 0 : 1>(d_tmem, ad, bd, C::IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
+              umma_pair<ES == 2 ? 0 : 1>(d_tmem, ad, bd, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
             } else {
               umma<ES == 2 ? 0 : 1>(d_tmem, ad, bd, C::IDESC, (ks > 0 || kk > 0) ? 1u : 0u);
             }
@@ -649,24 +708,38 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       if (!ok) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-      const int m_cta = ti.m0 + (int)rank * BM;             // this CTA's first tile row
-      const bool active = (m_cta + q * 32) < ti_rows<MODE>(ti, p);       // warp-uniform
-      int c1;                                               // tensor row of this slab
-      if constexpr (MODE == GROUP_K) c1 = ti.e * (p.c_group_rows ? p.c_group_rows : p.M) + m_cta + q * 32;
-      else c1 = ti_row_base(ti) + m_cta + q * 32;
+      // Full tile: this warp's 32 rows are rows q*32.. of the CTA's 128, over all BN accumulator
+      // columns. Pair tail tile (M = 128): rows (q&1)*32.. of the CTA's 64, over the BN/2 accumulator
+      // columns of its lane half, which hold output columns (q>>1)*BN/2 + [0, BN/2) of the tile.
+      const bool half = ti_half<PAIR, MODE>(ti, p);
+      const int slab = half ? ti.m0 + (int)rank * C::HALF_M + (q & 1) * 32
+                            : ti.m0 + (int)rank * BM + q * 32;  // first tile row of this warp
+      const int whalf = half ? (q >> 1) : 0;                   // lane half (tail tiles)
+      const bool active = slab < ti_rows<MODE>(ti, p);         // warp-uniform
+      int c1;                                                  // tensor row of this slab
+      if constexpr (MODE == GROUP_K) c1 = ti.e * (p.c_group_rows ? p.c_group_rows : p.M) + slab;
+      else c1 = ti_row_base(ti) + slab;
       // Every variant walks the accumulator in 32-column chunks and keeps the TMEM load of the next
       // chunk in flight while it converts and stages the current one; CPB chunks fill one box.
       constexpr int CPB = C::OEPR / 32;
-      if constexpr (EPI == EPI_SWIGLU_FWD) {
-        // accumulator columns [0, BN/2) gate, [BN/2, BN) up for output columns n0 + [0, BN/2)
-        constexpr int NCH = BN / 2 / 32;
-        if (active) {
+      // quantising epilogues: the warp's 32 rows are one 32-row column block of the routed buffer
+      const int64_t qrb = (int64_t)c1 >> 5;
+      if constexpr (epi_swiglu_fwd(EPI)) {
+        // Full tile: accumulator columns [0, BN/2) gate, [BN/2, BN) up, for output columns
+        // n0 + [0, BN/2). Tail tile: [0, BN/4) gate, [BN/4, BN/2) up, for output columns
+        // n0 + whalf*BN/4 + [0, BN/4).
+        auto swiglu = [&](auto nch_c) {
+          constexpr int NCH = decltype(nch_c)::value;  // 32-column chunks of output
+          constexpr int UP = NCH * 32;                 // accumulator column of the first up value
+          const int col0 = ti.n0 + whalf * UP;         // first output column of this warp
           uint32_t ga[32], ua[32], gb[32], ub[32];
           tmem_ld_32x32b_x32(t_row, ga);
-          tmem_ld_32x32b_x32(t_row + BN / 2, ua);
+          tmem_ld_32x32b_x32(t_row + UP, ua);
           uint8_t* bg = wstg;
           uint8_t* bu = wstg + 4096;
-          uint8_t* ba = wstg + 8192;
+          uint8_t* ba = wstg + 8192;   // a (bf16), or a's row-block codes
+          uint8_t* bac = wstg + 12288;  // a's column-block codes (quantising)
+          uint32_t srow = 0;            // row-block scale bytes of four consecutive chunks
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
             uint32_t(&rg)[32] = (j & 1) ? gb : ga;
@@ -675,7 +748,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             tmem_regs_after(ru);
             if (j + 1 < NCH) {
               tmem_ld_32x32b_x32(t_row + (j + 1) * 32, (j & 1) ? ga : gb);
-              tmem_ld_32x32b_x32(t_row + BN / 2 + (j + 1) * 32, (j & 1) ? ua : ub);
+              tmem_ld_32x32b_x32(t_row + UP + (j + 1) * 32, (j & 1) ? ua : ub);
             }
             if (j % CPB == 0) {
               if (lane == 0) bulk_wait_read<0>();
@@ -694,24 +767,51 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               stage_row32<C::OES>(bg, lane, ch0, g);
               stage_row32<C::OES>(bu, lane, ch0, u);
             }
-            stage_row32<C::OES>(ba, lane, ch0, a);
-            if (j % CPB == CPB - 1) {
-              const int c = (j / CPB) * C::OEPR;
+            if constexpr (EPI == EPI_SWIGLU_FWD_Q) {
+              // a as stored in bf16, quantised along the row (the next GEMM's contraction) and down
+              // the warp's 32-row column block (the weight gradient's contraction)
+#pragma unroll
+              for (int i = 0; i < 32; ++i) a[i] = round_out<2>(a[i]);
+              uint32_t cr[8], cc[8];
+              srow |= (uint32_t)mx_row_block(a, cr) << (8 * (j & 3));
+              const uint8_t scol = mx_col_blocks(a, lane, cc);
+              stage_codes32(ba, lane, j & 3, cr);
+              stage_codes32(bac, lane, j & 3, cc);
+              p.q_sc[tiled_sf_offset(col0 + j * 32 + lane, qrb, p.q_kb_col)] = scol;
+            } else {
+              stage_row32<C::OES>(ba, lane, ch0, a);
+            }
+            if (j % CPB == CPB - 1 || j == NCH - 1) {
+              const int c = col0 + (j / CPB) * C::OEPR;
               if (p.C) {
-                box_store(&tmC, bg, lane, ti.n0 + c, c1);
-                box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
+                box_store(&tmC, bg, lane, c, c1);
+                box_store(&tmC, bu, lane, p.F + c, c1);
               }
-              box_store(&tmC2, ba, lane, ti.n0 + c, c1);
+              if constexpr (EPI == EPI_SWIGLU_FWD) box_store(&tmC2, ba, lane, c, c1);
+            }
+            if constexpr (EPI == EPI_SWIGLU_FWD_Q) {
+              if ((j & 3) == 3) {  // 128 columns of codes: one box each, and the row's 4 scale bytes
+                const int c = col0 + (j & ~3) * 32;
+                box_store(&tmX1, ba, lane, c, c1);
+                box_store(&tmX2, bac, lane, c, c1);
+                *reinterpret_cast<uint32_t*>(p.q_sr + tiled_sf_offset(c1 + lane, c >> 5, p.q_kb_row)) = srow;
+                srow = 0;
+              }
             }
           }
+        };
+        if (active) {
+          if (half) swiglu(std::integral_constant<int, BN / 4 / 32>{});
+          else swiglu(std::integral_constant<int, BN / 2 / 32>{});
         }
-      } else if constexpr (EPI == EPI_SWIGLU_BWD) {
+      } else if constexpr (epi_swiglu_bwd(EPI)) {
         // dA chunk from TMEM; gate and up of the saved h13 for the same 32 columns from global
-        // memory, both fetched one chunk ahead
+        // memory, both fetched one chunk ahead. Quantising: dh13 leaves as row-block and column-block
+        // codes of its bf16 value (boxes: row codes gate / up, column codes gate / up).
         constexpr int NCH = BN / 32;
         constexpr int RW = 2 * C::OES;  // 16-byte words per 32 stored values
         const char* hrow = reinterpret_cast<const char*>(p.aux) +
-                           ((size_t)ti_row_base(ti) + m_cta + q * 32 + lane) * p.ldaux * C::OES;
+                           ((size_t)ti_row_base(ti) + slab + lane) * p.ldaux * C::OES;
         if (active) {
           uint32_t da[32], db[32];
           uint4 gwa[RW], uwa[RW], gwb[RW], uwb[RW];
@@ -722,6 +822,9 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           }
           uint8_t* bg = wstg;
           uint8_t* bu = wstg + 4096;
+          uint8_t* bgc = wstg + 8192;   // quantising: column-block codes of the gate half
+          uint8_t* buc = wstg + 12288;  // and of the up half
+          uint32_t srg = 0, sru = 0;    // row-block scale bytes of four consecutive chunks
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
             uint32_t(&rd)[32] = (j & 1) ? db : da;
@@ -738,7 +841,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               }
             }
             if (cols) {
-              if (j % CPB == 0) {
+              if (j % (EPI == EPI_SWIGLU_BWD_Q ? 4 : CPB) == 0) {
                 if (lane == 0) bulk_wait_read<0>();
                 __syncwarp();
               }
@@ -753,30 +856,61 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
                 g[i] = dav * u[i] * sg * (1.f + gi * (1.f - sg));  // d gate
                 u[i] = dav * gi * sg;                              // d up
               }
-              const int ch0 = ((j % CPB) * 32 * C::OES) >> 4;
-              stage_row32<C::OES>(bg, lane, ch0, g);
-              stage_row32<C::OES>(bu, lane, ch0, u);
-              if (j % CPB == CPB - 1) {
-                const int c = (j / CPB) * C::OEPR;
-                box_store(&tmC, bg, lane, ti.n0 + c, c1);
-                box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
+              if constexpr (EPI == EPI_SWIGLU_BWD_Q) {
+                uint32_t cr[8], cc[8];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  g[i] = round_out<2>(g[i]);
+                  u[i] = round_out<2>(u[i]);
+                }
+                srg |= (uint32_t)mx_row_block(g, cr) << (8 * (j & 3));
+                uint8_t sc = mx_col_blocks(g, lane, cc);
+                stage_codes32(bg, lane, j & 3, cr);
+                stage_codes32(bgc, lane, j & 3, cc);
+                p.q_sc[tiled_sf_offset(col + lane, qrb, p.q_kb_col)] = sc;
+                sru |= (uint32_t)mx_row_block(u, cr) << (8 * (j & 3));
+                sc = mx_col_blocks(u, lane, cc);
+                stage_codes32(bu, lane, j & 3, cr);
+                stage_codes32(buc, lane, j & 3, cc);
+                p.q_sc[tiled_sf_offset(p.F + col + lane, qrb, p.q_kb_col)] = sc;
+                if ((j & 3) == 3) {
+                  const int c = ti.n0 + (j & ~3) * 32;
+                  box_store(&tmX1, bg, lane, c, c1);
+                  box_store(&tmX1, bu, lane, p.F + c, c1);
+                  box_store(&tmX2, bgc, lane, c, c1);
+                  box_store(&tmX2, buc, lane, p.F + c, c1);
+                  *reinterpret_cast<uint32_t*>(p.q_sr + tiled_sf_offset(c1 + lane, c >> 5, p.q_kb_row)) = srg;
+                  *reinterpret_cast<uint32_t*>(p.q_sr + tiled_sf_offset(c1 + lane, (p.F + c) >> 5, p.q_kb_row)) = sru;
+                  srg = sru = 0;
+                }
+              } else {
+                const int ch0 = ((j % CPB) * 32 * C::OES) >> 4;
+                stage_row32<C::OES>(bg, lane, ch0, g);
+                stage_row32<C::OES>(bu, lane, ch0, u);
+                if (j % CPB == CPB - 1) {
+                  const int c = (j / CPB) * C::OEPR;
+                  box_store(&tmC, bg, lane, ti.n0 + c, c1);
+                  box_store(&tmC, bu, lane, p.F + ti.n0 + c, c1);
+                }
               }
             }
           }
         }
       } else {
         // plain store (act dtype), fp32 + bias (router scores), or a weight gradient (GROUP_K; an
-        // expert without rows has nst == 0 and gets zeros)
-        constexpr int NCH = BN / 32;
-        if (active) {
+        // expert without rows has nst == 0 and gets zeros). Tail tiles of a pair: BN/2 columns per
+        // warp, output columns n0 + whalf*BN/2 + [0, BN/2).
+        auto store = [&](auto nch_c) {
+          constexpr int NCH = decltype(nch_c)::value;
+          const int col0 = ti.n0 + whalf * (NCH * 32);
           const bool acc = nst > 0;
           uint32_t ra[32], rb[32];
           if (acc) tmem_ld_32x32b_x32(t_row, ra);
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
             uint32_t(&rc)[32] = (j & 1) ? rb : ra;
-            const int c = (j / CPB) * C::OEPR;  // first column of this chunk's box
-            const bool cols = ti.n0 + c < p.N;
+            const int c = col0 + (j / CPB) * C::OEPR;  // first column of this chunk's box
+            const bool cols = c < p.N;
             if (acc) {
               tmem_ld_wait_regs(rc);
               if (j + 1 < NCH) tmem_ld_32x32b_x32(t_row + (j + 1) * 32, (j & 1) ? ra : rb);
@@ -793,19 +927,23 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               if (p.bias) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                  const int col = ti.n0 + j * 32 + i;
+                  const int col = col0 + j * 32 + i;
                   if (col < p.N) v[i] += p.bias[col];
                 }
               }
             }
             if (cols) {
               stage_row32<C::OES>(bx, lane, ((j % CPB) * 32 * C::OES) >> 4, v);
-              if (j % CPB == CPB - 1) {
-                box_store(&tmC, bx, lane, ti.n0 + c, c1);
+              if (j % CPB == CPB - 1 || j == NCH - 1) {
+                box_store(&tmC, bx, lane, c, c1);
                 nb = (nb + 1) % C::NBUF;
               }
             }
           }
+        };
+        if (active) {
+          if (half) store(std::integral_constant<int, BN / 2 / 32>{});
+          else store(std::integral_constant<int, BN / 32>{});
         }
       }
       tc_fence_before();
@@ -946,7 +1084,7 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
     if (!make_tmap_mn(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::BK, C::BN_CTA / C::EPR, mn_sw))
       return MOE_ERR_CUDA;
   } else {
-    const int b_box_rows = B_MN ? 32 : ((PAIR || EPI != EPI_SWIGLU_FWD) ? C::BN_CTA : BN / 2);
+    const int b_box_rows = B_MN ? 32 : ((PAIR || !epi_swiglu_fwd(EPI)) ? C::BN_CTA : BN / 2);
     if (!make_tmap(&tb, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, b_box_rows, B_MN ? mn_sw : 2))
       return MOE_ERR_CUDA;
   }
@@ -954,17 +1092,41 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   CUtensorMap tc, tc2;
   const int64_t out_rows =
       (MODE == GROUP_K) ? (int64_t)k_groups(p) * (p.c_group_rows ? p.c_group_rows : p.M) : A.rows;
-  const int64_t out_cols = (EPI == EPI_SWIGLU_FWD || EPI == EPI_SWIGLU_BWD) ? 2 * (int64_t)p.F : p.N;
+  const int64_t out_cols = (epi_swiglu_fwd(EPI) || epi_swiglu_bwd(EPI)) ? 2 * (int64_t)p.F : p.N;
   if (EPI == EPI_SWIGLU_FWD && !make_tmap(&tc2, p.C2, C::OES, out_rows, p.F, p.ldc2, C::OEPR, 32, 2))
     return MOE_ERR_CUDA;
+  // quantising epilogues: code outputs [rows, F] (a) or [rows, 2F] (dh13), 32-row x 128-byte boxes
+  CUtensorMap tq1, tq2;
+  if (epi_quant(EPI)) {
+    const int64_t qcols = EPI == EPI_SWIGLU_FWD_Q ? p.F : 2 * (int64_t)p.F;
+    if (!p.q_qr || !p.q_qc || !p.q_sr || !p.q_sc) return MOE_ERR_INVALID_ARG;
+    if (!make_tmap(&tq1, p.q_qr, 1, out_rows, qcols, qcols, 128, 32, 2) ||
+        !make_tmap(&tq2, p.q_qc, 1, out_rows, qcols, qcols, 128, 32, 2))
+      return MOE_ERR_CUDA;
+  }
   if (p.C) {
     if (!make_tmap(&tc, p.C, C::OES, out_rows, out_cols, p.ldc, C::OEPR, 32, 2)) return MOE_ERR_CUDA;
+  } else if (EPI == EPI_SWIGLU_BWD_Q) {
+    tc = tq1;  // dh13 leaves as codes only: tc is never used
   } else if (EPI == EPI_SWIGLU_FWD) {
     tc = tc2;  // SwiGLU forward without h13: only a is stored, tc is never used
   } else {
     return MOE_ERR_INVALID_ARG;
   }
   if (EPI != EPI_SWIGLU_FWD) tc2 = tc;
+  // pair tail tiles (M = 128 over the pair): 64-row boxes of A, and of B for the SwiGLU forward,
+  // whose tail tile loads 64 gate + 64 up rows per CTA
+  CUtensorMap ta64 = ta, tb64 = tb;
+  if (epi_quant(EPI)) {
+    ta64 = tq1;
+    tb64 = tq2;
+  }
+  if (PAIR && MODE == GROUP_M) {
+    if (!make_tmap(&ta64, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, C::HALF_M, 2)) return MOE_ERR_CUDA;
+    if (EPI == EPI_SWIGLU_FWD &&
+        !make_tmap(&tb64, B.ptr, ES, B.rows, B.cols, B.ld, C::EPR, BN / 4, 2))
+      return MOE_ERR_CUDA;
+  }
   // persistent grid: one CTA (pair) per SM (pair of SMs), capped by the tile count where the host
   // knows it (GROUP_K: fixed tiles per group)
   int64_t cap = 0;
@@ -996,11 +1158,11 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
     if (cap > 0 && cap < pairs) pairs = cap;
     cfg.gridDim = dim3((unsigned)(2 * pairs));
     cfg.numAttrs = 2;  // cluster shape + programmatic dependent launch
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tc2, q) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tc2, ta64, tb64, q) != cudaSuccess) return MOE_ERR_CUDA;
   } else {
     int64_t grid = sm_count();
     if (cap > 0 && cap < grid) grid = cap;
-    MOE_LAUNCH(launch_pdl(kern, (unsigned)grid, C::THREADS, C::SMEM_BYTES, s, ta, tb, tc, tc2, q));
+    MOE_LAUNCH(launch_pdl(kern, (unsigned)grid, C::THREADS, C::SMEM_BYTES, s, ta, tb, tc, tc2, ta64, tb64, q));
   }
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
@@ -1037,6 +1199,9 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
       if (bn == 256)                                                                               \
         return launch_impl<ES_, false, false, 256, EPI_STORE_F32_BIAS, GROUP_M, false>(A, B, p, s); \
       return launch_impl<ES_, false, false, 128, EPI_STORE_F32_BIAS, GROUP_M, false>(A, B, p, s);  \
+    case GK_FWD1_SWIGLU_Q:                                                                         \
+    case GK_DGRAD2_SWIGLU_Q:                                                                       \
+      return MOE_ERR_UNSUPPORTED; /* quantising epilogues: MXFP8 only */                           \
     case GK_WGRAD_SPLIT:  /* fp32 partial products, no bias */                                     \
       if (bn == 256)                                                                               \
         return launch_impl<ES_, true, true, 256, EPI_STORE_F32_BIAS, GROUP_K, false>(A, B, p, s);  \
@@ -1055,6 +1220,8 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
     const bool wide = p.N % 256 == 0;
     switch (kind) {
       case GK_FWD1_SWIGLU: return launch_impl<1, false, false, 256, EPI_SWIGLU_FWD, GROUP_M, false>(A, B, p, s);
+      case GK_FWD1_SWIGLU_Q: return launch_impl<1, false, false, 256, EPI_SWIGLU_FWD_Q, GROUP_M, false>(A, B, p, s);
+      case GK_DGRAD2_SWIGLU_Q: return launch_impl<1, false, true, 128, EPI_SWIGLU_BWD_Q, GROUP_M, false>(A, B, p, s);
       case GK_FWD2:
         if (wide) return launch_impl<1, false, false, 256, EPI_STORE, GROUP_M, false>(A, B, p, s);
         return launch_impl<1, false, false, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);

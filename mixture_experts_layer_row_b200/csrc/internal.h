@@ -6,12 +6,33 @@
 namespace moe {
 
 // Grouped GEMM epilogues and grouping modes.
-enum { EPI_STORE = 0, EPI_SWIGLU_FWD = 1, EPI_SWIGLU_BWD = 2, EPI_STORE_F32_BIAS = 3 };
+// EPI_SWIGLU_FWD_Q / EPI_SWIGLU_BWD_Q (MXFP8 only): as the SwiGLU epilogues, but the activation they
+// produce (a, or dh13) leaves as E4M3 codes quantised along rows and along 32-row column blocks, with
+// tiled scales, instead of a bf16 copy (the forward still stores h13 in bf16).
+enum {
+  EPI_STORE = 0,
+  EPI_SWIGLU_FWD = 1,
+  EPI_SWIGLU_BWD = 2,
+  EPI_STORE_F32_BIAS = 3,
+  EPI_SWIGLU_FWD_Q = 4,
+  EPI_SWIGLU_BWD_Q = 5
+};
 enum { GROUP_M = 0, GROUP_K = 1 };
 
 // GK_WGRAD_SPLIT: single-group wgrad with the contraction split into chunks of ksplit rows, one fp32
 // partial product per chunk (summed afterwards by launch_split_reduce).
-enum GemmKind { GK_FWD1_SWIGLU, GK_FWD2, GK_DGRAD2_SWIGLU, GK_DGRAD1, GK_WGRAD, GK_ROUTER, GK_WGRAD_SPLIT };
+// GK_FWD1_SWIGLU_Q / GK_DGRAD2_SWIGLU_Q (MXFP8): the SwiGLU GEMMs with the quantising epilogues.
+enum GemmKind {
+  GK_FWD1_SWIGLU,
+  GK_FWD2,
+  GK_DGRAD2_SWIGLU,
+  GK_DGRAD1,
+  GK_WGRAD,
+  GK_ROUTER,
+  GK_WGRAD_SPLIT,
+  GK_FWD1_SWIGLU_Q,
+  GK_DGRAD2_SWIGLU_Q
+};
 
 // A row-major 2-D operand as the TMA unit sees it.
 struct GemmOperand {
@@ -50,6 +71,13 @@ struct GemmParams {
   // box when M is not a multiple of 32, so a box never reaches into the next split's rows.
   int ksplit;
   int c_group_rows;
+  // quantising epilogues: tiled scales of the row-block codes (K-blocks per row: q_kb_row) and of the
+  // column-block codes (K-blocks per column: q_kb_col); the codes go out through tensor maps
+  uint8_t* q_qr;  // row-block codes [A rows, output columns]
+  uint8_t* q_qc;  // column-block codes, same layout
+  uint8_t* q_sr;
+  uint8_t* q_sc;
+  int64_t q_kb_row, q_kb_col;
 };
 
 // Host-side count of kernels enqueued (every launcher adds the kernels it launched).
@@ -95,6 +123,15 @@ int launch_quantize(const void* src, int64_t rows, int cols, int mode, int64_t G
                     uint8_t* s, cudaStream_t st);
 int launch_quantize_rowcol(const void* src, int64_t rows, int cols, uint8_t* qr, uint8_t* sr,
                            uint8_t* qc, uint8_t* sc, cudaStream_t st);
+// MXFP8 layer: row- and column-block quantisation of a routed-row operand built from token-order rows
+// (rows with row_token < 0 are zero; 32-row blocks at or past *poff_end are skipped).
+int launch_dispatch_quant(const void* x, const int32_t* row_token, const int32_t* poff_end, int k,
+                          int64_t rows, int cols, uint8_t* qr, uint8_t* sr, uint8_t* qc, uint8_t* sc,
+                          cudaStream_t st);
+int launch_combine_bwd_quant(const void* dout, const void* y, const float* gates,
+                             const int32_t* row_token, const int32_t* poff_end, int k, int64_t rows,
+                             int cols, float* dgates, uint8_t* qr, uint8_t* sr, uint8_t* qc,
+                             uint8_t* sc, cudaStream_t st);
 int launch_bounded_wait_probe(uint32_t* err, uint64_t limit_ns, cudaStream_t s);
 // out[i] = round_to_act(sum over s < nsplit of part[s*stride + i]) for i < n (fixed summation order).
 int launch_split_reduce(const float* part, int nsplit, int64_t n, int64_t stride, void* out, bool bf16,
@@ -109,16 +146,21 @@ int launch_metadata(const int32_t* idx, int T, int E, int k, int align, int64_t 
                     int32_t* counts, int32_t* offsets, int32_t* poff, int32_t* perm, int32_t* prow,
                     int32_t* row_token, int32_t* hist_ws, uint32_t* err, cudaStream_t s);
 
+// Row kernels: every padded row outside [0, max_rows) (such as the -1 the metadata writes for an
+// invalid expert id) is skipped.
 int launch_dispatch(const void* x, const int32_t* prow, const int32_t* counts, const int32_t* poff,
-                    void* xp, int T, int k, int E, int row_bytes, cudaStream_t s);
+                    void* xp, int T, int k, int E, int row_bytes, int64_t max_rows, cudaStream_t s);
 int launch_combine(const void* y, const float* gates, const int32_t* prow, void* out, int T, int k,
-                   int row_bytes, bool bf16, cudaStream_t s);
+                   int row_bytes, bool bf16, int64_t max_rows, cudaStream_t s);
 int launch_combine_bwd(const void* dout, const void* y, const float* gates, const int32_t* prow,
                        const int32_t* idx, const int32_t* counts, const int32_t* poff, void* dy,
                        float* dgates, float* dlsel, void* dlogits, int T, int k, int E, int row_bytes,
-                       bool bf16, cudaStream_t s);
+                       bool bf16, int64_t max_rows, cudaStream_t s);
+// dlsel[t,j] = g_j (dg_j - sum_i g_i dg_i) and the dense score gradient dlogits [T,E] (act dtype).
+int launch_score_grad(const float* gates, const float* dgates, const int32_t* idx, float* dlsel,
+                      void* dlogits, int T, int k, int E, bool bf16, cudaStream_t s);
 int launch_token_reduce(const void* dxp, const int32_t* prow, const float* dlsel, const int32_t* idx,
                         const void* Wr, void* dx, int T, int k, int E, int row_bytes, bool bf16,
-                        cudaStream_t s);
+                        int64_t max_rows, cudaStream_t s);
 
 }  // namespace moe

@@ -24,21 +24,57 @@ static __device__ __align__(256) int32_t g_route_scratch[kNoAllocScratchInts];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
-int32_t* g_scratch_ptr[kMaxDevices] = {nullptr};
+struct ScratchSlot {
+  int32_t* ptr;
+  unsigned long long ctx_id;  // the context the address belongs to
+};
+ScratchSlot g_scratch[kMaxDevices] = {};
+
+// Unique id of the calling thread's current CUDA context (driver API through the runtime's entry
+// point lookup, so the library links no extra library). False if there is none or the lookup fails.
+bool current_context_id(unsigned long long* id) {
+  typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+  typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess)
+      return false;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    get_id = reinterpret_cast<CtxGetIdFn>(b);
+  }
+  CUcontext c = nullptr;
+  if (get_current(&c) != CUDA_SUCCESS || !c) return false;
+  return get_id(c, id) == CUDA_SUCCESS;
+}
 
 // Device address of the scratch array on the current device. In host code the array's name is only
-// a host-side stand-in, so the address is looked up once per device, with that device current.
+// a host-side stand-in, so the address is looked up with the device current: once per device, and
+// again whenever the device's context has been replaced (after cudaDeviceReset the module is loaded
+// anew and the array may sit at another address).
 int scratch_for_current_device(int32_t** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (!g_scratch_ptr[dev]) {
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
+  ScratchSlot& slot = g_scratch[dev];
+  if (!slot.ptr || !have_ctx || slot.ctx_id != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
-    g_scratch_ptr[dev] = static_cast<int32_t*>(p);
+    // the lookup above makes the primary context current if none was
+    if (!current_context_id(&ctx)) ctx = 0;
+    slot.ptr = static_cast<int32_t*>(p);
+    slot.ctx_id = ctx;
   }
-  *out = g_scratch_ptr[dev];
+  *out = slot.ptr;
   return MOE_OK;
 }
 
@@ -58,7 +94,7 @@ extern "C" MOE_API int moe_route_metadata_noalloc(const moe_config_t* cfg, const
   const int rc = moe::scratch_for_current_device(&hist);
   if (rc != MOE_OK) return rc;
   // Device-side routing errors are not reported by this variant (there is no workspace flag);
-  // invalid expert ids are still skipped by the kernels.
+  // entries with an expert id outside [0,E) still get perm = prow = -1 and no row.
   return moe::launch_metadata(idx, cfg->T, cfg->E, cfg->k, moe::group_align(cfg->dtype),
                               moe_max_rows(cfg), counts, offsets, poff, perm, prow, row_token, hist,
                               nullptr, reinterpret_cast<cudaStream_t>(stream));

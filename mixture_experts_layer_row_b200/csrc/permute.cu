@@ -7,7 +7,9 @@
 //   combine_bwd   dy[prow[t,j]] = g[t,j] dout[t];  dg[t,j] = <dout[t], y[prow[t,j]]> (+ score grads)
 //   token_reduce  dx[t] = sum_j dx_perm[prow[t,j]] (+ sum_j dl[t,j] W_r[idx[t,j]])
 // Every routed-row pad row (the tail of each expert's 32-aligned group) is written as zero by
-// dispatch and combine_bwd so the grouped GEMMs can run whole 32-row blocks.
+// dispatch and combine_bwd so the grouped GEMMs can run whole 32-row blocks. An entry whose padded row
+// lies outside [0, max_rows) -- the -1 that the metadata writes for an expert id outside [0,E) -- is
+// skipped by every kernel here: nothing is read or written through it.
 #include "internal.h"
 
 namespace moe {
@@ -50,6 +52,13 @@ struct Vec<false> {
   }
 };
 
+// Padded row of slot `lane` of token t, or -1 when the slot is unused or its row is out of range.
+__device__ __forceinline__ int slot_row(const int32_t* prow, int t, int k, int lane, int max_rows) {
+  if (lane >= k) return -1;
+  const int r = prow[(size_t)t * k + lane];
+  return (r >= 0 && r < max_rows) ? r : -1;
+}
+
 __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -69,7 +78,8 @@ __device__ __forceinline__ void zero_pad_rows(uint4* buf, int e, const int32_t* 
 
 __global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ prow, const int32_t* __restrict__ counts,
-    const int32_t* __restrict__ poff, uint4* __restrict__ xp, int T, int k, int vpr, int tok_blocks) {
+    const int32_t* __restrict__ poff, uint4* __restrict__ xp, int T, int k, int vpr, int tok_blocks,
+    int max_rows) {
   pdl_enter();  // wait for the previous kernel before any global access
   if ((int)blockIdx.x >= tok_blocks) {
     zero_pad_rows(xp, blockIdx.x - tok_blocks, counts, poff, vpr);
@@ -78,7 +88,7 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (t >= T) return;
-  const int myrow = lane < k ? prow[(size_t)t * k + lane] : 0;
+  const int myrow = slot_row(prow, t, k, lane, max_rows);
   int rows[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xffffffffu, myrow, j);
@@ -88,7 +98,7 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(
     const uint4 val = ldg_stream(src + v);
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (j < k) xp[(size_t)rows[j] * vpr + v] = val;
+      if (j < k && rows[j] >= 0) xp[(size_t)rows[j] * vpr + v] = val;
   }
 }
 
@@ -97,13 +107,13 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const uint4* __res
                                                               const float* __restrict__ gates,
                                                               const int32_t* __restrict__ prow,
                                                               uint4* __restrict__ out, int T, int k,
-                                                              int vpr) {
+                                                              int vpr, int max_rows) {
   pdl_enter();  // wait for the previous kernel before any global access
   using V = Vec<BF16>;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (t >= T) return;
-  const int myrow = lane < k ? prow[(size_t)t * k + lane] : 0;
+  const int myrow = slot_row(prow, t, k, lane, max_rows);
   const float myg = lane < k ? gates[(size_t)t * k + lane] : 0.f;
   int rows[8];
   float g[8];
@@ -119,7 +129,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const uint4* __res
     for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (j < k) {
+      if (j < k && rows[j] >= 0) {
         float f[V::N];
         V::unpack(ldg_stream(y + (size_t)rows[j] * vpr + v), f);
 #pragma unroll
@@ -137,7 +147,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) combine_bwd_kernel(
     const int32_t* __restrict__ prow, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ counts, const int32_t* __restrict__ poff, uint4* __restrict__ dy,
     float* __restrict__ dgates, float* __restrict__ dlsel, void* __restrict__ dlogits, int T, int k,
-    int E, int vpr, int tok_blocks) {
+    int E, int vpr, int tok_blocks, int max_rows) {
   pdl_enter();  // wait for the previous kernel before any global access
   using V = Vec<BF16>;
   if ((int)blockIdx.x >= tok_blocks) {
@@ -147,7 +157,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) combine_bwd_kernel(
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (t >= T) return;
-  const int myrow = lane < k ? prow[(size_t)t * k + lane] : 0;
+  const int myrow = slot_row(prow, t, k, lane, max_rows);
   const float myg = lane < k ? gates[(size_t)t * k + lane] : 0.f;
   int rows[8];
   float g[8], dot[8];
@@ -163,7 +173,7 @@ __global__ void __launch_bounds__(kWarps * 32, 4) combine_bwd_kernel(
     V::unpack(ldg_stream(dout + (size_t)t * vpr + v), fd);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (j < k) {
+      if (j < k && rows[j] >= 0) {
         float fy[V::N], o[V::N];
         V::unpack(ldg_stream(y + (size_t)rows[j] * vpr + v), fy);
 #pragma unroll
@@ -221,14 +231,14 @@ template <bool BF16>
 __global__ void __launch_bounds__(kWarps * 32) token_reduce_kernel(
     const uint4* __restrict__ dxp, const int32_t* __restrict__ prow, const float* __restrict__ dlsel,
     const int32_t* __restrict__ idx, const uint4* __restrict__ Wr, uint4* __restrict__ dx, int T,
-    int k, int E, int vpr) {
+    int k, int E, int vpr, int max_rows) {
   pdl_enter();  // wait for the previous kernel before any global access
   using V = Vec<BF16>;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (t >= T) return;
   const bool router = dlsel && idx && Wr;
-  const int myrow = lane < k ? prow[(size_t)t * k + lane] : 0;
+  const int myrow = slot_row(prow, t, k, lane, max_rows);
   const float mydl = (router && lane < k) ? dlsel[(size_t)t * k + lane] : 0.f;
   int mye = (router && lane < k) ? idx[(size_t)t * k + lane] : 0;
   if (mye < 0 || mye >= E) mye = 0;
@@ -247,7 +257,7 @@ __global__ void __launch_bounds__(kWarps * 32) token_reduce_kernel(
     for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (j < k) {
+      if (j < k && rows[j] >= 0) {
         float f[V::N];
         V::unpack(ldg_stream(dxp + (size_t)rows[j] * vpr + v), f);
 #pragma unroll
@@ -263,29 +273,76 @@ __global__ void __launch_bounds__(kWarps * 32) token_reduce_kernel(
   }
 }
 
+// Score gradients of a learned router with renormalised gates, from the gate gradients: per token,
+// dl_j = g_j (dg_j - sum_i g_i dg_i) for its k slots, and the dense row dlogits[t, e] (act dtype) that
+// is zero except at the chosen experts. One warp per token. (combine_bwd_kernel computes the same on
+// the way; the MXFP8 layer's fused combine backward leaves it to this kernel.)
+template <bool BF16>
+__global__ void __launch_bounds__(kWarps * 32) score_grad_kernel(const float* __restrict__ gates,
+                                                                 const float* __restrict__ dgates,
+                                                                 const int32_t* __restrict__ idx,
+                                                                 float* __restrict__ dlsel,
+                                                                 void* __restrict__ dlogits, int T,
+                                                                 int k, int E) {
+  pdl_enter();  // wait for the previous kernel before any global access
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float g = lane < k ? gates[(size_t)t * k + lane] : 0.f;
+  const float dg = lane < k ? dgates[(size_t)t * k + lane] : 0.f;
+  float s = g * dg;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  const float mydl = g * (dg - s);
+  const int mye = lane < k ? idx[(size_t)t * k + lane] : -1;
+  if (lane < k) dlsel[(size_t)t * k + lane] = mydl;
+  int ej[8];
+  float dj[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    ej[j] = __shfl_sync(0xffffffffu, mye, j);
+    dj[j] = __shfl_sync(0xffffffffu, mydl, j);
+  }
+  for (int e = lane; e < E; e += 32) {
+    float val = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < k && ej[j] == e) val = dj[j];
+    if (BF16)
+      reinterpret_cast<__nv_bfloat16*>(dlogits)[(size_t)t * E + e] = __float2bfloat16_rn(val);
+    else
+      reinterpret_cast<float*>(dlogits)[(size_t)t * E + e] = val;
+  }
+}
+
+// Row bound passed to the kernels (row indices are int32).
+inline int clamp_rows(int64_t max_rows) { return max_rows > INT32_MAX ? INT32_MAX : (int)max_rows; }
+
 }  // namespace
 
 int launch_dispatch(const void* x, const int32_t* prow, const int32_t* counts, const int32_t* poff,
-                    void* xp, int T, int k, int E, int row_bytes, cudaStream_t s) {
+                    void* xp, int T, int k, int E, int row_bytes, int64_t max_rows, cudaStream_t s) {
   const int vpr = row_bytes / 16;
+  const int mr = clamp_rows(max_rows);
   const int tok_blocks = (T + kWarps - 1) / kWarps;
   MOE_LAUNCH(launch_pdl(dispatch_kernel, tok_blocks + E, kWarps * 32, 0, s, 
       static_cast<const uint4*>(x), prow, counts, poff, static_cast<uint4*>(xp), T, k, vpr,
-      tok_blocks));
+      tok_blocks, mr));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_combine(const void* y, const float* gates, const int32_t* prow, void* out, int T, int k,
-                   int row_bytes, bool bf16, cudaStream_t s) {
+                   int row_bytes, bool bf16, int64_t max_rows, cudaStream_t s) {
   const int vpr = row_bytes / 16;
+  const int mr = clamp_rows(max_rows);
   const int blocks = (T + kWarps - 1) / kWarps;
   if (bf16)
     MOE_LAUNCH(launch_pdl(combine_kernel<true>, blocks, kWarps * 32, 0, s, static_cast<const uint4*>(y), gates, prow,
-                                                        static_cast<uint4*>(out), T, k, vpr));
+                                                        static_cast<uint4*>(out), T, k, vpr, mr));
   else
     MOE_LAUNCH(launch_pdl(combine_kernel<false>, blocks, kWarps * 32, 0, s, static_cast<const uint4*>(y), gates, prow,
-                                                         static_cast<uint4*>(out), T, k, vpr));
+                                                         static_cast<uint4*>(out), T, k, vpr, mr));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -293,34 +350,49 @@ int launch_combine(const void* y, const float* gates, const int32_t* prow, void*
 int launch_combine_bwd(const void* dout, const void* y, const float* gates, const int32_t* prow,
                        const int32_t* idx, const int32_t* counts, const int32_t* poff, void* dy,
                        float* dgates, float* dlsel, void* dlogits, int T, int k, int E, int row_bytes,
-                       bool bf16, cudaStream_t s) {
+                       bool bf16, int64_t max_rows, cudaStream_t s) {
   const int vpr = row_bytes / 16;
+  const int mr = clamp_rows(max_rows);
   const int tok_blocks = (T + kWarps - 1) / kWarps;
   if (bf16)
     MOE_LAUNCH(launch_pdl(combine_bwd_kernel<true>, tok_blocks + E, kWarps * 32, 0, s, 
         static_cast<const uint4*>(dout), static_cast<const uint4*>(y), gates, prow, idx, counts,
-        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks));
+        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks, mr));
   else
     MOE_LAUNCH(launch_pdl(combine_bwd_kernel<false>, tok_blocks + E, kWarps * 32, 0, s, 
         static_cast<const uint4*>(dout), static_cast<const uint4*>(y), gates, prow, idx, counts,
-        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks));
+        poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tok_blocks, mr));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 int launch_token_reduce(const void* dxp, const int32_t* prow, const float* dlsel, const int32_t* idx,
                         const void* Wr, void* dx, int T, int k, int E, int row_bytes, bool bf16,
-                        cudaStream_t s) {
+                        int64_t max_rows, cudaStream_t s) {
   const int vpr = row_bytes / 16;
+  const int mr = clamp_rows(max_rows);
   const int blocks = (T + kWarps - 1) / kWarps;
   if (bf16)
     MOE_LAUNCH(launch_pdl(token_reduce_kernel<true>, blocks, kWarps * 32, 0, s, 
         static_cast<const uint4*>(dxp), prow, dlsel, idx, static_cast<const uint4*>(Wr),
-        static_cast<uint4*>(dx), T, k, E, vpr));
+        static_cast<uint4*>(dx), T, k, E, vpr, mr));
   else
     MOE_LAUNCH(launch_pdl(token_reduce_kernel<false>, blocks, kWarps * 32, 0, s, 
         static_cast<const uint4*>(dxp), prow, dlsel, idx, static_cast<const uint4*>(Wr),
-        static_cast<uint4*>(dx), T, k, E, vpr));
+        static_cast<uint4*>(dx), T, k, E, vpr, mr));
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int launch_score_grad(const float* gates, const float* dgates, const int32_t* idx, float* dlsel,
+                      void* dlogits, int T, int k, int E, bool bf16, cudaStream_t s) {
+  const int blocks = (T + kWarps - 1) / kWarps;
+  if (bf16)
+    MOE_LAUNCH(launch_pdl(score_grad_kernel<true>, blocks, kWarps * 32, 0, s, gates, dgates, idx, dlsel,
+                          dlogits, T, k, E));
+  else
+    MOE_LAUNCH(launch_pdl(score_grad_kernel<false>, blocks, kWarps * 32, 0, s, gates, dgates, idx, dlsel,
+                          dlogits, T, k, E));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

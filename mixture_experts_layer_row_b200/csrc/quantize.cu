@@ -24,50 +24,6 @@
 namespace moe {
 namespace {
 
-// floor(log2(a)) for a finite a > 0 given as fp32 bits.
-__device__ __forceinline__ int floor_log2_bits(uint32_t bits) {
-  const int ex = (int)((bits >> 23) & 0xFFu);
-  if (ex != 0) return ex - 127;
-  const uint32_t man = bits & 0x7FFFFFu;  // subnormal: man * 2^-149
-  return -149 + (31 - __clz(man));
-}
-
-// 2^k as an fp32 value for k in [-127, 127] (2^-127 is subnormal, still exact).
-__device__ __forceinline__ float exp2_exact(int k) {
-  return k >= -126 ? __int_as_float((k + 127) << 23) : __int_as_float(1 << (k + 149));
-}
-
-// Block exponent and scale byte for a block with maximum magnitude amax (>= 0).
-__device__ __forceinline__ int block_exponent(float amax, uint8_t* scale_byte) {
-  if (!(amax > 0.f)) {
-    *scale_byte = 0;
-    return 127;  // unused: all codes are zero
-  }
-  int e = floor_log2_bits(__float_as_uint(amax)) - 8;
-  e = e < -127 ? -127 : (e > 127 ? 127 : e);
-  *scale_byte = (uint8_t)(e + 127);
-  return e;
-}
-
-// Two floats -> two E4M3 codes (round to nearest even, saturate to finite), packed lo | hi << 8.
-__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// Byte mask over four packed column codes that clears the codes of all-zero column blocks (whose
-// values, +0 or -0, would otherwise convert to +0 or -0 codes; an all-zero block has zero codes).
-__device__ __forceinline__ uint32_t zero_block_mask(const float (&amax)[4]) {
-  return (amax[0] > 0.f ? 0x000000FFu : 0u) | (amax[1] > 0.f ? 0x0000FF00u : 0u) |
-         (amax[2] > 0.f ? 0x00FF0000u : 0u) | (amax[3] > 0.f ? 0xFF000000u : 0u);
-}
-
-// Byte offset of the scale of (MN index i, K-block b) in the tiled layout with KB K-blocks per MN index.
-__device__ __forceinline__ int64_t tiled_sf_offset(int64_t i, int64_t b, int64_t KB) {
-  return ((i >> 7) * (KB >> 2) + (b >> 2)) * 512 + (i & 31) * 16 + ((i >> 5) & 3) * 4 + (b & 3);
-}
-
 __device__ __forceinline__ int64_t scale_index(int layout, int64_t i, int64_t b, int64_t KB, int64_t G) {
   if (layout == 0) return i * KB + b;  // plain
   if (layout == 2) {                   // tiled gate/up: remap the row inside its [gate; up] stack
@@ -247,6 +203,147 @@ __global__ void __launch_bounds__(kRcThreads) quant_rowcol_kernel(const uint4* _
   }
 }
 
+// Both tiled quantisations of an expert-grouped routed-row operand, built straight from token-order
+// rows, so that no bf16 copy of the routed buffer is written (the MXFP8 layer's fused dispatch and
+// fused combine backward):
+//   GQ_X   padded row r holds x[t], t = row_token[r] / k                 (row-wise dispatch);
+//   GQ_DY  padded row r holds dy = bf16(gates[n] * dout[t]), n = row_token[r], t = n / k (the combine
+//          backward), and dgates[n] = <dout[t], y[r]> (fp32, fixed summation order) comes out on the
+//          way;
+// pad rows (row_token < 0) are zero. One CTA of 128 threads per 32-row block walks the row's
+// 128-column tiles; each tile is quantised exactly as quant_rowcol_kernel does (row blocks from
+// registers, column blocks through shared memory), so codes and scales are bit-identical to
+// quantising the bf16 routed buffer. Blocks at or past the used rows (poff[E]) are skipped: no GEMM
+// reads them.
+enum { GQ_X = 0, GQ_DY = 1 };
+
+template <int SRC>
+__global__ void __launch_bounds__(kRcThreads) gather_quant_kernel(
+    const uint4* __restrict__ tok, const int32_t* __restrict__ row_token,
+    const int32_t* __restrict__ poff_end, int k, int64_t rows, int cols,
+    const float* __restrict__ gates, const uint4* __restrict__ y, float* __restrict__ dgates,
+    uint2* __restrict__ qr, uint8_t* __restrict__ sr, uint4* __restrict__ qc, uint8_t* __restrict__ sc) {
+  __shared__ __align__(16) uint4 tile[kRcRows * kRcCols / 8];  // bf16 [32][128]
+  __shared__ __align__(16) uint8_t codes[kRcRows * kRcCols];    // column-block codes [32][128]
+  pdl_enter();  // wait for the previous kernel before any global access
+  const int64_t row0 = (int64_t)blockIdx.x * kRcRows;
+  if (row0 >= *poff_end) return;
+  const int t = threadIdx.x;
+  const int c16 = t & 15;        // this thread's 16-byte column word inside a tile
+  const int64_t w16 = cols / 8;  // 16-byte words per row
+  const int ctiles = cols / kRcCols;
+  const int kb = cols / 32;
+  // the four rows this thread loads: r = t/16 + 8i
+  int64_t srow[4];
+  int ent[4];
+  float g[4], dot[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = (t >> 4) + 8 * i;
+    const int n = row_token[row0 + r];
+    ent[i] = n;
+    srow[i] = n >= 0 ? (int64_t)(n / k) : -1;
+    g[i] = (SRC == GQ_DY && n >= 0) ? gates[n] : 0.f;
+    dot[i] = 0.f;
+  }
+  for (int cb = 0; cb < ctiles; ++cb) {
+    uint4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = (t >> 4) + 8 * i;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (srow[i] >= 0) w = tok[srow[i] * w16 + cb * 16 + c16];
+      if constexpr (SRC == GQ_DY) {
+        if (srow[i] >= 0) {
+          const uint4 yv = y[(row0 + r) * w16 + cb * 16 + c16];
+          const uint32_t du[4] = {w.x, w.y, w.z, w.w};
+          const uint32_t yu[4] = {yv.x, yv.y, yv.z, yv.w};
+          uint32_t o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float d0 = bf16lo(du[j]), d1 = bf16hi(du[j]);
+            dot[i] = fmaf(d0, bf16lo(yu[j]), dot[i]);
+            dot[i] = fmaf(d1, bf16hi(yu[j]), dot[i]);
+            o[j] = pack_bf16(g[i] * d0, g[i] * d1);
+          }
+          w = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      v[i] = w;
+    }
+    __syncthreads();  // the previous tile's shared buffers are free
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tile[((t >> 4) + 8 * i) * 16 + c16] = v[i];
+    // row blocks from registers: lanes 4j..4j+3 hold the 32 columns of one block of one row
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = (t >> 4) + 8 * i;
+      const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      float f[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        f[2 * j] = bf16lo(u[j]);
+        f[2 * j + 1] = bf16hi(u[j]);
+      }
+      float m = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(f[j]));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      uint8_t sb;
+      const float ir = exp2_exact(-block_exponent(m, &sb));
+      uint2 c;
+      c.x = cvt_e4m3x2(f[0] * ir, f[1] * ir) | ((uint32_t)cvt_e4m3x2(f[2] * ir, f[3] * ir) << 16);
+      c.y = cvt_e4m3x2(f[4] * ir, f[5] * ir) | ((uint32_t)cvt_e4m3x2(f[6] * ir, f[7] * ir) << 16);
+      if (!(m > 0.f)) c = make_uint2(0u, 0u);
+      qr[(row0 + r) * w16 + cb * 16 + c16] = c;
+      if ((t & 3) == 0) sr[tiled_sf_offset(row0 + r, (int64_t)cb * 4 + (c16 >> 2), kb)] = sb;
+    }
+    __syncthreads();
+    // column blocks: thread t owns column t of the tile (32 rows)
+    {
+      const __nv_bfloat16* tb = reinterpret_cast<const __nv_bfloat16*>(tile);
+      float f[kRcRows];
+      float amax = 0.f;
+#pragma unroll
+      for (int r = 0; r < kRcRows; ++r) {
+        f[r] = __bfloat162float(tb[r * kRcCols + t]);
+        amax = fmaxf(amax, fabsf(f[r]));
+      }
+      uint8_t sb;
+      const int e = block_exponent(amax, &sb);
+      const float inv = amax > 0.f ? exp2_exact(-e) : 0.f;
+      sc[tiled_sf_offset((int64_t)cb * kRcCols + t, blockIdx.x, rows / 32)] = sb;
+#pragma unroll
+      for (int r = 0; r < kRcRows; r += 2) {
+        const uint32_t c2 = amax > 0.f ? cvt_e4m3x2(f[r] * inv, f[r + 1] * inv) : 0u;
+        codes[r * kRcCols + t] = (uint8_t)(c2 & 0xFFu);
+        codes[(r + 1) * kRcCols + t] = (uint8_t)(c2 >> 8);
+      }
+    }
+    __syncthreads();
+    const uint4* cw = reinterpret_cast<const uint4*>(codes);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int idx = t + kRcThreads * j;  // 16-byte word of the code tile: 8 per row
+      const int r = idx >> 3, c = idx & 7;
+      qc[((row0 + r) * cols + (int64_t)cb * kRcCols) / 16 + c] = cw[idx];
+    }
+  }
+  if constexpr (SRC == GQ_DY) {
+    // the 16 threads that share a row hold its partial dot products over their columns
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float d = dot[i];
+      d += __shfl_xor_sync(0xffffffffu, d, 1);
+      d += __shfl_xor_sync(0xffffffffu, d, 2);
+      d += __shfl_xor_sync(0xffffffffu, d, 4);
+      d += __shfl_xor_sync(0xffffffffu, d, 8);
+      if (c16 == 0 && ent[i] >= 0) dgates[ent[i]] = d;
+    }
+  }
+}
+
 }  // namespace
 
 // Row-block and column-block tiled quantisations (MOE_QUANT_ROW_TILED into qr/sr, MOE_QUANT_COL_TILED
@@ -256,6 +353,33 @@ int launch_quantize_rowcol(const void* src, int64_t rows, int cols, uint8_t* qr,
   const int64_t grid = (rows / kRcRows) * (cols / kRcCols);
   MOE_LAUNCH(launch_pdl(quant_rowcol_kernel, (unsigned)grid, kRcThreads, 0, st,
                         static_cast<const uint4*>(src), rows, cols, reinterpret_cast<uint2*>(qr), sr,
+                        reinterpret_cast<uint4*>(qc), sc));
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// MXFP8 dispatch: both tiled quantisations of the routed input built from x [T, cols] through
+// row_token (rows = routed-row buffer rows, a multiple of 128; cols % 128 == 0).
+int launch_dispatch_quant(const void* x, const int32_t* row_token, const int32_t* poff_end, int k,
+                          int64_t rows, int cols, uint8_t* qr, uint8_t* sr, uint8_t* qc, uint8_t* sc,
+                          cudaStream_t st) {
+  MOE_LAUNCH(launch_pdl(gather_quant_kernel<GQ_X>, (unsigned)(rows / kRcRows), kRcThreads, 0, st,
+                        static_cast<const uint4*>(x), row_token, poff_end, k, rows, cols,
+                        (const float*)nullptr, (const uint4*)nullptr, (float*)nullptr,
+                        reinterpret_cast<uint2*>(qr), sr, reinterpret_cast<uint4*>(qc), sc));
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// MXFP8 combine backward: dy = bf16(g * dout) quantised both ways straight from dout [T, cols], and
+// dgates[n] = <dout[t], y[row]>.
+int launch_combine_bwd_quant(const void* dout, const void* y, const float* gates,
+                             const int32_t* row_token, const int32_t* poff_end, int k, int64_t rows,
+                             int cols, float* dgates, uint8_t* qr, uint8_t* sr, uint8_t* qc,
+                             uint8_t* sc, cudaStream_t st) {
+  MOE_LAUNCH(launch_pdl(gather_quant_kernel<GQ_DY>, (unsigned)(rows / kRcRows), kRcThreads, 0, st,
+                        static_cast<const uint4*>(dout), row_token, poff_end, k, rows, cols, gates,
+                        static_cast<const uint4*>(y), dgates, reinterpret_cast<uint2*>(qr), sr,
                         reinterpret_cast<uint4*>(qc), sc));
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

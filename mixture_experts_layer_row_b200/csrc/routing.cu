@@ -239,8 +239,13 @@ __global__ void __launch_bounds__(kChunk) rank_kernel(const int32_t* __restrict_
   for (int it = 0; it < 8; ++it) {
     if (it >= k) break;
     const int e = ex[it];
-    if (e < 0) continue;
     const int64_t n = seg + it * 32 + lane;
+    if (e < 0) {
+      // an expert id outside [0,E) (flagged by the histogram): the entry has no row; -1 makes the row
+      // kernels skip it instead of following a stale position
+      if (n < total) perm[n] = prow[n] = -1;
+      continue;
+    }
     const int r = chunk_base[(size_t)blockIdx.x * E + e] + wcnt[w][e] + lrank[it];
     perm[n] = offsets[e] + r;
     const int pr = poff[e] + r;

@@ -51,15 +51,20 @@ class MoELayer:
         self.counts, self.offsets, self.poff = z(E, i32), z(E + 1, i32), z(E + 1, i32)
         self.perm, self.prow, self.row_token = z(T * k, i32), z(T * k, i32), z(R, i32)
         self.recompute = recompute
-        self.x_perm, self.a, self.y = z((R, d), act), z((R, F), act), z((R, d), act)
+        self.mx = dtype == "mxfp8"
+        # MXFP8: the routed input, a, dy and dh13 exist only as their two quantised forms (qa_t)
+        self.x_perm = None if self.mx else z((R, d), act)
+        self.a = None if self.mx else z((R, F), act)
+        self.y = z((R, d), act)
         self.h13 = None if recompute else z((R, 2 * F), act)
         self.out = z((T, d), act)
         self.dx = z((T, d), act)
         self.dW13, self.dW2 = z((E, 2 * F, d), act), z((E, d, F), act)
         self.dW_r = z((E, d), act) if learned_router else None
         self.dgates = z((T, k), f32)
-        self.dy, self.dh13, self.dx_perm = z((R, d), act), z((R, 2 * F), act), z((R, d), act)
-        self.mx = dtype == "mxfp8"
+        self.dy = None if self.mx else z((R, d), act)
+        self.dh13 = None if self.mx else z((R, 2 * F), act)
+        self.dx_perm = z((R, d), act)
         if self.mx:
             u8 = torch.uint8
             self.qw_t = {  # quantised weights
@@ -77,6 +82,8 @@ class MoELayer:
             order = ["xq", "xs", "xtq", "xts", "aq", "as", "atq", "ats", "dyq", "dys", "dytq", "dyts",
                      "dhq", "dhs", "dhtq", "dhts"]
             self.qa = L.MxActs(*[L.ptr(self.qa_t[n]) for n in order])
+            self.q_ops = {nm: L.mx_operand(self.qa_t[nm + "q"], self.qa_t[nm + "s"], self.qa_t[nm + "tq"],
+                                           self.qa_t[nm + "ts"]) for nm in ("x", "a", "dy", "dh")}
         self.saved = L.Saved(*[L.ptr(t) for t in (self.logits, self.idx, self.gates, self.counts,
                                                   self.offsets, self.poff, self.perm, self.prow,
                                                   self.row_token, self.x_perm, self.h13, self.a,

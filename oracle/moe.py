@@ -374,6 +374,18 @@ def token_out(t, x, W13, W2, idx, gates) -> np.ndarray:
     return acc
 
 
+def token_expert_outputs(t, x, W13, W2, idx) -> np.ndarray:
+    """The k expert outputs of token t before gating, y_{S_t,j}(x_t) = W2_e (silu(W1_e x_t) * W3_e
+    x_t), one row per slot [k, d]; out_t is their gate-weighted sum and the gate gradient of slot j
+    is <dout_t, row j>."""
+    F = W13.shape[1] // 2
+    ys = np.zeros((idx.shape[1], x.shape[1]))
+    for j in range(idx.shape[1]):
+        e = int(idx[t, j])
+        ys[j] = W2[e] @ (silu(W13[e, :F] @ x[t]) * (W13[e, F:] @ x[t]))
+    return ys
+
+
 def token_dx(t, x, W13, W2, idx, gates, dout, W_r=None, renorm=True) -> np.ndarray:
     """d(loss)/d(x_t) for one token, straight from the definition (router term included when W_r
     is given, renormalised gates assumed)."""

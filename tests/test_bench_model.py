@@ -1,7 +1,7 @@
 """The benchmark's per-op work model (algorithmic bytes and flops behind every roofline figure),
 checked against plain counts on CPU: the op list follows the layer's launch order, the recompute
-variant adds exactly one GEMM1 and drops the h13 store from the forward one, and the MXFP8 step
-counts one read and two quantised writes per activation."""
+variant adds exactly one GEMM1 and drops the h13 store from the forward one, and the MXFP8 step's
+activations leave their producers quantised."""
 import bench
 from moe_workloads import WORKLOADS
 
@@ -39,13 +39,21 @@ def test_total_flops_are_the_layer_count():
     assert gemm == 3 * 2 * R * w.d * 3 * w.F
 
 
-def test_mxfp8_quantisation_counts_one_read_two_writes():
+def test_mxfp8_activations_leave_their_producers_quantised():
+    """MXFP8 step: no separate quantisation launch. Each routed activation is written only as its two
+    quantised forms (codes + 1/32 scale bytes each) by the kernel that produces it, which reads its bf16
+    inputs once; the op list is the fused layer's launch order."""
     w = WORKLOADS["e128_mxfp8"]
-    R, d, F = w.T * w.k, w.d, w.F
+    T, R, d, F, E, k = w.T, w.T * w.k, w.d, w.F, w.E, w.k
     ops = bench.op_work(w)
     q = lambda n: n + n // 32
-    assert ops["quant_x"] == (R * d * 2 + 2 * q(R * d), 0)
-    assert ops["quant_a"] == (R * F * 2 + 2 * q(R * F), 0)
-    assert ops["quant_dy"] == (R * d * 2 + 2 * q(R * d), 0)
-    assert ops["quant_dh"] == (R * 2 * F * 2 + 2 * q(R * 2 * F), 0)
-    assert not any(n.endswith("_row") or n.endswith("_col") for n in ops)
+    assert list(ops) == [
+        "route_metadata", "dispatch_quant", "gemm_fwd1_swiglu_quant", "gemm_fwd2", "combine",
+        "combine_bwd_quant", "gemm_dgrad2_swiglu_quant", "gemm_wgrad2", "gemm_dgrad1", "gemm_wgrad1",
+        "token_reduce"]
+    assert not any(n.startswith("quant_") for n in ops)
+    assert ops["dispatch_quant"] == (T * d * 2 + R * 4 + 2 * q(R * d), 0)
+    # GEMM1: fp8 x_perm and W13 read, bf16 h13 written, a written as two quantised forms
+    assert ops["gemm_fwd1_swiglu_quant"][0] == q(R * d) + q(E * 2 * F * d) + R * 2 * F * 2 + 2 * q(R * F)
+    assert ops["combine_bwd_quant"][0] == (T * d + R * d) * 2 + T * k * 8 + R * 4 + 2 * q(R * d)
+    assert ops["gemm_dgrad2_swiglu_quant"][0] == q(R * d) + q(E * d * F) + R * 2 * F * 2 + 2 * q(R * 2 * F)

@@ -255,3 +255,116 @@ def test_mx_wgrad(shape, which):
             assert np.all(DW[e] == 0)
         else:
             assert_close_rel(DW[e], O.gemm_wgrad(Gn[r0:r0 + n], Xn[r0:r0 + n], COLQ), TOL, f"dW e{e}")
+
+
+# ------------------------------------------------------------------------------------------------
+# Fused MXFP8 producers: the routed input, dy, a and dh13 leave their producing kernel only as their
+# two quantised forms. Codes and scales must equal the oracle's quantisers applied to the values the
+# unfused path holds in bf16 (bit for bit: the quantiser is exact given its input).
+# ------------------------------------------------------------------------------------------------
+
+def _operand(P, cols, fill=0xAB):
+    z = lambda *sh: torch.full(sh, fill, dtype=torch.uint8, device=dev())
+    t = dict(q_row=z(P.R32, cols), s_row=z(P.R32 * cols // 32), q_col=z(P.R32, cols),
+             s_col=z(P.R32 * cols // 32))
+    return t, P.L.mx_operand(t["q_row"], t["s_row"], t["q_col"], t["s_col"])
+
+
+def _check_operand(t, vals, used, R32, what):
+    """vals: [used, cols] fp64 values (exact bf16) of the routed operand's used rows; rows >= used are
+    not written by the fused kernels and are not compared."""
+    cols = vals.shape[1]
+    rq, rs = MX.quantize_rows(vals)
+    cq, cs = MX.quantize_cols(vals)
+    assert np.array_equal(t["q_row"][:used].cpu().numpy(), rq), what + " row codes"
+    assert np.array_equal(t["q_col"][:used].cpu().numpy(), cq), what + " column codes"
+    assert np.array_equal(t["s_row"][:used * cols // 32].cpu().numpy(), tiled(rs)), what + " row scales"
+    # column scales: tiled over (column, 32-row block) with R32/32 blocks per column
+    full = np.zeros((cols, R32 // 32), dtype=np.uint8)
+    full[:, :used // 32] = cs.T
+    ref = tiled(full)
+    mask = np.zeros((cols, R32 // 32), dtype=bool)
+    mask[:, :used // 32] = True
+    sel = tiled(mask.astype(np.uint8)).astype(bool)
+    assert np.array_equal(t["s_col"].cpu().numpy()[sel], ref[sel]), what + " column scales"
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_dispatch_mxfp8_bitexact(shape):
+    """Row-wise dispatch straight into the two MXFP8 forms = the oracle's dispatch (x_perm[prow] =
+    x[t], zero pad rows) quantised by the oracle."""
+    P = MxProblem(shape)
+    L = P.L
+    x = _bf16_matrix(P.T, P.d, 11 + P.T)
+    t, op = _operand(P, P.d)
+    row_token = torch.full((P.R32,), -1, dtype=torch.int32)
+    row_token[:len(P.meta["row_token"])] = torch.from_numpy(P.meta["row_token"].astype(np.int32))
+    L.dispatch_mxfp8(P.cfg, x.to(dev()), row_token.to(dev()), P.poff, op)
+    torch.cuda.synchronize()
+    used = int(P.meta["poff"][-1])
+    xp = O.dispatch(x.double().numpy(), P.meta, P.k)
+    _check_operand(t, xp[:used], used, P.R32, "x_perm")
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_combine_bwd_mxfp8(shape):
+    """Combine backward straight into dy's MXFP8 forms: dy = bf16(g * dout) quantised (bit-exact with
+    the oracle's quantiser of the oracle's bf16-stored dy), and the gate gradients <dout_t, y_row>."""
+    P = MxProblem(shape)
+    L = P.L
+    g = torch.Generator().manual_seed(3)
+    dout = torch.randn((P.T, P.d), generator=g).to(torch.bfloat16)
+    y = P.rows(P.d)
+    gates = torch.rand((P.T, P.k), generator=g)
+    t, op = _operand(P, P.d)
+    dgates = torch.full((P.T, P.k), 9.0, device=dev())
+    row_token = torch.full((P.R32,), -1, dtype=torch.int32)
+    row_token[:len(P.meta["row_token"])] = torch.from_numpy(P.meta["row_token"].astype(np.int32))
+    L.combine_bwd_mxfp8(P.cfg, dout.to(dev()), y.to(dev()), gates.to(dev()), row_token.to(dev()), P.poff,
+                        dgates, op)
+    torch.cuda.synchronize()
+    used = int(P.meta["poff"][-1])
+    dy, dg = O.combine_bwd(dout.double().numpy(), np64(y), gates.double().numpy(), P.meta)
+    _check_operand(t, O.bf16_round(dy[:used]), used, P.R32, "dy")
+    assert_close_rel(dgates.cpu().double().numpy(), dg, 1e-4, "dgates")
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_mx_fwd1_quantised_a(shape):
+    """GEMM1 + SwiGLU with a quantised in the epilogue: h13 equals the unfused GEMM's bit for bit, and
+    a's codes and scales equal the oracle's quantisers applied to the unfused GEMM's bf16 a (itself
+    checked against the oracle in test_mx_fwd1)."""
+    P = MxProblem(shape)
+    L = P.L
+    X, W13 = P.rows(P.d), P.weights(P.E, 2 * P.F, P.d)
+    XA, WB = P.quant(X, 0), P.quant(W13.reshape(-1, P.d), 0)
+    h13, a = P.run(L.GEMM_FWD1_SWIGLU, XA, WB, torch.zeros((P.R32, 2 * P.F), dtype=torch.bfloat16),
+                   torch.zeros((P.R32, P.F), dtype=torch.bfloat16))
+    h13q = torch.full((P.R32, 2 * P.F), 3.0, dtype=torch.bfloat16, device=dev())
+    t, op = _operand(P, P.F)
+    L.grouped_gemm_mxfp8_quant(P.cfg, L.GEMM_FWD1_SWIGLU, XA[0], XA[1], WB[0], WB[1], h13q, None, op,
+                               P.counts, P.poff, P.ws)
+    torch.cuda.synchronize()
+    assert L.get_error(P.ws) == 0
+    used = int(P.meta["poff"][-1])
+    assert torch.equal(h13q[:used], h13[:used])
+    _check_operand(t, np64(a)[:used], used, P.R32, "a")
+
+
+@pytest.mark.parametrize("shape", list(SHAPES))
+def test_mx_dgrad2_quantised_dh13(shape):
+    """GEMM2 dgrad + SwiGLU backward with dh13 quantised in the epilogue: codes and scales equal the
+    oracle's quantisers applied to the unfused GEMM's bf16 dh13 (checked in test_mx_dgrad2)."""
+    P = MxProblem(shape)
+    L = P.L
+    dY, W2, H13 = P.rows(P.d), P.weights(P.E, P.d, P.F), P.rows(2 * P.F, 2.0)
+    YA, WB = P.quant(dY, 0), P.quant(W2.reshape(-1, P.F), 1)
+    dh, _ = P.run(L.GEMM_DGRAD2_SWIGLU, YA, WB, torch.zeros((P.R32, 2 * P.F), dtype=torch.bfloat16),
+                  aux=H13)
+    t, op = _operand(P, 2 * P.F)
+    L.grouped_gemm_mxfp8_quant(P.cfg, L.GEMM_DGRAD2_SWIGLU, YA[0], YA[1], WB[0], WB[1], None,
+                               H13.to(dev()), op, P.counts, P.poff, P.ws)
+    torch.cuda.synchronize()
+    assert L.get_error(P.ws) == 0
+    used = int(P.meta["poff"][-1])
+    _check_operand(t, np64(dh)[:used], used, P.R32, "dh13")

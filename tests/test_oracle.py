@@ -625,3 +625,17 @@ def test_mxfp8_max_error_against_unquantised_is_the_formats_own():
     err = {"out": rel(outq, out), **{k: rel(grq[k], gr[k]) for k in ("dx", "dW13", "dW2", "dgates")}}
     assert all(0.02 < v < 0.2 for v in err.values()), err
     assert err["dW13"] > 0.08 and err["dW2"] > 0.08, err  # above the 8e-2 bar: the format, not a kernel
+
+
+def test_token_expert_outputs_sum_to_the_output_and_give_the_gate_gradients():
+    """Per-slot expert outputs of one token: their gate-weighted sum is the layer output, and their
+    inner products with dout are the grouped backward's gate gradients."""
+    k = 3
+    x, W_r, W13, W2, dout = _small_problem(9, T=20, d=8, F=6, E=5, k=k)
+    idx, g = O.route(O.router_logits(x, W_r), k)
+    out, saved = O.layer_fwd(x, W13, W2, idx, g)
+    gr = O.layer_bwd(dout, x, W13, W2, idx, g, saved)
+    for t in range(20):
+        ys = O.token_expert_outputs(t, x, W13, W2, idx)
+        np.testing.assert_allclose(g[t] @ ys, out[t], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(ys @ dout[t], gr["dgates"][t], rtol=1e-12, atol=1e-13)

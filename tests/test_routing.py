@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from oracle import moe as O
-from _util import dev, idx_from_counts
+from _util import assert_close_rel, dev, idx_from_counts, np64
 
 pytestmark = pytest.mark.gpu
 
@@ -154,3 +154,51 @@ def test_metadata_invalid_ids_flagged():
     valid = (idx >= 0) & (idx < 8)
     pr = got["prow"].reshape(idx.shape)[valid]
     assert np.all((pr >= 0) & (pr < R)) and len(np.unique(pr)) == pr.size
+    # the invalid entries have no row: perm and prow are -1 there (not a stale value)
+    assert np.all(got["prow"].reshape(idx.shape)[~valid] == -1)
+    assert np.all(got["perm"].reshape(idx.shape)[~valid] == -1)
+    assert np.array_equal(got["counts"], np.bincount(idx[valid], minlength=8))
+
+
+def test_row_kernels_skip_entries_without_a_row():
+    """An entry with an invalid expert id gets prow = -1; dispatch, combine, combine_bwd and the token
+    reduce skip it (no read or write through it) and treat the rest of the token as usual."""
+    L = _lib()
+    T, d, E, k = 64, 64, 8, 2
+    idx = _uniform_idx(T, E, k, 3).astype(np.int32)
+    idx[4, 1] = E + 3
+    idx[17, 0] = -1
+    valid = (idx >= 0) & (idx < E)
+    cfg = L.make_config(T, d, 128, E, k)
+    R = L.max_rows(cfg)
+    ws = torch.zeros(L.workspace_size(cfg), dtype=torch.uint8, device=dev())
+    z = lambda n: torch.full((n,), -99, dtype=torch.int32, device=dev())
+    counts, offsets, poff = z(E), z(E + 1), z(E + 1)
+    perm, prow, row_token = z(T * k), z(T * k), z(R)
+    tidx = torch.from_numpy(idx).to(dev())
+    L.route_metadata(cfg, tidx, counts, offsets, poff, perm, prow, row_token, ws)
+    g = torch.Generator(device=dev()).manual_seed(5)
+    x = torch.randn((T, d), generator=g, device=dev()).to(torch.bfloat16)
+    gates = torch.rand((T, k), generator=g, device=dev())
+    xp = torch.full((R, d), 7.0, dtype=torch.bfloat16, device=dev())
+    L.dispatch(cfg, x, prow, counts, poff, xp)
+    out = torch.empty((T, d), dtype=torch.bfloat16, device=dev())
+    L.combine(cfg, xp, gates, prow, out)
+    dy = torch.full((R, d), 7.0, dtype=torch.bfloat16, device=dev())
+    dg = torch.full((T, k), 5.0, device=dev())
+    L.combine_bwd(cfg, x, xp, gates, prow, tidx, counts, poff, dy, dg)
+    dx = torch.empty((T, d), dtype=torch.bfloat16, device=dev())
+    L.token_reduce(cfg, xp, prow, dx)
+    torch.cuda.synchronize()
+    assert L.get_error(ws) & L.DEVERR_ROUTING
+    pr = prow.cpu().numpy().reshape(T, k)
+    assert np.all(pr[~valid] == -1)
+    x64, g64 = np64(x), gates.cpu().double().numpy()
+    w = np.where(valid, g64, 0.0)
+    assert_close_rel(np64(out), w.sum(1)[:, None] * x64, 1e-2, "combine")
+    assert_close_rel(np64(dx), valid.sum(1)[:, None] * x64, 1e-2, "token reduce")
+    dgn = dg.cpu().numpy()
+    assert np.all(dgn[~valid] == 0.0)  # no row: nothing to contract with
+    used = int(poff[E])
+    xpn = np64(xp)
+    assert np.all(xpn[used:] == 7.0)  # rows past the groups untouched

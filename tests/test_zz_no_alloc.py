@@ -53,3 +53,28 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     rc = L.lib.moe_route_metadata_noalloc(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake,
                                           fake, None)
     assert rc == -3  # MOE_ERR_WORKSPACE, nothing enqueued
+
+
+def test_noalloc_invalid_ids_get_no_row():
+    """An expert id outside [0,E) is skipped by the allocation-free variant as by the workspace one:
+    perm and prow are -1 for that entry (this variant has no error flag to raise)."""
+    from mixture_experts_layer_row_b200 import _lib as L
+    dev = torch.device("cuda", 0)
+    T, E, k = 300, 8, 2
+    cfg = L.make_config(T, 64, 128, E, k)
+    idx_np = _idx(T, E, k, 7)
+    idx_np[5, 0] = E
+    idx_np[9, 1] = -3
+    idx = torch.from_numpy(idx_np).to(dev)
+    ws = torch.zeros(L.workspace_size(cfg), dtype=torch.uint8, device=dev)
+    ref, got = _outputs(L, cfg, dev), _outputs(L, cfg, dev)
+    L.route_metadata(cfg, idx, ref["counts"], ref["offsets"], ref["poff"], ref["perm"], ref["prow"],
+                     ref["row_token"], ws)
+    L.route_metadata_noalloc(cfg, idx, got["counts"], got["offsets"], got["poff"], got["perm"],
+                             got["prow"], got["row_token"])
+    torch.cuda.synchronize()
+    for name in ref:
+        assert torch.equal(got[name], ref[name]), name
+    bad = ~((idx_np >= 0) & (idx_np < E))
+    assert np.all(got["prow"].cpu().numpy().reshape(T, k)[bad] == -1)
+    assert np.all(got["perm"].cpu().numpy().reshape(T, k)[bad] == -1)
