@@ -575,6 +575,7 @@ def main():
         for n in step.names:
             per_op[n] += step.op_ms(i, n)
     per_op = {n: v / args.steps for n, v in per_op.items()}
+    ms_instrumented = sum(step.ev[i][0].elapsed_time(step.ev[i][-1]) for i in range(args.steps)) / args.steps
     dom = max(per_op, key=lambda n: per_op[n])
     # timed region: K steps issued back to back as the layer API issues them, with events only around
     # the dominant kernel (its duration for the roofline)
@@ -796,6 +797,7 @@ def main():
             "per_op_ms": {n: round(v, 4) for n, v in per_op.items()},
             "per_op_note": "instrumented pass of K steps with an event at every op boundary, run before "
                            "the timed region (each event serialises the kernels around it)",
+            "ms_per_step_instrumented": ms_instrumented,
             "per_op_hbm": hbm_ops,
             "weight_quantisation": wq,
             "cpu_baseline": cpu,

@@ -426,6 +426,67 @@ MOE_API int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w,
                                 const moe_mxfp8_acts_t* qa, const void* x, const void* dout, void* dx,
                                 moe_grads_t* g, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- expert parallelism across the GPUs of one node (bf16) --------------------------------------------
+ *
+ * Row-wise expert parallelism (unite.ai, "Parallelismo, precisione e tecniche di memoria": each routed
+ * token row goes directly into the input buffer of the expert that owns it, then device-scheduled
+ * grouped GEMMs run every GPU's local experts). G = world ranks, one GPU each (G <= 8, E % G == 0);
+ * rank h owns the E/G consecutive experts [h*E/G, (h+1)*E/G). cfg is the per-rank config: T = this
+ * rank's tokens, E = all experts. Per step:
+ *   1. each rank: moe_route_metadata on its own idx (counts over all E experts, offsets, perm);
+ *   2. the caller all-gathers the ranks' counts into all_counts [G][E] (int32, rank-major) with a
+ *      collective on the stream (NCCL all_gather);
+ *   3. each rank: moe_ep_layout -- every rank derives the same layout of every owner's routed-row
+ *      buffers: local expert e's group starts at poff_loc[e] (32-aligned), and inside it the rows of
+ *      source rank 0 come first, then rank 1, ...; each source's rows in its own token order;
+ *   4. after a collective that orders the ranks (the owners' buffers are free), moe_ep_dispatch stores
+ *      this rank's token rows into the owners' x_perm through peer pointers; each owner zeroes its pad
+ *      rows with moe_ep_zero_pad;
+ *   5. after a collective (every dispatch is done), each owner runs the grouped GEMMs on its local
+ *      experts with cfg_loc = {T: G*T*k, k: 1, E: E/G} (so moe_max_rows(cfg_loc) == moe_ep_max_rows),
+ *      counts_loc and poff_loc;
+ *   6. after a collective, moe_ep_combine gathers the k expert outputs of each token from the owners.
+ *   Backward: moe_ep_combine_bwd (dy stored into the owners, gate gradients), moe_ep_zero_pad of dy,
+ *   a collective, the owners' dgrad / wgrad GEMMs, a collective, moe_ep_token_reduce.
+ * Peer arguments ("*_peers") are HOST arrays of G device pointers, entry h = that buffer on rank h (a
+ * peer mapping on a multi-GPU node, e.g. symmetric memory; any device pointers the GPU can reach).
+ * Kernels never wait on another GPU: the caller's collectives order the phases. */
+
+/* Rows of each owner's routed-row buffers: G*T*k + 31*E/G rounded up to 32 (every entry of every rank
+ * could go to one owner). Returns 0 for an invalid config or world. */
+MOE_API int64_t moe_ep_max_rows(const moe_config_t* cfg, int world);
+
+/* Step 3. all_counts [G][E] int32; idx [T,k], perm and offsets from this rank's moe_route_metadata.
+ * Outputs: src_base [E] (row, in the owner's buffers, of this rank's first entry for each expert),
+ * counts_loc [E/G] and poff_loc [E/G + 1] (this rank as owner), dst_row [T*k] (each entry's row in its
+ * owner's buffers; -1 for an expert id outside [0,E)). */
+MOE_API int moe_ep_layout(const moe_config_t* cfg, int rank, int world, const int32_t* all_counts,
+                          const int32_t* idx, const int32_t* perm, const int32_t* offsets,
+                          int32_t* src_base, int32_t* counts_loc, int32_t* poff_loc, int32_t* dst_row,
+                          void* stream);
+
+/* Zero the owner's pad rows [poff_loc[e] + counts_loc[e], poff_loc[e+1]) of buf [moe_ep_max_rows, d]. */
+MOE_API int moe_ep_zero_pad(const moe_config_t* cfg, int world, void* buf, const int32_t* counts_loc,
+                            const int32_t* poff_loc, void* stream);
+
+/* x_perm_owner[dst_row[t*k+j]] = x[t] (owner = idx[t,j] / (E/G)), peer stores. x: bf16 [T,d]. */
+MOE_API int moe_ep_dispatch(const moe_config_t* cfg, int world, const void* x, const int32_t* idx,
+                            const int32_t* dst_row, void* const* x_perm_peers, void* stream);
+
+/* out[t] = sum_j gates[t,j] * y_owner[dst_row[t*k+j]] (fp32 accumulation), peer loads. */
+MOE_API int moe_ep_combine(const moe_config_t* cfg, int world, void* const* y_peers, const float* gates,
+                           const int32_t* idx, const int32_t* dst_row, void* out, void* stream);
+
+/* dy_owner[row] = gates[t,j] * dout[t] (peer stores), dgates[t,j] = <dout[t], y_owner[row]> (peer
+ * loads), row = dst_row[t*k+j]. A learned router's score gradients are not formed here. */
+MOE_API int moe_ep_combine_bwd(const moe_config_t* cfg, int world, const void* dout, void* const* y_peers,
+                               const float* gates, const int32_t* idx, const int32_t* dst_row,
+                               void* const* dy_peers, float* dgates, void* stream);
+
+/* dx[t] = sum_j dx_perm_owner[dst_row[t*k+j]], peer loads. */
+MOE_API int moe_ep_token_reduce(const moe_config_t* cfg, int world, void* const* dx_perm_peers,
+                                const int32_t* idx, const int32_t* dst_row, void* dx, void* stream);
+
 /* ---- test support ------------------------------------------------------------------------------------- */
 
 /* Launch one block whose thread waits on a pipeline barrier that nothing ever completes, with the

@@ -28,7 +28,8 @@ EXPORTS = [
     "moe_test_bounded_wait", "moe_version", "moe_launch_count", "moe_route_metadata_noalloc",
     "moe_quantize_mxfp8", "moe_quantize_mxfp8_rowcol", "moe_grouped_gemm_mxfp8", "moe_quantize_weights_mxfp8",
     "moe_layer_fwd_mxfp8", "moe_layer_bwd_mxfp8", "moe_dispatch_mxfp8", "moe_combine_bwd_mxfp8",
-    "moe_grouped_gemm_mxfp8_quant",
+    "moe_grouped_gemm_mxfp8_quant", "moe_ep_max_rows", "moe_ep_layout", "moe_ep_zero_pad",
+    "moe_ep_dispatch", "moe_ep_combine", "moe_ep_combine_bwd", "moe_ep_token_reduce",
 ]
 
 
@@ -113,6 +114,14 @@ def _load():
         "moe_combine_bwd_mxfp8": ([cfgp, vp, vp, vp, vp, vp, vp, ctypes.POINTER(MxOperand), vp], i),
         "moe_grouped_gemm_mxfp8_quant": ([cfgp, i, vp, vp, vp, vp, vp, vp, ctypes.POINTER(MxOperand),
                                           vp, vp, vp, sz, vp], i),
+        "moe_ep_max_rows": ([cfgp, i], ctypes.c_int64),
+        "moe_ep_layout": ([cfgp, i, i, vp, vp, vp, vp, vp, vp, vp, vp, vp], i),
+        "moe_ep_zero_pad": ([cfgp, i, vp, vp, vp, vp], i),
+        "moe_ep_dispatch": ([cfgp, i, vp, vp, vp, ctypes.POINTER(vp), vp], i),
+        "moe_ep_combine": ([cfgp, i, ctypes.POINTER(vp), vp, vp, vp, vp, vp], i),
+        "moe_ep_combine_bwd": ([cfgp, i, vp, ctypes.POINTER(vp), vp, vp, vp, ctypes.POINTER(vp), vp,
+                                vp], i),
+        "moe_ep_token_reduce": ([cfgp, i, ctypes.POINTER(vp), vp, vp, vp, vp], i),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -320,6 +329,50 @@ def layer_bwd_mxfp8(cfg, weights, qw, saved, qa, x, dout, dx, grads, ws, stream=
                                   ctypes.byref(saved), ctypes.byref(qa), ptr(x), ptr(dout), ptr(dx),
                                   ctypes.byref(grads), w, n, stream_handle(stream)),
           "moe_layer_bwd_mxfp8")
+
+
+# ---- expert parallelism across the GPUs of one node -----------------------------------------------
+
+def peer_array(ptrs) -> ctypes.Array:
+    """A host array of device pointers (one per rank) for the *_peers arguments."""
+    return (ctypes.c_void_p * len(ptrs))(*[ctypes.c_void_p(int(p)) for p in ptrs])
+
+
+def ep_max_rows(cfg, world) -> int:
+    return int(lib.moe_ep_max_rows(ctypes.byref(cfg), int(world)))
+
+
+def ep_layout(cfg, rank, world, all_counts, idx, perm, offsets, src_base, counts_loc, poff_loc, dst_row,
+              stream=None):
+    check(lib.moe_ep_layout(ctypes.byref(cfg), int(rank), int(world), ptr(all_counts), ptr(idx), ptr(perm),
+                            ptr(offsets), ptr(src_base), ptr(counts_loc), ptr(poff_loc), ptr(dst_row),
+                            stream_handle(stream)), "moe_ep_layout")
+
+
+def ep_zero_pad(cfg, world, buf, counts_loc, poff_loc, stream=None):
+    check(lib.moe_ep_zero_pad(ctypes.byref(cfg), int(world), ptr(buf), ptr(counts_loc), ptr(poff_loc),
+                              stream_handle(stream)), "moe_ep_zero_pad")
+
+
+def ep_dispatch(cfg, world, x, idx, dst_row, x_perm_peers, stream=None):
+    check(lib.moe_ep_dispatch(ctypes.byref(cfg), int(world), ptr(x), ptr(idx), ptr(dst_row),
+                              x_perm_peers, stream_handle(stream)), "moe_ep_dispatch")
+
+
+def ep_combine(cfg, world, y_peers, gates, idx, dst_row, out, stream=None):
+    check(lib.moe_ep_combine(ctypes.byref(cfg), int(world), y_peers, ptr(gates), ptr(idx), ptr(dst_row),
+                             ptr(out), stream_handle(stream)), "moe_ep_combine")
+
+
+def ep_combine_bwd(cfg, world, dout, y_peers, gates, idx, dst_row, dy_peers, dgates, stream=None):
+    check(lib.moe_ep_combine_bwd(ctypes.byref(cfg), int(world), ptr(dout), y_peers, ptr(gates), ptr(idx),
+                                 ptr(dst_row), dy_peers, ptr(dgates), stream_handle(stream)),
+          "moe_ep_combine_bwd")
+
+
+def ep_token_reduce(cfg, world, dx_perm_peers, idx, dst_row, dx, stream=None):
+    check(lib.moe_ep_token_reduce(ctypes.byref(cfg), int(world), dx_perm_peers, ptr(idx), ptr(dst_row),
+                                  ptr(dx), stream_handle(stream)), "moe_ep_token_reduce")
 
 
 def version() -> str:

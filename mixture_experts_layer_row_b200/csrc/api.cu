@@ -705,6 +705,80 @@ int moe_layer_bwd_mxfp8(const moe_config_t* cfg, const moe_weights_t* w, const m
   return MOE_OK;
 }
 
+// ---- expert parallelism across the GPUs of one node ------------------------------------------------
+
+namespace {
+int check_ep(const moe_config_t* cfg, int world) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(world >= 1 && world <= kMaxEpRanks, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(cfg->E % world == 0, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(cfg->dtype == MOE_DTYPE_BF16, MOE_ERR_UNSUPPORTED);
+  return MOE_OK;
+}
+int64_t ep_rows(const moe_config_t* c, int world) {
+  const int64_t EL = c->E / world;
+  return ((int64_t)world * c->T * c->k + 31 * EL + 31) / 32 * 32;
+}
+}  // namespace
+
+int64_t moe_ep_max_rows(const moe_config_t* cfg, int world) {
+  if (check_ep(cfg, world) != MOE_OK) return 0;
+  const int64_t r = ep_rows(cfg, world);
+  return r < (1ll << 31) - 256 ? r : 0;
+}
+
+int moe_ep_layout(const moe_config_t* cfg, int rank, int world, const int32_t* all_counts,
+                  const int32_t* idx, const int32_t* perm, const int32_t* offsets, int32_t* src_base,
+                  int32_t* counts_loc, int32_t* poff_loc, int32_t* dst_row, void* stream) {
+  MOE_TRY(check_ep(cfg, world));
+  MOE_REQUIRE(rank >= 0 && rank < world, MOE_ERR_INVALID_ARG);
+  MOE_REQUIRE(all_counts && idx && perm && offsets && src_base && counts_loc && poff_loc && dst_row,
+              MOE_ERR_INVALID_ARG);
+  return launch_ep_layout(all_counts, world, cfg->E, rank, idx, perm, offsets,
+                          (int64_t)cfg->T * cfg->k, src_base, counts_loc, poff_loc, dst_row, S(stream));
+}
+
+int moe_ep_zero_pad(const moe_config_t* cfg, int world, void* buf, const int32_t* counts_loc,
+                    const int32_t* poff_loc, void* stream) {
+  MOE_TRY(check_ep(cfg, world));
+  MOE_REQUIRE(buf && counts_loc && poff_loc && aligned16(buf), MOE_ERR_INVALID_ARG);
+  return launch_ep_zero_pad(buf, counts_loc, poff_loc, cfg->E / world, cfg->d * 2, S(stream));
+}
+
+int moe_ep_dispatch(const moe_config_t* cfg, int world, const void* x, const int32_t* idx,
+                    const int32_t* dst_row, void* const* x_perm_peers, void* stream) {
+  MOE_TRY(check_ep(cfg, world));
+  MOE_REQUIRE(x && idx && dst_row && x_perm_peers && aligned16(x), MOE_ERR_INVALID_ARG);
+  return launch_ep_rows(0, world, cfg->T, cfg->k, cfg->E, cfg->d * 2, ep_rows(cfg, world), x,
+                        x_perm_peers, nullptr, nullptr, idx, dst_row, nullptr, nullptr, S(stream));
+}
+
+int moe_ep_combine(const moe_config_t* cfg, int world, void* const* y_peers, const float* gates,
+                   const int32_t* idx, const int32_t* dst_row, void* out, void* stream) {
+  MOE_TRY(check_ep(cfg, world));
+  MOE_REQUIRE(y_peers && gates && idx && dst_row && out && aligned16(out), MOE_ERR_INVALID_ARG);
+  return launch_ep_rows(1, world, cfg->T, cfg->k, cfg->E, cfg->d * 2, ep_rows(cfg, world), nullptr,
+                        y_peers, nullptr, gates, idx, dst_row, out, nullptr, S(stream));
+}
+
+int moe_ep_combine_bwd(const moe_config_t* cfg, int world, const void* dout, void* const* y_peers,
+                       const float* gates, const int32_t* idx, const int32_t* dst_row,
+                       void* const* dy_peers, float* dgates, void* stream) {
+  MOE_TRY(check_ep(cfg, world));
+  MOE_REQUIRE(dout && y_peers && gates && idx && dst_row && dy_peers && dgates && aligned16(dout),
+              MOE_ERR_INVALID_ARG);
+  return launch_ep_rows(2, world, cfg->T, cfg->k, cfg->E, cfg->d * 2, ep_rows(cfg, world), dout,
+                        y_peers, dy_peers, gates, idx, dst_row, nullptr, dgates, S(stream));
+}
+
+int moe_ep_token_reduce(const moe_config_t* cfg, int world, void* const* dx_perm_peers,
+                        const int32_t* idx, const int32_t* dst_row, void* dx, void* stream) {
+  MOE_TRY(check_ep(cfg, world));
+  MOE_REQUIRE(dx_perm_peers && idx && dst_row && dx && aligned16(dx), MOE_ERR_INVALID_ARG);
+  return launch_ep_rows(3, world, cfg->T, cfg->k, cfg->E, cfg->d * 2, ep_rows(cfg, world), nullptr,
+                        dx_perm_peers, nullptr, nullptr, idx, dst_row, dx, nullptr, S(stream));
+}
+
 int moe_test_bounded_wait(void* ws, uint64_t limit_ns, void* stream) {
   MOE_REQUIRE(ws, MOE_ERR_INVALID_ARG);
   return launch_bounded_wait_probe(err_of(ws), limit_ns, S(stream));

@@ -75,11 +75,12 @@ struct Cfg {
   // MXFP8 tiles of 256 columns, whose per-stage scale columns leave no room for a second
   static constexpr int NACC = (MX && BN == 256) ? 1 : 2;
   static_assert(!epi_quant(EPI) || (MX && !PAIR), "quantising epilogues are MXFP8-only");
-  // staging boxes per epilogue warp: SwiGLU forward h13 gate + up + a (quantising: gate + up + a's row
-  // codes + a's column codes); SwiGLU backward dh13 gate + up (quantising: row and column codes of
-  // each); stores round robin over NBUF boxes
+  // staging boxes per epilogue warp: SwiGLU forward h13 gate + up + a (quantising: gate + up; a's codes
+  // go straight to global memory); SwiGLU backward dh13 gate + up (quantising: none, dh13's codes go
+  // straight to global memory); plain stores round robin over NBUF boxes
   static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3
-                              : epi_quant(EPI)        ? 4
+                              : (EPI == EPI_SWIGLU_FWD_Q) ? 2
+                              : (EPI == EPI_SWIGLU_BWD_Q) ? 0
                               : (EPI == EPI_SWIGLU_BWD) ? 2
                               : (NACC == 1 ? 1 : 2);
   static constexpr int STAGING_BYTES = 4 * NBUF * 4096;
@@ -234,12 +235,12 @@ __device__ __forceinline__ void stage_row32(uint8_t* box, int lane, int ch0, con
   }
 }
 
-// Write 32 one-byte codes (8 words, column order) of this thread's row into a staged 32-row x 128-byte
-// box (128B swizzle) at 32-byte position `pos` (0..3).
-__device__ __forceinline__ void stage_codes32(uint8_t* box, int lane, int pos, const uint32_t (&c)[8]) {
-  uint8_t* row = box + lane * 128;
-  st_shared_v4(row + (((2 * pos) ^ (lane & 7)) << 4), make_uint4(c[0], c[1], c[2], c[3]));
-  st_shared_v4(row + (((2 * pos + 1) ^ (lane & 7)) << 4), make_uint4(c[4], c[5], c[6], c[7]));
+// Store 32 one-byte codes (8 words, column order) of this thread's row: one whole, aligned 32-byte
+// sector of the [rows, cols] code array (the chunk's first column is a multiple of 32).
+__device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t (&c)[8]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(c[0], c[1], c[2], c[3]);
+  d[1] = make_uint4(c[4], c[5], c[6], c[7]);
 }
 
 // Hand a fully written box to the TMA unit: every lane fences its writes, lane 0 stores the box.
@@ -287,8 +288,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
                         const __grid_constant__ CUtensorMap tmC2,
                         const __grid_constant__ CUtensorMap tmX1,
                         const __grid_constant__ CUtensorMap tmX2, const GemmParams p) {
-  // tmX1 / tmX2: pair tail tiles -- 64-row boxes of A / of B (SwiGLU forward); quantising epilogues --
-  // the row-block / column-block code outputs
+  // tmX1 / tmX2: pair tail tiles -- 64-row boxes of A / of B (SwiGLU forward)
   const CUtensorMap& tmA64 = tmX1;
   const CUtensorMap& tmB64 = tmX2;
   using C = Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>;
@@ -337,10 +337,6 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     prefetch_tensormap(&tmB);
     prefetch_tensormap(&tmC);
     if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmC2);
-    if constexpr (epi_quant(EPI)) {
-      prefetch_tensormap(&tmX1);
-      prefetch_tensormap(&tmX2);
-    }
     if constexpr (PAIR && MODE == GROUP_M) {
       prefetch_tensormap(&tmA64);
       if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmB64);
@@ -737,9 +733,8 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           tmem_ld_32x32b_x32(t_row + UP, ua);
           uint8_t* bg = wstg;
           uint8_t* bu = wstg + 4096;
-          uint8_t* ba = wstg + 8192;   // a (bf16), or a's row-block codes
-          uint8_t* bac = wstg + 12288;  // a's column-block codes (quantising)
-          uint32_t srow = 0;            // row-block scale bytes of four consecutive chunks
+          uint8_t* ba = wstg + 8192;  // a (bf16; not used by the quantising variant)
+          uint32_t srow = 0;           // row-block scale bytes of four consecutive chunks
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
             uint32_t(&rg)[32] = (j & 1) ? gb : ga;
@@ -775,8 +770,9 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               uint32_t cr[8], cc[8];
               srow |= (uint32_t)mx_row_block(a, cr) << (8 * (j & 3));
               const uint8_t scol = mx_col_blocks(a, lane, cc);
-              stage_codes32(ba, lane, j & 3, cr);
-              stage_codes32(bac, lane, j & 3, cc);
+              const size_t off = (size_t)(c1 + lane) * (p.q_kb_row * 32) + col0 + j * 32;
+              store_codes32(p.q_qr + off, cr);
+              store_codes32(p.q_qc + off, cc);
               p.q_sc[tiled_sf_offset(col0 + j * 32 + lane, qrb, p.q_kb_col)] = scol;
             } else {
               stage_row32<C::OES>(ba, lane, ch0, a);
@@ -790,10 +786,8 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               if constexpr (EPI == EPI_SWIGLU_FWD) box_store(&tmC2, ba, lane, c, c1);
             }
             if constexpr (EPI == EPI_SWIGLU_FWD_Q) {
-              if ((j & 3) == 3) {  // 128 columns of codes: one box each, and the row's 4 scale bytes
+              if ((j & 3) == 3) {  // the row's 4 scale bytes of 128 columns
                 const int c = col0 + (j & ~3) * 32;
-                box_store(&tmX1, ba, lane, c, c1);
-                box_store(&tmX2, bac, lane, c, c1);
                 *reinterpret_cast<uint32_t*>(p.q_sr + tiled_sf_offset(c1 + lane, c >> 5, p.q_kb_row)) = srow;
                 srow = 0;
               }
@@ -822,9 +816,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           }
           uint8_t* bg = wstg;
           uint8_t* bu = wstg + 4096;
-          uint8_t* bgc = wstg + 8192;   // quantising: column-block codes of the gate half
-          uint8_t* buc = wstg + 12288;  // and of the up half
-          uint32_t srg = 0, sru = 0;    // row-block scale bytes of four consecutive chunks
+          uint32_t srg = 0, sru = 0;  // quantising: row-block scale bytes of four consecutive chunks
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
             uint32_t(&rd)[32] = (j & 1) ? db : da;
@@ -841,7 +833,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               }
             }
             if (cols) {
-              if (j % (EPI == EPI_SWIGLU_BWD_Q ? 4 : CPB) == 0) {
+              if (EPI == EPI_SWIGLU_BWD && j % CPB == 0) {
                 if (lane == 0) bulk_wait_read<0>();
                 __syncwarp();
               }
@@ -863,22 +855,19 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
                   g[i] = round_out<2>(g[i]);
                   u[i] = round_out<2>(u[i]);
                 }
+                const size_t row_off = (size_t)(c1 + lane) * (p.q_kb_row * 32);
                 srg |= (uint32_t)mx_row_block(g, cr) << (8 * (j & 3));
                 uint8_t sc = mx_col_blocks(g, lane, cc);
-                stage_codes32(bg, lane, j & 3, cr);
-                stage_codes32(bgc, lane, j & 3, cc);
+                store_codes32(p.q_qr + row_off + col, cr);
+                store_codes32(p.q_qc + row_off + col, cc);
                 p.q_sc[tiled_sf_offset(col + lane, qrb, p.q_kb_col)] = sc;
                 sru |= (uint32_t)mx_row_block(u, cr) << (8 * (j & 3));
                 sc = mx_col_blocks(u, lane, cc);
-                stage_codes32(bu, lane, j & 3, cr);
-                stage_codes32(buc, lane, j & 3, cc);
+                store_codes32(p.q_qr + row_off + p.F + col, cr);
+                store_codes32(p.q_qc + row_off + p.F + col, cc);
                 p.q_sc[tiled_sf_offset(p.F + col + lane, qrb, p.q_kb_col)] = sc;
                 if ((j & 3) == 3) {
                   const int c = ti.n0 + (j & ~3) * 32;
-                  box_store(&tmX1, bg, lane, c, c1);
-                  box_store(&tmX1, bu, lane, p.F + c, c1);
-                  box_store(&tmX2, bgc, lane, c, c1);
-                  box_store(&tmX2, buc, lane, p.F + c, c1);
                   *reinterpret_cast<uint32_t*>(p.q_sr + tiled_sf_offset(c1 + lane, c >> 5, p.q_kb_row)) = srg;
                   *reinterpret_cast<uint32_t*>(p.q_sr + tiled_sf_offset(c1 + lane, (p.F + c) >> 5, p.q_kb_row)) = sru;
                   srg = sru = 0;
@@ -1095,19 +1084,12 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   const int64_t out_cols = (epi_swiglu_fwd(EPI) || epi_swiglu_bwd(EPI)) ? 2 * (int64_t)p.F : p.N;
   if (EPI == EPI_SWIGLU_FWD && !make_tmap(&tc2, p.C2, C::OES, out_rows, p.F, p.ldc2, C::OEPR, 32, 2))
     return MOE_ERR_CUDA;
-  // quantising epilogues: code outputs [rows, F] (a) or [rows, 2F] (dh13), 32-row x 128-byte boxes
-  CUtensorMap tq1, tq2;
-  if (epi_quant(EPI)) {
-    const int64_t qcols = EPI == EPI_SWIGLU_FWD_Q ? p.F : 2 * (int64_t)p.F;
-    if (!p.q_qr || !p.q_qc || !p.q_sr || !p.q_sc) return MOE_ERR_INVALID_ARG;
-    if (!make_tmap(&tq1, p.q_qr, 1, out_rows, qcols, qcols, 128, 32, 2) ||
-        !make_tmap(&tq2, p.q_qc, 1, out_rows, qcols, qcols, 128, 32, 2))
-      return MOE_ERR_CUDA;
-  }
+  // quantising epilogues: the codes [rows, F] (a) or [rows, 2F] (dh13) are stored from registers
+  if (epi_quant(EPI) && (!p.q_qr || !p.q_qc || !p.q_sr || !p.q_sc)) return MOE_ERR_INVALID_ARG;
   if (p.C) {
     if (!make_tmap(&tc, p.C, C::OES, out_rows, out_cols, p.ldc, C::OEPR, 32, 2)) return MOE_ERR_CUDA;
   } else if (EPI == EPI_SWIGLU_BWD_Q) {
-    tc = tq1;  // dh13 leaves as codes only: tc is never used
+    tc = ta;  // dh13 leaves as codes only: tc is never used
   } else if (EPI == EPI_SWIGLU_FWD) {
     tc = tc2;  // SwiGLU forward without h13: only a is stored, tc is never used
   } else {
@@ -1117,10 +1099,6 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   // pair tail tiles (M = 128 over the pair): 64-row boxes of A, and of B for the SwiGLU forward,
   // whose tail tile loads 64 gate + 64 up rows per CTA
   CUtensorMap ta64 = ta, tb64 = tb;
-  if (epi_quant(EPI)) {
-    ta64 = tq1;
-    tb64 = tq2;
-  }
   if (PAIR && MODE == GROUP_M) {
     if (!make_tmap(&ta64, A.ptr, ES, A.rows, A.cols, A.ld, C::EPR, C::HALF_M, 2)) return MOE_ERR_CUDA;
     if (EPI == EPI_SWIGLU_FWD &&

@@ -163,4 +163,19 @@ int launch_token_reduce(const void* dxp, const int32_t* prow, const float* dlsel
                         const void* Wr, void* dx, int T, int k, int E, int row_bytes, bool bf16,
                         int64_t max_rows, cudaStream_t s);
 
+// Expert parallelism across the GPUs of one node (ep.cu). Up to kMaxEpRanks ranks.
+constexpr int kMaxEpRanks = 8;
+int launch_ep_layout(const int32_t* all_counts, int G, int E, int rank, const int32_t* idx,
+                     const int32_t* perm, const int32_t* offsets, int64_t n_entries,
+                     int32_t* src_base, int32_t* counts_loc, int32_t* poff_loc, int32_t* dst_row,
+                     cudaStream_t s);
+int launch_ep_zero_pad(void* buf, const int32_t* counts_loc, const int32_t* poff_loc, int EL,
+                       int row_bytes, cudaStream_t s);
+// op 0 dispatch (x -> peers_a), 1 combine (peers_a = y -> out), 2 combine backward (dout, peers_a = y,
+// peers_b = dy, dgates), 3 token reduce (peers_a = dx_perm -> out)
+int launch_ep_rows(int op, int G, int T, int k, int E, int row_bytes, int64_t max_rows,
+                   const void* x_or_dout, void* const* peers_a, void* const* peers_b,
+                   const float* gates, const int32_t* idx, const int32_t* dst_row, void* out,
+                   float* dgates, cudaStream_t s);
+
 }  // namespace moe

@@ -210,12 +210,85 @@ __global__ void __launch_bounds__(kRcThreads) quant_rowcol_kernel(const uint4* _
 //   GQ_DY  padded row r holds dy = bf16(gates[n] * dout[t]), n = row_token[r], t = n / k (the combine
 //          backward), and dgates[n] = <dout[t], y[r]> (fp32, fixed summation order) comes out on the
 //          way;
-// pad rows (row_token < 0) are zero. One CTA of 128 threads per 32-row block walks the row's
-// 128-column tiles; each tile is quantised exactly as quant_rowcol_kernel does (row blocks from
-// registers, column blocks through shared memory), so codes and scales are bit-identical to
-// quantising the bf16 routed buffer. Blocks at or past the used rows (poff[E]) are skipped: no GEMM
-// reads them.
+// pad rows (row_token < 0) are zero. Each 32-row x 128-column tile is quantised exactly as
+// quant_rowcol_kernel does (row blocks from registers, column blocks through shared memory), so codes
+// and scales are bit-identical to quantising the bf16 routed buffer. Blocks at or past the used rows
+// (poff[E]) are skipped: no GEMM reads them.
+// One CTA per 32-row block walks the row's tiles and fetches the next tile's rows while it quantises
+// the current one (GQ_DY's dot products run across the tiles; for GQ_X one CTA per tile was measured
+// 15 % slower).
 enum { GQ_X = 0, GQ_DY = 1 };
+
+// Quantise the 32 x 128 tile held as v[4] (rows t/16 + 8i, 16-byte column word t%16) into the row and
+// column forms; the shared buffers are free on entry and on exit.
+__device__ __forceinline__ void quant_tile_32x128(const uint4 (&v)[4], uint4* tile, uint8_t* codes,
+                                                  int64_t row0, int64_t rb, int cb, int cols,
+                                                  int64_t rows, uint2* __restrict__ qr,
+                                                  uint8_t* __restrict__ sr, uint4* __restrict__ qc,
+                                                  uint8_t* __restrict__ sc) {
+  const int t = threadIdx.x;
+  const int c16 = t & 15;
+  const int64_t w16 = cols / 8;
+  const int kb = cols / 32;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) tile[((t >> 4) + 8 * i) * 16 + c16] = v[i];
+  // row blocks from registers: lanes 4j..4j+3 hold the 32 columns of one block of one row
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = (t >> 4) + 8 * i;
+    const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[2 * j] = bf16lo(u[j]);
+      f[2 * j + 1] = bf16hi(u[j]);
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(f[j]));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    uint8_t sb;
+    const float ir = exp2_exact(-block_exponent(m, &sb));
+    uint2 c;
+    c.x = cvt_e4m3x2(f[0] * ir, f[1] * ir) | ((uint32_t)cvt_e4m3x2(f[2] * ir, f[3] * ir) << 16);
+    c.y = cvt_e4m3x2(f[4] * ir, f[5] * ir) | ((uint32_t)cvt_e4m3x2(f[6] * ir, f[7] * ir) << 16);
+    if (!(m > 0.f)) c = make_uint2(0u, 0u);
+    qr[(row0 + r) * w16 + cb * 16 + c16] = c;
+    if ((t & 3) == 0) sr[tiled_sf_offset(row0 + r, (int64_t)cb * 4 + (c16 >> 2), kb)] = sb;
+  }
+  __syncthreads();
+  // column blocks: thread t owns column t of the tile (32 rows)
+  {
+    const __nv_bfloat16* tb = reinterpret_cast<const __nv_bfloat16*>(tile);
+    float f[kRcRows];
+    float amax = 0.f;
+#pragma unroll
+    for (int r = 0; r < kRcRows; ++r) {
+      f[r] = __bfloat162float(tb[r * kRcCols + t]);
+      amax = fmaxf(amax, fabsf(f[r]));
+    }
+    uint8_t sb;
+    const int e = block_exponent(amax, &sb);
+    const float inv = amax > 0.f ? exp2_exact(-e) : 0.f;
+    sc[tiled_sf_offset((int64_t)cb * kRcCols + t, rb, rows / 32)] = sb;
+#pragma unroll
+    for (int r = 0; r < kRcRows; r += 2) {
+      const uint32_t c2 = amax > 0.f ? cvt_e4m3x2(f[r] * inv, f[r + 1] * inv) : 0u;
+      codes[r * kRcCols + t] = (uint8_t)(c2 & 0xFFu);
+      codes[(r + 1) * kRcCols + t] = (uint8_t)(c2 >> 8);
+    }
+  }
+  __syncthreads();
+  const uint4* cw = reinterpret_cast<const uint4*>(codes);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int idx = t + kRcThreads * j;  // 16-byte word of the code tile: 8 per row
+    const int r = idx >> 3, c = idx & 7;
+    qc[((row0 + r) * cols + (int64_t)cb * kRcCols) / 16 + c] = cw[idx];
+  }
+  __syncthreads();  // the shared buffers are free again
+}
 
 template <int SRC>
 __global__ void __launch_bounds__(kRcThreads) gather_quant_kernel(
@@ -226,111 +299,82 @@ __global__ void __launch_bounds__(kRcThreads) gather_quant_kernel(
   __shared__ __align__(16) uint4 tile[kRcRows * kRcCols / 8];  // bf16 [32][128]
   __shared__ __align__(16) uint8_t codes[kRcRows * kRcCols];    // column-block codes [32][128]
   pdl_enter();  // wait for the previous kernel before any global access
-  const int64_t row0 = (int64_t)blockIdx.x * kRcRows;
+  const int ctiles = cols / kRcCols;
+  const int64_t rb = blockIdx.x;
+  const int64_t row0 = rb * kRcRows;
   if (row0 >= *poff_end) return;
   const int t = threadIdx.x;
   const int c16 = t & 15;        // this thread's 16-byte column word inside a tile
   const int64_t w16 = cols / 8;  // 16-byte words per row
-  const int ctiles = cols / kRcCols;
-  const int kb = cols / 32;
   // the four rows this thread loads: r = t/16 + 8i
   int64_t srow[4];
   int ent[4];
-  float g[4], dot[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = (t >> 4) + 8 * i;
-    const int n = row_token[row0 + r];
+    const int n = row_token[row0 + (t >> 4) + 8 * i];
     ent[i] = n;
     srow[i] = n >= 0 ? (int64_t)(n / k) : -1;
-    g[i] = (SRC == GQ_DY && n >= 0) ? gates[n] : 0.f;
-    dot[i] = 0.f;
   }
-  for (int cb = 0; cb < ctiles; ++cb) {
-    uint4 v[4];
+  if constexpr (SRC == GQ_X) {
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    uint4 vn[4];  // the next tile's words
+#pragma unroll
+    for (int i = 0; i < 4; ++i) vn[i] = srow[i] >= 0 ? tok[srow[i] * w16 + c16] : z4;
+    for (int cb = 0; cb < ctiles; ++cb) {
+      uint4 v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = vn[i];
+      if (cb + 1 < ctiles) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) vn[i] = srow[i] >= 0 ? tok[srow[i] * w16 + (cb + 1) * 16 + c16] : z4;
+      }
+      quant_tile_32x128(v, tile, codes, row0, rb, cb, cols, rows, qr, sr, qc, sc);
+    }
+  } else {
+    float g[4], dot[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int r = (t >> 4) + 8 * i;
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (srow[i] >= 0) w = tok[srow[i] * w16 + cb * 16 + c16];
-      if constexpr (SRC == GQ_DY) {
-        if (srow[i] >= 0) {
-          const uint4 yv = y[(row0 + r) * w16 + cb * 16 + c16];
-          const uint32_t du[4] = {w.x, w.y, w.z, w.w};
-          const uint32_t yu[4] = {yv.x, yv.y, yv.z, yv.w};
-          uint32_t o[4];
+      g[i] = ent[i] >= 0 ? gates[ent[i]] : 0.f;
+      dot[i] = 0.f;
+    }
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    uint4 dn[4], yn[4];  // the next tile's dout and y words
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float d0 = bf16lo(du[j]), d1 = bf16hi(du[j]);
-            dot[i] = fmaf(d0, bf16lo(yu[j]), dot[i]);
-            dot[i] = fmaf(d1, bf16hi(yu[j]), dot[i]);
-            o[j] = pack_bf16(g[i] * d0, g[i] * d1);
-          }
-          w = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int i = 0; i < 4; ++i) {
+      dn[i] = srow[i] >= 0 ? tok[srow[i] * w16 + c16] : z4;
+      yn[i] = srow[i] >= 0 ? y[(row0 + (t >> 4) + 8 * i) * w16 + c16] : z4;
+    }
+    for (int cb = 0; cb < ctiles; ++cb) {
+      uint4 dc[4], yc[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        dc[i] = dn[i];
+        yc[i] = yn[i];
+      }
+      if (cb + 1 < ctiles) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          dn[i] = srow[i] >= 0 ? tok[srow[i] * w16 + (cb + 1) * 16 + c16] : z4;
+          yn[i] = srow[i] >= 0 ? y[(row0 + (t >> 4) + 8 * i) * w16 + (cb + 1) * 16 + c16] : z4;
         }
       }
-      v[i] = w;
-    }
-    __syncthreads();  // the previous tile's shared buffers are free
+      uint4 v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) tile[((t >> 4) + 8 * i) * 16 + c16] = v[i];
-    // row blocks from registers: lanes 4j..4j+3 hold the 32 columns of one block of one row
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t du[4] = {dc[i].x, dc[i].y, dc[i].z, dc[i].w};
+        const uint32_t yu[4] = {yc[i].x, yc[i].y, yc[i].z, yc[i].w};
+        uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = (t >> 4) + 8 * i;
-      const uint32_t u[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      float f[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        f[2 * j] = bf16lo(u[j]);
-        f[2 * j + 1] = bf16hi(u[j]);
+        for (int j = 0; j < 4; ++j) {
+          const float d0 = bf16lo(du[j]), d1 = bf16hi(du[j]);
+          dot[i] = fmaf(d0, bf16lo(yu[j]), dot[i]);
+          dot[i] = fmaf(d1, bf16hi(yu[j]), dot[i]);
+          o[j] = pack_bf16(g[i] * d0, g[i] * d1);
+        }
+        v[i] = make_uint4(o[0], o[1], o[2], o[3]);
       }
-      float m = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(f[j]));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      uint8_t sb;
-      const float ir = exp2_exact(-block_exponent(m, &sb));
-      uint2 c;
-      c.x = cvt_e4m3x2(f[0] * ir, f[1] * ir) | ((uint32_t)cvt_e4m3x2(f[2] * ir, f[3] * ir) << 16);
-      c.y = cvt_e4m3x2(f[4] * ir, f[5] * ir) | ((uint32_t)cvt_e4m3x2(f[6] * ir, f[7] * ir) << 16);
-      if (!(m > 0.f)) c = make_uint2(0u, 0u);
-      qr[(row0 + r) * w16 + cb * 16 + c16] = c;
-      if ((t & 3) == 0) sr[tiled_sf_offset(row0 + r, (int64_t)cb * 4 + (c16 >> 2), kb)] = sb;
+      quant_tile_32x128(v, tile, codes, row0, rb, cb, cols, rows, qr, sr, qc, sc);
     }
-    __syncthreads();
-    // column blocks: thread t owns column t of the tile (32 rows)
-    {
-      const __nv_bfloat16* tb = reinterpret_cast<const __nv_bfloat16*>(tile);
-      float f[kRcRows];
-      float amax = 0.f;
-#pragma unroll
-      for (int r = 0; r < kRcRows; ++r) {
-        f[r] = __bfloat162float(tb[r * kRcCols + t]);
-        amax = fmaxf(amax, fabsf(f[r]));
-      }
-      uint8_t sb;
-      const int e = block_exponent(amax, &sb);
-      const float inv = amax > 0.f ? exp2_exact(-e) : 0.f;
-      sc[tiled_sf_offset((int64_t)cb * kRcCols + t, blockIdx.x, rows / 32)] = sb;
-#pragma unroll
-      for (int r = 0; r < kRcRows; r += 2) {
-        const uint32_t c2 = amax > 0.f ? cvt_e4m3x2(f[r] * inv, f[r + 1] * inv) : 0u;
-        codes[r * kRcCols + t] = (uint8_t)(c2 & 0xFFu);
-        codes[(r + 1) * kRcCols + t] = (uint8_t)(c2 >> 8);
-      }
-    }
-    __syncthreads();
-    const uint4* cw = reinterpret_cast<const uint4*>(codes);
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int idx = t + kRcThreads * j;  // 16-byte word of the code tile: 8 per row
-      const int r = idx >> 3, c = idx & 7;
-      qc[((row0 + r) * cols + (int64_t)cb * kRcCols) / 16 + c] = cw[idx];
-    }
-  }
-  if constexpr (SRC == GQ_DY) {
     // the 16 threads that share a row hold its partial dot products over their columns
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

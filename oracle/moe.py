@@ -359,6 +359,50 @@ def layer_bwd(dout, x, W13, W2, idx, gates, saved, W_r=None, renorm=True, logits
 
 
 # ----------------------------------------------------------------------------------------------
+# Expert parallelism across G ranks (row-wise: each routed row lands in the buffer of the rank that
+# owns its expert -- unite.ai, "Parallelismo, precisione e tecniche di memoria"). Rank h owns experts
+# [h*E/G, (h+1)*E/G). Inside an owner's group for expert e the rows come source rank by source rank,
+# each source's rows in its own token order; groups start on ALIGN-row boundaries of the owner's
+# buffer, experts in ascending order.
+# ----------------------------------------------------------------------------------------------
+
+def ep_layout(all_counts: np.ndarray, world: int, align: int = ALIGN) -> dict:
+    """From every rank's per-expert counts all_counts [G, E]: per owner h its local counts and padded
+    group starts, and base[g, e] = row in the owner's buffer of source g's first entry for expert e."""
+    G, E = all_counts.shape
+    EL = E // world
+    total = all_counts.sum(axis=0)
+    base = np.zeros((G, E), dtype=np.int64)
+    counts_loc = np.zeros((world, EL), dtype=np.int64)
+    poff_loc = np.zeros((world, EL + 1), dtype=np.int64)
+    for h in range(world):
+        start = 0
+        for el in range(EL):
+            e = h * EL + el
+            counts_loc[h, el] = total[e]
+            poff_loc[h, el] = start
+            before = 0
+            for g in range(G):
+                base[g, e] = start + before
+                before += all_counts[g, e]
+            start += -(-int(total[e]) // align) * align
+        poff_loc[h, EL] = start
+    return dict(base=base, counts_loc=counts_loc, poff_loc=poff_loc)
+
+
+def ep_dst_rows(idx_g: np.ndarray, base_g: np.ndarray, E: int) -> np.ndarray:
+    """Row in the owner's buffer of each entry (t, j) of one source rank: the source's base for the
+    expert plus the entry's rank among the source's own entries for that expert (token order)."""
+    flat = idx_g.reshape(-1)
+    seen = np.zeros(E, dtype=np.int64)
+    rows = np.empty(flat.size, dtype=np.int64)
+    for n, e in enumerate(flat):
+        rows[n] = base_g[e] + seen[e]
+        seen[e] += 1
+    return rows
+
+
+# ----------------------------------------------------------------------------------------------
 # Layer, per-token direct form (no grouping; used to pin the grouped form and for sampled checks)
 # ----------------------------------------------------------------------------------------------
 

@@ -639,3 +639,39 @@ def test_token_expert_outputs_sum_to_the_output_and_give_the_gate_gradients():
         ys = O.token_expert_outputs(t, x, W13, W2, idx)
         np.testing.assert_allclose(g[t] @ ys, out[t], rtol=1e-12, atol=1e-13)
         np.testing.assert_allclose(ys @ dout[t], gr["dgates"][t], rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------------------------------------------------
+# expert parallelism layout
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("world,E,T,k", [(1, 8, 50, 2), (2, 8, 40, 3), (4, 16, 33, 4), (8, 32, 20, 2)])
+def test_ep_layout_is_a_source_major_stable_placement(world, E, T, k):
+    """Brute force: building each owner's buffer by appending, expert by expert, every source's entries
+    in token order (then padding the group to 32 rows) gives exactly the rows the layout assigns; every
+    owner row below its end is used once or is a pad row; with one rank it is the single-GPU
+    metadata."""
+    rng = np.random.default_rng(world * 100 + E)
+    idx = [np.stack([rng.permutation(E)[:k] for _ in range(T)]) for _ in range(world)]
+    all_counts = np.stack([np.bincount(i.reshape(-1), minlength=E) for i in idx])
+    L = O.ep_layout(all_counts, world)
+    EL = E // world
+    for h in range(world):
+        buf = []  # (source, entry) per row, None for pad rows
+        for el in range(EL):
+            e = h * EL + el
+            assert len(buf) == L["poff_loc"][h, el]
+            for g in range(world):
+                buf += [(g, n) for n, ee in enumerate(idx[g].reshape(-1)) if ee == e]
+            while len(buf) % 32:
+                buf.append(None)
+        assert len(buf) == L["poff_loc"][h, EL]
+        for g in range(world):
+            rows = O.ep_dst_rows(idx[g], L["base"][g], E)
+            for n, ee in enumerate(idx[g].reshape(-1)):
+                if ee // EL == h:
+                    assert buf[rows[n]] == (g, n)
+    if world == 1:
+        meta = O.route_metadata(idx[0], E)
+        assert np.array_equal(O.ep_dst_rows(idx[0], L["base"][0], E), meta["prow"])
+        assert np.array_equal(L["poff_loc"][0], meta["poff"])
