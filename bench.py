@@ -60,7 +60,11 @@ def load_peaks():
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, taken from a committed ncu
 # capture of the kernel as it is now; an entry is removed whenever its kernel changes, so a kernel or
 # workload not listed reports null.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    # e128_bf16, one-pass capture of the full-size launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    ("e128_bf16", "gemm_wgrad1"): 286.05e6 + 1.01e9,
+    ("e128_bf16", "gemm_fwd1_swiglu"): 1.27e9 + 199.85e6,
+}
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
 
 
@@ -641,6 +645,20 @@ def main():
                 "algorithmic_bytes": b, "flops": f, "ms": dom_ms,
                 "peak_source": f"{peaks['source']} bf16_tflops (burst) x {ratio} ({w.dtype})"}
 
+    # activation memory kept between the forward and the backward (the layer's own buffers)
+    nb = lambda t: t.numel() * t.element_size()
+    if layer.mx:
+        kept = sum(nb(layer.qa_t[n]) for n in ("xtq", "xts", "atq", "ats")) + nb(layer.h13) + nb(layer.y)
+        R, es = layer.R, 2
+        kept_bf16 = R * (2 * w.d + 2 * w.F + w.F + w.d) * es  # x_perm, h13, a, y of the bf16 layer
+        act_mem = {"kept_between_passes_bytes": kept, "bf16_layer_same_shapes_bytes": kept_bf16,
+                   "ratio": kept / kept_bf16,
+                   "note": "MXFP8 keeps the column forms of x and a (codes + scales), h13 and y"}
+    else:
+        # with activation recompute neither h13 nor a is kept (a is scratch the backward rewrites)
+        kept = nb(layer.x_perm) + nb(layer.y) + (0 if layer.recompute else nb(layer.h13) + nb(layer.a))
+        act_mem = {"kept_between_passes_bytes": kept}
+
     wq = None
     if layer.mx:  # weights are quantised once per update: timed on their own, not in the step
         q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -805,6 +823,7 @@ def main():
             "gpu_launches": launches,
             "clocks": clk,
             "peak_mem_gb": round(peak_mem_gb, 2),
+            "activation_memory": act_mem,
         }
         if rc is not None:
             line["recompute"] = rc
