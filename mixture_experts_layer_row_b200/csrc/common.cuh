@@ -23,6 +23,24 @@ __device__ __forceinline__ void set_error(uint32_t* flag, uint32_t bits) {
   if (flag) atomicOr(flag, bits);
 }
 
+// Division by a loop-invariant divisor d >= 1 through a precomputed multiplier (T. Granlund and
+// P. Montgomery, "Division by invariant integers using multiplication", 1994, the round-up variant):
+// with l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1, floor(n / d) = (mulhi(m, n) + n) >> l
+// for every 0 <= n < 2^32 (the sum taken in 64 bits).
+struct FastDiv {
+  uint32_t m, l;
+  int d;
+  __host__ __device__ FastDiv() : m(1), l(0), d(1) {}
+  __host__ __device__ explicit FastDiv(int div) : d(div) {
+    l = 0;
+    while ((1ull << l) < (uint64_t)div) ++l;
+    m = (uint32_t)((((1ull << 32) * ((1ull << l) - (uint64_t)div)) / (uint64_t)div) + 1);
+  }
+  __device__ __forceinline__ int div(int n) const {
+    return (int)(((uint64_t)__umulhi((uint32_t)n, m) + (uint32_t)n) >> l);
+  }
+};
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -301,9 +319,11 @@ __device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
   return r;
 }
 // Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address.
+// The arrive keeps the default CTA-scope release: the barriers that cross the pair only hand over
+// tensor memory, whose accesses the tcgen05 fences on either side of the arrive / wait order. A
+// cluster-scope release would add a fence at that scope to every handover.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 // try_wait with acquire at cluster scope (for barriers that the peer CTA arrives on).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {

@@ -158,9 +158,20 @@ __device__ __forceinline__ int prefix_m_tiles(const int* prefix, int e, int n_ti
   return (prefix[e + 1] - prefix[e]) / n_tiles;
 }
 
+// The device tile schedule as every role of a CTA sees it. GROUP_M: prefix[e] = first tile of group
+// e (inclusive scan of its tile counts). GROUP_K: prefix[e] = poff[e] (the groups' contraction row
+// ranges, staged in shared memory) and a fixed m_tiles x n_tiles block of tiles per group, whose
+// index is split by multiply-shift division.
+struct Sched {
+  const int* prefix;
+  int n_tiles, m_tiles_fixed, total;
+  FastDiv per_group, per_row;  // GROUP_K: divisors m_tiles_fixed * n_tiles and n_tiles
+};
+
 template <class C, int EPI, int MODE>
-__device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const int* prefix,
-                                          int n_tiles, int m_tiles_fixed, TileInfo& ti) {
+__device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const Sched& sch, TileInfo& ti) {
+  const int* prefix = sch.prefix;
+  const int n_tiles = sch.n_tiles;
   if constexpr (MODE == GROUP_M) {
     int e = 0;
     if (p.counts) {
@@ -184,15 +195,15 @@ __device__ __forceinline__ void tile_info(int tile, const GemmParams& p, const i
       ti.hi = p.M;
     }
   } else {
-    const int per = m_tiles_fixed * n_tiles;
-    const int e = tile / per;
-    const int local = tile - e * per;
+    const int e = sch.per_group.div(tile);
+    const int local = tile - e * sch.per_group.d;
+    const int mi = sch.per_row.div(local);
     ti.e = e;
-    ti.m0 = (local / n_tiles) * C::TILE_M;
-    ti.n0 = (local % n_tiles) * C::TILE_N;
+    ti.m0 = mi * C::TILE_M;
+    ti.n0 = (local - mi * n_tiles) * C::TILE_N;
     if (p.counts) {
-      ti.lo = p.poff[e];
-      ti.hi = p.poff[e + 1];
+      ti.lo = prefix[e];
+      ti.hi = prefix[e + 1];
     } else if (p.ksplit) {
       ti.lo = e * p.ksplit;
       ti.hi = min(p.K, ti.lo + p.ksplit);
@@ -394,6 +405,17 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     n_tiles = (p.N + BN - 1) / BN;
     m_tiles_fixed = (p.M + C::TILE_M - 1) / C::TILE_M;
     total = k_groups(p) * m_tiles_fixed * n_tiles;
+    if (p.counts)
+      for (int e = threadIdx.x; e <= p.E; e += blockDim.x) prefix[e] = p.poff[e];
+  }
+  Sched sch;
+  sch.prefix = prefix;
+  sch.n_tiles = n_tiles;
+  sch.m_tiles_fixed = m_tiles_fixed;
+  sch.total = total;
+  if constexpr (MODE == GROUP_K) {
+    sch.per_group = FastDiv(max(1, m_tiles_fixed * n_tiles));
+    sch.per_row = FastDiv(max(1, n_tiles));
   }
 
   tc_fence_before();
@@ -415,10 +437,10 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       int it = 0;
       bool ok = true;
       TileInfo nxt;  // the next tile's entry is fetched a tile ahead
-      if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, prefix, n_tiles, m_tiles_fixed, nxt);
+      if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, sch, nxt);
       for (int tile = tile0; tile < total && ok; tile += tstep) {
         const TileInfo ti = nxt;
-        if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
+        if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, sch, nxt);
         const int nst = num_kstages<C, MODE>(ti, p);
         // tail tile (<= BM rows left): 64 rows of A per CTA for an M = 128 pair MMA
         const bool half = ti_half<PAIR, MODE>(ti, p);
@@ -476,10 +498,10 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       int it = 0;
       bool ok = true;
       TileInfo nxt;  // the next tile's entry is fetched a tile ahead
-      if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, prefix, n_tiles, m_tiles_fixed, nxt);
+      if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, sch, nxt);
       for (int tile = tile0; tile < total && ok; tile += tstep) {
         const TileInfo ti = nxt;
-        if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
+        if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, sch, nxt);
         const int nst = num_kstages<C, MODE>(ti, p);
         for (int ks = 0; ks < nst; ++ks, ++it) {
           const int s = it % C::STAGES;
@@ -606,10 +628,10 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       bool ok = true;
       bool issued = false;
       TileInfo nxt;  // the next tile's entry is fetched a tile ahead
-      if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, prefix, n_tiles, m_tiles_fixed, nxt);
+      if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, sch, nxt);
       for (int tile = tile0; tile < total && ok; tile += tstep, ++local) {
         const TileInfo ti = nxt;
-        if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
+        if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, sch, nxt);
         const int nst = num_kstages<C, MODE>(ti, p);
         const uint32_t idesc = ti_half<PAIR, MODE>(ti, p) ? C::IDESC_HALF : C::IDESC;
         const int buf = local % C::NACC;
@@ -690,10 +712,10 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     int nb = 0;                           // next staging box (round robin)
     int local = 0;
     TileInfo nxt;  // the next tile's entry is fetched a tile ahead
-    if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, prefix, n_tiles, m_tiles_fixed, nxt);
+    if (tile0 < total) tile_info<C, EPI, MODE>(tile0, p, sch, nxt);
     for (int tile = tile0; tile < total; tile += tstep, ++local) {
       const TileInfo ti = nxt;
-      if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, prefix, n_tiles, m_tiles_fixed, nxt);
+      if (tile + tstep < total) tile_info<C, EPI, MODE>(tile + tstep, p, sch, nxt);
       const int nst = num_kstages<C, MODE>(ti, p);
       const int buf = local % C::NACC;
       int ok = 1;
