@@ -61,9 +61,10 @@ def load_peaks():
 # capture of the kernel as it is now; an entry is removed whenever its kernel changes, so a kernel or
 # workload not listed reports null.
 MEASURED_TRAFFIC = {
-    # e128_bf16, one-pass capture of the full-size launch (dram__bytes_read.sum + dram__bytes_write.sum)
-    ("e128_bf16", "gemm_wgrad1"): 286.05e6 + 1.01e9,
-    ("e128_bf16", "gemm_fwd1_swiglu"): 1.27e9 + 199.85e6,
+    # e128_bf16, ncu capture of the full-size launch of the current kernel
+    # (dram__bytes_read.sum + dram__bytes_write.sum)
+    ("e128_bf16", "gemm_wgrad1"): 286.04e6 + 1.0147e9,
+    ("e128_bf16", "gemm_fwd1_swiglu"): 1.2758e9 + 202.77e6,
 }
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
 
