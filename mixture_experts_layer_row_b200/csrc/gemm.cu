@@ -1173,9 +1173,11 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
 // Dispatch a GEMM request to its compiled variant. The caller (api.cu) has validated shapes.
 // The ragged-row bf16 / tf32 GEMMs with light epilogues (fwd1 + SwiGLU, fwd2, dgrad1) run on CTA
 // pairs: 256 x 256 tiles with cta_group::2 MMAs, so each weight tile is fetched once per 256 routed
-// rows and each SM holds half of B. The SwiGLU backward and the wgrads are bound by their epilogues,
-// which a pair would couple (the MMA then waits for the slower CTA of the two): they run on single
-// CTAs with 128-row tiles, as do the router GEMM and MXFP8.
+// rows and each SM holds half of B. The bf16 expert wgrads run on pairs as well: each SM then loads
+// half of the other operand's 256 columns, and the accumulator hand-back to the leader is one
+// CTA-scope arrive per epilogue warp. The SwiGLU backward (whose epilogue a pair would couple: the
+// MMA then waits for the slower CTA of the two), the router GEMMs and MXFP8 run on single CTAs with
+// 128-row tiles.
 int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmOperand& B,
                 const GemmParams& p, cudaStream_t s) {
 #define MOE_GEMM_CASES(ES_)                                                                        \
@@ -1193,6 +1195,8 @@ int launch_gemm(GemmKind kind, int es, int bn, const GemmOperand& A, const GemmO
       if (bn == 256) return launch_impl<ES_, false, true, 256, EPI_STORE, GROUP_M, true>(A, B, p, s);  \
       return launch_impl<ES_, false, true, 128, EPI_STORE, GROUP_M, false>(A, B, p, s);            \
     case GK_WGRAD:                                                                                 \
+      if (bn == 256 && ES_ == 2 && p.counts) /* bf16 expert wgrads: CTA pairs */                   \
+        return launch_impl<ES_, true, true, 256, EPI_STORE, GROUP_K, ES_ == 2>(A, B, p, s);        \
       if (bn == 256) return launch_impl<ES_, true, true, 256, EPI_STORE, GROUP_K, false>(A, B, p, s); \
       return launch_impl<ES_, true, true, 128, EPI_STORE, GROUP_K, false>(A, B, p, s);             \
     case GK_ROUTER:                                                                                \
