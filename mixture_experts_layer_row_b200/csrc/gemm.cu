@@ -77,12 +77,15 @@ struct Cfg {
   static_assert(!epi_quant(EPI) || (MX && !PAIR), "quantising epilogues are MXFP8-only");
   // staging boxes per epilogue warp: SwiGLU forward h13 gate + up + a (quantising: gate + up; a's codes
   // go straight to global memory); SwiGLU backward dh13 gate + up (quantising: none, dh13's codes go
-  // straight to global memory); plain stores round robin over NBUF boxes
+  // straight to global memory); plain stores round robin over NBUF boxes. With one accumulator the
+  // MMA waits for the epilogue: the short-contraction wgrad tiles take two boxes (the epilogue hands
+  // the accumulator back sooner) at the price of a pipeline stage; long-contraction tiles keep the
+  // deeper ring and one box.
   static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3
                               : (EPI == EPI_SWIGLU_FWD_Q) ? 2
                               : (EPI == EPI_SWIGLU_BWD_Q) ? 0
                               : (EPI == EPI_SWIGLU_BWD) ? 2
-                              : (NACC == 1 ? 1 : 2);
+                              : (NACC == 1 ? (MODE == GROUP_K ? 2 : 1) : 2);
   static constexpr int STAGING_BYTES = 4 * NBUF * 4096;
   // MXFP8: per stage, one 512-byte scale chunk per 128 rows of A and of B (TMEM: 4 columns each)
   static constexpr int SF_BYTES = MX ? 512 + (BN / 128) * 512 : 0;
