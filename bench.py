@@ -677,8 +677,9 @@ def main():
     # end to end through the public layer API: host inputs in, host results out, every step. The
     # loop is the one a training job runs: step i+1's inputs are copied host -> device on one copy
     # stream while step i computes (two device input buffers), and step i's out / dx are read back
-    # on another copy stream while the next step's work proceeds; the layer's own buffers are only
-    # rewritten after their read-back has finished.
+    # on another copy stream while the next step's work proceeds. out and dx alternate between two
+    # device buffers (the layer API writes into the caller's), so a step never waits for the
+    # previous step's read-back; a buffer is only rewritten after its own read-back has finished.
     e2e = None
     if not args.no_e2e:
         hx = inp["x"].cpu().pin_memory()
@@ -689,17 +690,19 @@ def main():
         bd = [torch.empty_like(inp["dout"]) for _ in range(2)]
         bi = [torch.empty_like(inp["idx"]) for _ in range(2)] if not learned else [None, None]
         bg = [torch.empty_like(inp["gates"]) for _ in range(2)] if not learned else [None, None]
-        ho = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
-        hdx = torch.empty(layer.dx.shape, dtype=layer.dx.dtype).pin_memory()
+        bo = [torch.empty_like(layer.out) for _ in range(2)]
+        bdx = [torch.empty_like(layer.dx) for _ in range(2)]
+        ho = [torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory() for _ in range(2)]
+        hdx = [torch.empty(layer.dx.shape, dtype=layer.dx.dtype).pin_memory() for _ in range(2)]
         h2d = hx.numel() * hx.element_size() + hd.numel() * hd.element_size()
         if not learned:
             h2d += hi.numel() * 4 + hg.numel() * 4
-        d2h = ho.numel() * ho.element_size() + hdx.numel() * hdx.element_size()
+        d2h = ho[0].numel() * ho[0].element_size() + hdx[0].numel() * hdx[0].element_size()
         comp = torch.cuda.current_stream()
         up, down = torch.cuda.Stream(), torch.cuda.Stream()
         ev = lambda: torch.cuda.Event()
         loaded, consumed = [ev(), ev()], [ev(), ev()]
-        out_read, dx_read, fwd_done, bwd_done = ev(), ev(), ev(), ev()
+        out_read, dx_read, fwd_done, bwd_done = [ev(), ev()], [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
         def upload(j):
             with torch.cuda.stream(up):
@@ -718,22 +721,24 @@ def main():
                 comp.wait_event(loaded[j])
                 if i + 1 < n:
                     upload(1 - j)
-                comp.wait_event(out_read)  # the previous step's out has been read back
-                layer.forward(bx[j], bias=inp["bias"], idx=bi[j], gates=bg[j])
-                fwd_done.record(comp)
+                comp.wait_event(out_read[j])  # bo[j]'s read-back (two steps ago) has finished
+                layer.forward(bx[j], bias=inp["bias"], idx=bi[j], gates=bg[j], out=bo[j])
+                fwd_done[j].record(comp)
                 with torch.cuda.stream(down):
-                    down.wait_event(fwd_done)
-                    ho.copy_(layer.out, non_blocking=True)
-                    out_read.record(down)
-                comp.wait_event(dx_read)
-                layer.backward(bd[j])
+                    down.wait_event(fwd_done[j])
+                    ho[j].copy_(bo[j], non_blocking=True)
+                    out_read[j].record(down)
+                comp.wait_event(dx_read[j])
+                layer.backward(bd[j], dx=bdx[j])
                 consumed[j].record(comp)
-                bwd_done.record(comp)
+                bwd_done[j].record(comp)
                 with torch.cuda.stream(down):
-                    down.wait_event(bwd_done)
-                    hdx.copy_(layer.dx, non_blocking=True)
-                    dx_read.record(down)
-            comp.wait_event(dx_read)  # the timed region ends with the last result on the host
+                    down.wait_event(bwd_done[j])
+                    hdx[j].copy_(bdx[j], non_blocking=True)
+                    dx_read[j].record(down)
+            for j in range(2):  # the timed region ends with every result on the host
+                comp.wait_event(out_read[j])
+                comp.wait_event(dx_read[j])
 
         e2e_run(args.warmup)
         torch.cuda.synchronize()
@@ -747,9 +752,10 @@ def main():
         e2e = {"value": world * w.T / (ems / args.steps / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": ems / args.steps,
-               "api": "MoELayer.forward/backward -> moe_layer_fwd/bwd; copies on two streams overlap "
-                      "the neighbouring steps' compute"}
-        assert torch.equal(ho.cuda(), ref[0]) and torch.equal(hdx.cuda(), ref[1])
+               "api": "MoELayer.forward/backward -> moe_layer_fwd/bwd into alternating out / dx "
+                      "buffers; copies on two streams overlap the neighbouring steps' compute"}
+        jl = (args.steps - 1) % 2
+        assert torch.equal(ho[jl].cuda(), ref[0]) and torch.equal(hdx[jl].cuda(), ref[1])
 
     # activation recompute against stored activations, both through the public layer API on the
     # same device-resident inputs, timed in alternation (so clock and power drift hit both alike),

@@ -107,31 +107,45 @@ class MoELayer:
         """Refresh the MXFP8 weight copies (after every weight update)."""
         L.quantize_weights_mxfp8(self.cfg, self._w, self.qw, stream)
 
-    def forward(self, x, bias=None, idx=None, gates=None, stream=None):
+    def _result(self, t, own):
+        """The caller's output buffer (any [T, d] contiguous tensor of the activation dtype on this
+        layer's device), or the layer's own."""
+        if t is None:
+            return own
+        if tuple(t.shape) != (self.T, self.d) or t.dtype != self.act or not t.is_contiguous() \
+                or t.device != own.device:
+            raise ValueError("output buffer shape/dtype/layout/device mismatch")
+        return t
+
+    def forward(self, x, bias=None, idx=None, gates=None, stream=None, out=None):
         """out = layer(x). With a learned router, routing comes from x W_r^T (+ bias); otherwise
-        `idx` [T,k] int32 and `gates` [T,k] fp32 are copied in as the routing."""
+        `idx` [T,k] int32 and `gates` [T,k] fp32 are copied in as the routing. `out`: where to write
+        the result (default: the layer's own buffer), e.g. to let a host copy of the previous step's
+        result run on while this step computes."""
         if self._w is None:
             raise RuntimeError("set_weights first")
+        out = self._result(out, self.out)
         if not self.learned_router:
             self.idx.copy_(idx)
             self.gates.copy_(gates)
         self._x = x
         if self.mx:
-            L.layer_fwd_mxfp8(self.cfg, self._w, self.qw, x, bias, self.out, self.saved, self.qa,
+            L.layer_fwd_mxfp8(self.cfg, self._w, self.qw, x, bias, out, self.saved, self.qa,
                               self.ws, stream)
         else:
-            L.layer_fwd(self.cfg, self._w, x, bias, self.out, self.saved, self.ws, stream)
-        return self.out
+            L.layer_fwd(self.cfg, self._w, x, bias, out, self.saved, self.ws, stream)
+        return out
 
-    def backward(self, dout, stream=None):
-        """Fills dx, dW13, dW2 (and dW_r, dgates)."""
+    def backward(self, dout, stream=None, dx=None):
+        """Fills dx (the layer's own buffer, or `dx`), dW13, dW2 (and dW_r, dgates)."""
+        dx = self._result(dx, self.dx)
         if self.mx:
-            L.layer_bwd_mxfp8(self.cfg, self._w, self.qw, self.saved, self.qa, self._x, dout, self.dx,
+            L.layer_bwd_mxfp8(self.cfg, self._w, self.qw, self.saved, self.qa, self._x, dout, dx,
                               self.grads, self.ws, stream)
         else:
-            L.layer_bwd(self.cfg, self._w, self.saved, self._x, dout, self.dx, self.grads, self.ws,
+            L.layer_bwd(self.cfg, self._w, self.saved, self._x, dout, dx, self.grads, self.ws,
                         stream)
-        return self.dx
+        return dx
 
     def error_flags(self, stream=None) -> int:
         return L.get_error(self.ws, stream)

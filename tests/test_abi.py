@@ -115,3 +115,23 @@ def test_host_validation_before_any_launch(L):
     assert L.lib.moe_grouped_gemm_mxfp8(ctypes.byref(mx), 1, fake, fake, fake, fake, fake, None, None,
                                         fake, fake, fake, 10 ** 9, None) == -2
     assert L.lib.moe_layer_fwd(c, None, fake, None, fake, None, fake, 10 ** 9, None) == -1
+
+
+def test_layer_output_buffers_checked_on_host():
+    """MoELayer.forward(out=) / backward(dx=) reject a buffer of the wrong shape, dtype or layout
+    before anything is enqueued (host buffers: no GPU needed)."""
+    import torch
+    from mixture_experts_layer_row_b200 import MoELayer
+    T, d, F, E, k = 64, 128, 128, 8, 2
+    layer = MoELayer(T, d, F, E, k, dtype="bf16", device="cpu", learned_router=False)
+    layer.set_weights(torch.zeros((E, 2 * F, d), dtype=torch.bfloat16),
+                      torch.zeros((E, d, F), dtype=torch.bfloat16))
+    x = torch.zeros((T, d), dtype=torch.bfloat16)
+    kw = {"idx": torch.zeros((T, k), dtype=torch.int32), "gates": torch.zeros((T, k))}
+    bad = [torch.zeros((T, d // 2), dtype=torch.bfloat16), torch.zeros((T, d), dtype=torch.float32),
+           torch.zeros((d, T), dtype=torch.bfloat16).t()]
+    for b in bad:
+        with pytest.raises(ValueError):
+            layer.forward(x, out=b, **kw)
+        with pytest.raises(ValueError):
+            layer.backward(x, dx=b)

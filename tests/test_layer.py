@@ -231,6 +231,28 @@ def test_layer_twice_is_deterministic():
     assert torch.equal(o1, o2) and torch.equal(dx1, l2.dx) and torch.equal(dw1, l2.dW13)
 
 
+def test_layer_caller_output_buffers():
+    """forward(out=...) / backward(dx=...) write the same bits into the caller's buffers as into the
+    layer's own, and leave the layer's own untouched."""
+    from mixture_experts_layer_row_b200 import MoELayer
+    w = SMALL["e32_uniform_small"]
+    inp = make_inputs(w, seed=5, device="cuda")
+    layer = MoELayer(w.T, w.d, w.F, w.E, w.k, dtype=w.dtype, learned_router=w.routing == "learned")
+    layer.set_weights(inp["W13"], inp["W2"], inp["W_r"] if w.routing == "learned" else None)
+    kw = {} if w.routing == "learned" else {"idx": inp["idx"], "gates": inp["gates"]}
+    o_ref = layer.forward(inp["x"], bias=inp["bias"], **kw).clone()
+    dx_ref = layer.backward(inp["dout"]).clone()
+    layer.out.zero_()
+    layer.dx.zero_()
+    out, dx = torch.full_like(o_ref, 7.0), torch.full_like(dx_ref, 7.0)
+    assert layer.forward(inp["x"], bias=inp["bias"], out=out, **kw) is out
+    assert layer.backward(inp["dout"], dx=dx) is dx
+    torch.cuda.synchronize()
+    assert torch.equal(out, o_ref) and torch.equal(dx, dx_ref)
+    assert not layer.out.any() and not layer.dx.any()
+    assert layer.error_flags() == 0
+
+
 # ------------------------------------------------------------------------------------------------
 # MXFP8 layer. Three comparisons:
 #  - against the oracle with the same quantisation (OCP MX along every GEMM's contraction axis, bf16
