@@ -58,12 +58,16 @@ struct Cfg {
   static constexpr int TILE_N = BN;                  // accumulator columns per tile
   static constexpr int BN_CTA = PAIR ? BN / 2 : BN;  // rows of B (along N) held by one CTA
   static constexpr int EPR = 128 / ES;       // elements per 128-byte smem row
-  static constexpr int BK = EPR;             // K elements per pipeline stage
+  // K elements per pipeline stage: one 128-byte row, except for the bf16 wgrads on CTA pairs (both
+  // operands MN-major), whose short contractions take 128 rows per stage. Each stage costs the MMA
+  // thread a barrier wait and a commit that the tensor pipe does not overlap, and a pair's halved
+  // B share leaves room for three such stages.
+  static constexpr int BK = (ES == 2 && MODE == GROUP_K && PAIR) ? 2 * EPR : EPR;
   static constexpr int UK = 32 / ES;         // K per tcgen05.mma (32 bytes)
   static constexpr int KSTEPS = BK / UK;     // MMAs per full stage (4)
   static constexpr int CHUNKS = BK / 32;     // 32-row K chunks per stage (MN-major operands)
-  static constexpr int A_BYTES = BM * 128;
-  static constexpr int B_BYTES = BN_CTA * 128;
+  static constexpr int A_BYTES = BM * BK * ES;
+  static constexpr int B_BYTES = BN_CTA * BK * ES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   // output staging: each epilogue warp owns NBUF swizzled 32-row x 128-byte boxes
   static constexpr bool MX = (ES == 1);      // MXFP8 block-scaled (E4M3 operands, UE8M0 scales)
@@ -448,7 +452,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
         // tail tile (<= BM rows left): 64 rows of A per CTA for an M = 128 pair MMA
         const bool half = ti_half<PAIR, MODE>(ti, p);
         const int cta_rows = half ? C::HALF_M : BM;
-        const uint32_t a_bytes = (uint32_t)cta_rows * 128;
+        const uint32_t a_bytes = (uint32_t)cta_rows * C::BK * ES;
         const bool a0 = ti.m0 < ti_rows<MODE>(ti, p), a1 = ti.m0 + cta_rows < ti_rows<MODE>(ti, p);
         const bool mine = rank == 0 ? a0 : a1;
         const uint32_t tx = (a0 ? a_bytes : 0) + (a1 ? a_bytes : 0) + 2 * C::B_BYTES;
