@@ -40,8 +40,6 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128;
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
 
 constexpr int kSmemBudget = 232448;  // 227 KB of opt-in shared memory per CTA
 constexpr int kCtrlBytes = 2048;      // mbarriers, TMEM slot, abort word, tile prefix [<=257 ints]
@@ -72,7 +70,12 @@ struct Cfg {
   // output staging: each epilogue warp owns NBUF swizzled 32-row x 128-byte boxes
   static constexpr bool MX = (ES == 1);      // MXFP8 block-scaled (E4M3 operands, UE8M0 scales)
   static_assert(!(PAIR && MX), "block-scaled MMAs run on single CTAs");
-  static constexpr int THREADS = kThreads;
+  // epilogue warps: four (one per TMEM lane quadrant), or eight (two per quadrant, each taking half
+  // of the accumulator columns) where the MMA waits for the epilogue on every tile: MXFP8 wgrad tiles,
+  // with one accumulator and a contraction of a few stages. The stores a warp keeps in flight bound
+  // how fast it drains the accumulator.
+  static constexpr int EPW = (ES == 1 && BN == 256 && MODE == GROUP_K && !PAIR && EPI == EPI_STORE) ? 8 : 4;
+  static constexpr int THREADS = 64 + 32 * EPW;  // producer, MMA issuer, epilogue
   static constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : (MX ? 2 : ES);  // output element size
   static constexpr int OEPR = 128 / OES;     // output columns per staged box
   // accumulators in TMEM: two (the epilogue drains one while the MMA fills the other), or one for
@@ -90,7 +93,7 @@ struct Cfg {
                               : (EPI == EPI_SWIGLU_BWD_Q) ? 0
                               : (EPI == EPI_SWIGLU_BWD) ? 2
                               : (NACC == 1 ? (MODE == GROUP_K ? 2 : 1) : 2);
-  static constexpr int STAGING_BYTES = 4 * NBUF * 4096;
+  static constexpr int STAGING_BYTES = EPW * NBUF * 4096;
   // MXFP8: per stage, one 512-byte scale chunk per 128 rows of A and of B (TMEM: 4 columns each)
   static constexpr int SF_BYTES = MX ? 512 + (BN / 128) * 512 : 0;
   static constexpr int SF_COLS = MX ? 4 + 4 * (BN / 128) : 0;
@@ -343,7 +346,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       // single CTA: every epilogue thread arrives; pair: lane 0 of the 4 epilogue warps of each CTA
-      mbar_init(&tempty[b], PAIR ? 8 : kEpiThreads);
+      mbar_init(&tempty[b], PAIR ? 8 : C::EPW * 32);
     }
     mbar_init(done, 1);
     *abort_word = 0;
@@ -708,14 +711,16 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
         mbar_wait_bounded(done, 0, p.wait_limit_ns, nullptr, p.err);
       }
     }
-  } else if (warp >= 2 && warp < 6) {
+  } else if (warp >= 2 && warp < 2 + C::EPW) {
     // ===================== epilogue (warps 2..5) =====================
     // Each warp owns the 32 accumulator rows of its TMEM lane quadrant (one row per thread). It
     // stages 32-row x 128-byte boxes in swizzled shared memory and stores them with TMA. A warp's
     // slab of 32 rows is entirely inside or entirely outside its expert's 32-aligned group, so whole
     // slabs are skipped instead of masking rows; columns past N are clipped by the tensor bounds.
     const int q = warp & 3;               // TMEM lane quadrant this warp may access
-    uint8_t* wstg = stg + (size_t)q * C::NBUF * 4096;
+    const int ew = warp - 2;              // epilogue warp index
+    const int chalf = ew >> 2;            // eight epilogue warps: the accumulator column half
+    uint8_t* wstg = stg + (size_t)ew * C::NBUF * 4096;
     int nb = 0;                           // next staging box (round robin)
     int local = 0;
     TileInfo nxt;  // the next tile's entry is fetched a tile ahead
@@ -732,14 +737,15 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + chalf * (BN / 2);
       // Full tile: this warp's 32 rows are rows q*32.. of the CTA's 128, over all BN accumulator
       // columns. Pair tail tile (M = 128): rows (q&1)*32.. of the CTA's 64, over the BN/2 accumulator
       // columns of its lane half, which hold output columns (q>>1)*BN/2 + [0, BN/2) of the tile.
       const bool half = ti_half<PAIR, MODE>(ti, p);
       const int slab = half ? ti.m0 + (int)rank * C::HALF_M + (q & 1) * 32
                             : ti.m0 + (int)rank * BM + q * 32;  // first tile row of this warp
-      const int whalf = half ? (q >> 1) : 0;                   // lane half (tail tiles)
+      // output column half: the lane half of a pair tail tile, or this warp's half of the columns
+      const int whalf = half ? (q >> 1) : chalf;
       const bool active = slab < ti_rows<MODE>(ti, p);         // warp-uniform
       int c1;                                                  // tensor row of this slab
       if constexpr (MODE == GROUP_K) c1 = ti.e * (p.c_group_rows ? p.c_group_rows : p.M) + slab;
@@ -961,7 +967,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
         };
         if (active) {
           if (half) store(std::integral_constant<int, BN / 2 / 32>{});
-          else store(std::integral_constant<int, BN / 32>{});
+          else store(std::integral_constant<int, BN / 32 / (C::EPW / 4)>{});
         }
       }
       tc_fence_before();
