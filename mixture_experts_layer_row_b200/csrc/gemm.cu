@@ -345,8 +345,8 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      // single CTA: every epilogue thread arrives; pair: lane 0 of the 4 epilogue warps of each CTA
-      mbar_init(&tempty[b], PAIR ? 8 : C::EPW * 32);
+      // single CTA: every epilogue thread arrives; pair: lane 0 of every epilogue warp of each CTA
+      mbar_init(&tempty[b], PAIR ? 2 * C::EPW : C::EPW * 32);
     }
     mbar_init(done, 1);
     *abort_word = 0;
@@ -972,7 +972,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
       }
       tc_fence_before();
       if constexpr (PAIR) {
-        // the leader's MMA thread waits for all eight epilogue warps of the pair
+        // the leader's MMA thread waits for every epilogue warp of both CTAs of the pair
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * (uint32_t)buf);
       } else {
