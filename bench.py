@@ -650,8 +650,10 @@ def main():
     nb = lambda t: t.numel() * t.element_size()
     if layer.mx:
         kept = sum(nb(layer.qa_t[n]) for n in ("xtq", "xts", "atq", "ats")) + nb(layer.h13) + nb(layer.y)
-        R, es = layer.R, 2
-        kept_bf16 = R * (2 * w.d + 2 * w.F + w.F + w.d) * es  # x_perm, h13, a, y of the bf16 layer
+        # the bf16 layer of the same shapes keeps x_perm [R, d], h13 [R, 2F], a [R, F] and y [R, d],
+        # with its own routed-row count (its groups are padded to 32 rows, the MXFP8 layer's to 128)
+        R_bf16 = L.max_rows(L.make_config(w.T, w.d, w.F, w.E, w.k, L.DTYPE_BF16))
+        kept_bf16 = R_bf16 * (2 * w.d + 3 * w.F) * 2
         act_mem = {"kept_between_passes_bytes": kept, "bf16_layer_same_shapes_bytes": kept_bf16,
                    "ratio": kept / kept_bf16,
                    "note": "MXFP8 keeps the column forms of x and a (codes + scales), h13 and y"}
