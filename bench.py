@@ -120,11 +120,12 @@ def op_work(w, es=2, recompute=False):
     ops["combine_bwd"] = ((T * d + 2 * R * d) * es + T * k * 12, 0)
     if recompute:
         ops["gemm_fwd1_recompute"] = fwd1
+    # in the order moe_layer_bwd issues them
     ops["gemm_dgrad2_swiglu"] = ((R * d + E * d * F + 2 * R * 2 * F) * es, 2 * R * d * F)
-    ops["gemm_wgrad2"] = ((R * d + R * F + E * d * F) * es, 2 * R * d * F)
     ops["gemm_dgrad1"] = ((R * 2 * F + E * 2 * F * d + R * d) * es, 2 * R * 2 * F * d)
-    ops["gemm_wgrad1"] = ((R * 2 * F + R * d + E * 2 * F * d) * es, 2 * R * 2 * F * d)
     ops["token_reduce"] = ((R * d + T * d) * es + (T * k * 8 if w.routing == "learned" else 0), 0)
+    ops["gemm_wgrad2"] = ((R * d + R * F + E * d * F) * es, 2 * R * d * F)
+    ops["gemm_wgrad1"] = ((R * 2 * F + R * d + E * 2 * F * d) * es, 2 * R * 2 * F * d)
     if w.routing == "learned":
         ops["router_wgrad"] = ((T * E + T * d + E * d) * es, 2 * T * E * d)
     return ops
@@ -204,14 +205,14 @@ class Step:
             h13 = lay.dh13
         mark(); L.grouped_gemm(c, L.GEMM_DGRAD2_SWIGLU, lay.dy, inp["W2"], lay.dh13, None, h13,
                                lay.counts, lay.poff, lay.ws)
-        mark(); L.grouped_gemm(c, L.GEMM_WGRAD2, lay.dy, lay.a, lay.dW2, None, None, lay.counts,
-                               lay.poff, lay.ws)
         mark(); L.grouped_gemm(c, L.GEMM_DGRAD1, lay.dh13, inp["W13"], lay.dx_perm, None, None,
-                               lay.counts, lay.poff, lay.ws)
-        mark(); L.grouped_gemm(c, L.GEMM_WGRAD1, lay.dh13, lay.x_perm, lay.dW13, None, None,
                                lay.counts, lay.poff, lay.ws)
         mark(); L.token_reduce(c, lay.dx_perm, lay.prow, lay.dx, dls,
                                lay.idx if self.learned else None, inp["W_r"] if self.learned else None)
+        mark(); L.grouped_gemm(c, L.GEMM_WGRAD2, lay.dy, lay.a, lay.dW2, None, None, lay.counts,
+                               lay.poff, lay.ws)
+        mark(); L.grouped_gemm(c, L.GEMM_WGRAD1, lay.dh13, lay.x_perm, lay.dW13, None, None,
+                               lay.counts, lay.poff, lay.ws)
         if self.learned:
             mark(); L.router_wgrad(c, self.dlogits, inp["x"], lay.dW_r, lay.ws)
         mark()

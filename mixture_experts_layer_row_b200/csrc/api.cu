@@ -579,16 +579,18 @@ int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_sav
                     sv->poff, ws, s));
     h13 = g->dh13;
   }
+  // The data path first (dgrad2 -> dgrad1 -> token reduce, each reading what the one before it just
+  // wrote, partly still in L2), then the two weight gradients.
   MOE_TRY(gemm_op(cfg, MOE_GEMM_DGRAD2_SWIGLU, g->dy, w->W2, g->dh13, nullptr, h13, sv->counts,
                   sv->poff, ws, s));
-  MOE_TRY(gemm_op(cfg, MOE_GEMM_WGRAD2, g->dy, sv->a, g->dW2, nullptr, nullptr, sv->counts, sv->poff,
-                  ws, s));
   MOE_TRY(gemm_op(cfg, MOE_GEMM_DGRAD1, g->dh13, w->W13, g->dx_perm, nullptr, nullptr, sv->counts,
-                  sv->poff, ws, s));
-  MOE_TRY(gemm_op(cfg, MOE_GEMM_WGRAD1, g->dh13, sv->x_perm, g->dW13, nullptr, nullptr, sv->counts,
                   sv->poff, ws, s));
   MOE_TRY(launch_token_reduce(g->dx_perm, sv->prow, dlsel, router ? sv->idx : nullptr, w->W_r, dx,
                               cfg->T, cfg->k, cfg->E, rb, bf, max_rows_of(cfg), s));
+  MOE_TRY(gemm_op(cfg, MOE_GEMM_WGRAD2, g->dy, sv->a, g->dW2, nullptr, nullptr, sv->counts, sv->poff,
+                  ws, s));
+  MOE_TRY(gemm_op(cfg, MOE_GEMM_WGRAD1, g->dh13, sv->x_perm, g->dW13, nullptr, nullptr, sv->counts,
+                  sv->poff, ws, s));
   if (router) MOE_TRY(router_wgrad_impl(cfg, dlog, x, g->dW_r, ws, s));
   return MOE_OK;
 }

@@ -10,7 +10,7 @@ def test_bf16_op_order_is_the_launch_order():
     w = WORKLOADS["e128_bf16"]
     assert list(bench.op_work(w)) == [
         "route_metadata", "dispatch", "gemm_fwd1_swiglu", "gemm_fwd2", "combine", "combine_bwd",
-        "gemm_dgrad2_swiglu", "gemm_wgrad2", "gemm_dgrad1", "gemm_wgrad1", "token_reduce"]
+        "gemm_dgrad2_swiglu", "gemm_dgrad1", "token_reduce", "gemm_wgrad2", "gemm_wgrad1"]
 
 
 def test_recompute_adds_one_gemm1_and_drops_the_h13_store():
