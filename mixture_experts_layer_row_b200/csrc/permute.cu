@@ -4,7 +4,9 @@
 //                 placement straight into each expert's contiguous input buffer: bytechap.com, "Como
 //                 funciona"; unite.ai, "Parallelismo, precisione e tecniche di memoria"); pad rows 0.
 //   combine       out[t] = sum_j g[t,j] y[prow[t,j]]  (a gather: deterministic, no atomics)
-//   combine_bwd   dy[prow[t,j]] = g[t,j] dout[t];  dg[t,j] = <dout[t], y[prow[t,j]]> (+ score grads)
+//   combine_bwd   dy[prow[t,j]] = g[t,j] dout[t];  dg[t,j] = <dout[t], y[prow[t,j]]> (+ score grads);
+//                 its reads are staged in shared memory by bulk copies (three streams per token: the
+//                 register-staged loop could not keep enough of them in flight)
 //   token_reduce  dx[t] = sum_j dx_perm[prow[t,j]] (+ sum_j dl[t,j] W_r[idx[t,j]])
 // Every routed-row pad row (the tail of each expert's 32-aligned group) is written as zero by
 // dispatch and combine_bwd so the grouped GEMMs can run whole 32-row blocks. An entry whose padded row
@@ -17,6 +19,9 @@ namespace moe {
 namespace {
 
 constexpr int kWarps = 8;  // warps per block = tokens per block
+// combine backward with bulk-staged rows: staging per block, and the dynamic shared-memory ceiling
+constexpr size_t kCbStageBudget = 60 * 1024;
+constexpr size_t kCbSmemMax = 227 * 1024;
 
 // 16-byte vector <-> floats. BF16: 8 values per vector; FP32: 4.
 template <bool BF16>
@@ -150,6 +155,56 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(const uint4* __res
   }
 }
 
+// The end of a token's combine backward, once each lane holds its partial dot products with the k
+// rows: dgates[t,j] = <dout[t], y[row_j]>, and for a learned router the score gradients dl_j =
+// g_j (dg_j - sum_i g_i dg_i) and the dense row dlogits[t, e] (act dtype), zero except at the chosen
+// experts.
+template <bool BF16>
+__device__ __forceinline__ void combine_bwd_finish(float (&dot)[8], const float (&g)[8], int t, int k,
+                                                   int E, int lane, const int32_t* __restrict__ idx,
+                                                   float* __restrict__ dgates, float* __restrict__ dlsel,
+                                                   void* __restrict__ dlogits) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], off);
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < k) s = fmaf(g[j], dot[j], s);
+  float mydl = 0.f;
+  int mye = -1;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < k && lane == j) {
+      dgates[(size_t)t * k + j] = dot[j];
+      mydl = g[j] * (dot[j] - s);
+      if (dlsel) dlsel[(size_t)t * k + j] = mydl;
+      mye = idx ? idx[(size_t)t * k + j] : -1;
+    }
+  }
+  if (dlogits) {
+    int ej[8];
+    float dj[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      ej[j] = __shfl_sync(0xffffffffu, mye, j);
+      dj[j] = __shfl_sync(0xffffffffu, mydl, j);
+    }
+    for (int e = lane; e < E; e += 32) {
+      float val = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < k && ej[j] == e) val = dj[j];
+      if (BF16)
+        reinterpret_cast<__nv_bfloat16*>(dlogits)[(size_t)t * E + e] = __float2bfloat16_rn(val);
+      else
+        reinterpret_cast<float*>(dlogits)[(size_t)t * E + e] = val;
+    }
+  }
+}
+
 template <bool BF16>
 // 64 registers at most: four blocks (32 warps) per SM keep enough loads in flight
 __global__ void __launch_bounds__(kWarps * 32, 4) combine_bwd_kernel(
@@ -195,46 +250,88 @@ __global__ void __launch_bounds__(kWarps * 32, 4) combine_bwd_kernel(
       }
     }
   }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dot[j] += __shfl_xor_sync(0xffffffffu, dot[j], off);
+  combine_bwd_finish<BF16>(dot, g, t, k, E, lane, idx, dgates, dlsel, dlogits);
+}
+
+// The same combine backward with the reads staged in shared memory by bulk copies. One thread of the
+// block copies the block's dout rows (one copy: they are consecutive) and every routed y row of its
+// tokens, all completing on one mbarrier; then one warp per token computes from shared memory. Data
+// in flight no longer occupies registers (a register-staged 16-byte load holds four until it lands),
+// so with three blocks per SM about twice as many bytes of the gather are in flight, and one block
+// computes while the others' copies land (60 KB per block measured best: 62 us against 65 us for
+// 100 KB and 81 us for 150 KB, e128 bf16 shapes).
+template <bool BF16>
+__global__ void __launch_bounds__(kWarps * 32) combine_bwd_bulk_kernel(
+    const uint4* __restrict__ dout, const uint4* __restrict__ y, const float* __restrict__ gates,
+    const int32_t* __restrict__ prow, const int32_t* __restrict__ idx,
+    const int32_t* __restrict__ counts, const int32_t* __restrict__ poff, uint4* __restrict__ dy,
+    float* __restrict__ dgates, float* __restrict__ dlsel, void* __restrict__ dlogits, int T, int k,
+    int E, int vpr, int tok_blocks, int max_rows, int tpb) {
+  pdl_enter();  // wait for the previous kernel before any global access
+  using V = Vec<BF16>;
+  if ((int)blockIdx.x >= tok_blocks) {
+    zero_pad_rows(dy, blockIdx.x - tok_blocks, counts, poff, vpr);
+    return;
   }
-  float s = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (j < k) s = fmaf(g[j], dot[j], s);
-  float mydl = 0.f;
-  int mye = -1;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j < k && lane == j) {
-      dgates[(size_t)t * k + j] = dot[j];
-      mydl = g[j] * (dot[j] - s);
-      if (dlsel) dlsel[(size_t)t * k + j] = mydl;
-      mye = idx ? idx[(size_t)t * k + j] : -1;
+  extern __shared__ __align__(128) uint8_t cb_smem[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(cb_smem);
+  uint4* sdout = reinterpret_cast<uint4*>(cb_smem + 128);  // [tpb][vpr]
+  uint4* sy = sdout + (size_t)tpb * vpr;                    // [tpb][k][vpr], slot-major per token
+  const int t0 = blockIdx.x * tpb;
+  const int nt = min(tpb, T - t0);
+  const uint32_t rb = (uint32_t)vpr * 16u;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    uint32_t bytes = (uint32_t)nt * rb;
+    for (int i = 0; i < nt * k; ++i) {
+      const int r = prow[(size_t)t0 * k + i];
+      if (r >= 0 && r < max_rows) bytes += rb;
+    }
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(sdout, dout + (size_t)t0 * vpr, (uint32_t)nt * rb, bar);
+    for (int i = 0; i < nt * k; ++i) {
+      const int r = prow[(size_t)t0 * k + i];
+      if (r >= 0 && r < max_rows) bulk_load(sy + (size_t)i * vpr, y + (size_t)r * vpr, rb, bar);
     }
   }
-  if (dlogits) {
-    // dense score-gradient row: zero except the k chosen experts
-    int ej[8];
-    float dj[8];
+  __syncthreads();
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // every copy lands unless the memory system fails; the wait is bounded all the same
+  const bool ready = mbar_wait_bounded(bar, 0, 2000000000ull, nullptr, nullptr);
+  if (w >= nt || !ready) return;
+  const int t = t0 + w;
+  const int myrow = slot_row(prow, t, k, lane, max_rows);
+  const float myg = lane < k ? gates[(size_t)t * k + lane] : 0.f;
+  int rows[8];
+  float g[8], dot[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    rows[j] = __shfl_sync(0xffffffffu, myrow, j);
+    g[j] = __shfl_sync(0xffffffffu, myg, j);
+    dot[j] = 0.f;
+  }
+  const uint4* sd = sdout + (size_t)w * vpr;
+  const uint4* sw = sy + (size_t)w * k * vpr;
+#pragma unroll 1
+  for (int v = lane; v < vpr; v += 32) {
+    float fd[V::N];
+    V::unpack(sd[v], fd);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      ej[j] = __shfl_sync(0xffffffffu, mye, j);
-      dj[j] = __shfl_sync(0xffffffffu, mydl, j);
-    }
-    for (int e = lane; e < E; e += 32) {
-      float val = 0.f;
+      if (j < k && rows[j] >= 0) {
+        float fy[V::N], o[V::N];
+        V::unpack(sw[(size_t)j * vpr + v], fy);
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j < k && ej[j] == e) val = dj[j];
-      if (BF16)
-        reinterpret_cast<__nv_bfloat16*>(dlogits)[(size_t)t * E + e] = __float2bfloat16_rn(val);
-      else
-        reinterpret_cast<float*>(dlogits)[(size_t)t * E + e] = val;
+        for (int i = 0; i < V::N; ++i) {
+          dot[j] = fmaf(fd[i], fy[i], dot[j]);
+          o[i] = g[j] * fd[i];
+        }
+        dy[(size_t)rows[j] * vpr + v] = V::pack(o);
+      }
     }
   }
+  combine_bwd_finish<BF16>(dot, g, t, k, E, lane, idx, dgates, dlsel, dlogits);
 }
 
 template <bool BF16>
@@ -363,6 +460,38 @@ int launch_combine_bwd(const void* dout, const void* y, const float* gates, cons
                        bool bf16, int64_t max_rows, cudaStream_t s) {
   const int vpr = row_bytes / 16;
   const int mr = clamp_rows(max_rows);
+  // bulk-staged kernel: tokens per block sized for about 60 KB of staged rows (three blocks per SM)
+  const size_t per_tok = (size_t)(1 + k) * row_bytes;
+  const int tpb = (int)std::min<size_t>(kWarps, std::max<size_t>(1, kCbStageBudget / per_tok));
+  const size_t smem = 128 + (size_t)tpb * per_tok;
+  if (smem <= kCbSmemMax) {
+    static bool attr_done[2][64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!attr_done[bf16][dev]) {
+      const cudaError_t e = bf16 ? cudaFuncSetAttribute(combine_bwd_bulk_kernel<true>,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                        (int)kCbSmemMax)
+                                 : cudaFuncSetAttribute(combine_bwd_bulk_kernel<false>,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                        (int)kCbSmemMax);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
+      attr_done[bf16][dev] = true;
+    }
+    const int tb = (T + tpb - 1) / tpb;
+    if (bf16)
+      MOE_LAUNCH(launch_pdl(combine_bwd_bulk_kernel<true>, tb + E, kWarps * 32, smem, s,
+          static_cast<const uint4*>(dout), static_cast<const uint4*>(y), gates, prow, idx, counts,
+          poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tb, mr, tpb));
+    else
+      MOE_LAUNCH(launch_pdl(combine_bwd_bulk_kernel<false>, tb + E, kWarps * 32, smem, s,
+          static_cast<const uint4*>(dout), static_cast<const uint4*>(y), gates, prow, idx, counts,
+          poff, static_cast<uint4*>(dy), dgates, dlsel, dlogits, T, k, E, vpr, tb, mr, tpb));
+    count_launches(1);
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+  // rows too wide to stage even one token: the register-staged kernel
   const int tok_blocks = (T + kWarps - 1) / kWarps;
   if (bf16)
     MOE_LAUNCH(launch_pdl(combine_bwd_kernel<true>, tok_blocks + E, kWarps * 32, 0, s, 
