@@ -63,7 +63,12 @@ def test_combine(dtype, T, d, E, k):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("T,d,E,k", [(300, 128, 8, 2), (1000, 2048, 128, 4)])
+@pytest.mark.parametrize("T,d,E,k", [(300, 128, 8, 2), (1000, 2048, 128, 4),
+                                     # k = 8, a ragged last block of the bulk-staged kernel
+                                     (37, 64, 5, 5), (45, 128, 8, 8),
+                                     # one token per block (rows of 16-32 KB), and rows too wide to
+                                     # stage (the register-staged kernel)
+                                     (40, 8192, 8, 8), (24, 16384, 8, 8)])
 def test_combine_bwd(dtype, T, d, E, k):
     L, cfg, R, idx, meta, t32, _, gates = _setup(T, d, E, k, dtype, 4)
     g = torch.Generator().manual_seed(5)
