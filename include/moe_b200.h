@@ -367,10 +367,11 @@ typedef struct {
 MOE_API int moe_layer_fwd(const moe_config_t* cfg, const moe_weights_t* w, const void* x, const float* bias,
                   void* out, moe_saved_t* saved, void* ws, size_t ws_bytes, void* stream);
 
-/* Whole backward given dout (act [T,d]): combine_bwd -> GEMM2 dgrad + SwiGLU bwd -> GEMM2 wgrad ->
- * GEMM1 dgrad -> GEMM1 wgrad -> token reduce (+ router terms). x is the forward input. The
- * selection is held fixed (no gradient through the top-k choice). Requires cfg->renorm == 1 when
- * the router is learned. */
+/* Whole backward given dout (act [T,d]): combine_bwd -> GEMM2 dgrad + SwiGLU bwd -> GEMM1 dgrad ->
+ * token reduce (+ router input term) -> GEMM2 wgrad -> GEMM1 wgrad (-> router wgrad): the data path
+ * first, each op reading what the one before it just wrote, then the weight gradients. x is the
+ * forward input; dx (act [T,d]) is the caller's buffer. The selection is held fixed (no gradient
+ * through the top-k choice). Requires cfg->renorm == 1 when the router is learned. */
 MOE_API int moe_layer_bwd(const moe_config_t* cfg, const moe_weights_t* w, const moe_saved_t* saved,
                   const void* x, const void* dout, void* dx, moe_grads_t* g, void* ws,
                   size_t ws_bytes, void* stream);
