@@ -22,6 +22,7 @@ constexpr int kWarps = 8;  // warps per block = tokens per block
 // combine backward with bulk-staged rows: staging per block, and the dynamic shared-memory ceiling
 constexpr size_t kCbStageBudget = 60 * 1024;
 constexpr size_t kCbSmemMax = 227 * 1024;
+static_assert(kWarps * 8 <= 64, "one warp issues a block's routed-row copies, two slots per lane (k <= 8)");
 
 // 16-byte vector <-> floats. BF16: 8 values per vector; FP32: 4.
 template <bool BF16>
@@ -283,20 +284,27 @@ __global__ void __launch_bounds__(kWarps * 32) combine_bwd_bulk_kernel(
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     fence_barrier_init();
-    uint32_t bytes = (uint32_t)nt * rb;
-    for (int i = 0; i < nt * k; ++i) {
-      const int r = prow[(size_t)t0 * k + i];
-      if (r >= 0 && r < max_rows) bytes += rb;
-    }
-    mbar_arrive_expect_tx(bar, bytes);
-    bulk_load(sdout, dout + (size_t)t0 * vpr, (uint32_t)nt * rb, bar);
-    for (int i = 0; i < nt * k; ++i) {
-      const int r = prow[(size_t)t0 * k + i];
-      if (r >= 0 && r < max_rows) bulk_load(sy + (size_t)i * vpr, y + (size_t)r * vpr, rb, bar);
-    }
   }
   __syncthreads();
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (w == 0) {
+    // lane i owns routed slots i and i + 32 of the block (tpb * k <= 64): one parallel read of the
+    // rows, a ballot for the byte count, and each lane issues its own copies once lane 0 has armed
+    // the barrier
+    const int ns = nt * k;
+    int r0 = lane < ns ? prow[(size_t)t0 * k + lane] : -1;
+    int r1 = lane + 32 < ns ? prow[(size_t)t0 * k + lane + 32] : -1;
+    if (!(r0 >= 0 && r0 < max_rows)) r0 = -1;
+    if (!(r1 >= 0 && r1 < max_rows)) r1 = -1;
+    const int nvalid = __popc(__ballot_sync(0xffffffffu, r0 >= 0)) + __popc(__ballot_sync(0xffffffffu, r1 >= 0));
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar, (uint32_t)(nt + nvalid) * rb);
+      bulk_load(sdout, dout + (size_t)t0 * vpr, (uint32_t)nt * rb, bar);
+    }
+    __syncwarp();
+    if (r0 >= 0) bulk_load(sy + (size_t)lane * vpr, y + (size_t)r0 * vpr, rb, bar);
+    if (r1 >= 0) bulk_load(sy + (size_t)(lane + 32) * vpr, y + (size_t)r1 * vpr, rb, bar);
+  }
   // every copy lands unless the memory system fails; the wait is bounded all the same
   const bool ready = mbar_wait_bounded(bar, 0, 2000000000ull, nullptr, nullptr);
   if (w >= nt || !ready) return;
