@@ -164,10 +164,20 @@ __global__ void __launch_bounds__(256) scan_kernel(int32_t* __restrict__ hist, i
   const int e = threadIdx.x;
   int run = 0;
   if (e < E) {
-    for (int c = 0; c < nchunks; ++c) {
-      const int v = hist[(size_t)c * E + e];
-      hist[(size_t)c * E + e] = run;
-      run += v;
+    // the expert's per-chunk counts in batches of 16 loads in flight (a loop that waited on each load
+    // in turn took 12 us for 32 chunks), replaced in place by their exclusive prefix
+    constexpr int kB = 16;
+    for (int c0 = 0; c0 < nchunks; c0 += kB) {
+      int v[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) v[u] = c0 + u < nchunks ? hist[(size_t)(c0 + u) * E + e] : 0;
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        if (c0 + u < nchunks) {
+          hist[(size_t)(c0 + u) * E + e] = run;
+          run += v[u];
+        }
+      }
     }
   }
   const int cnt = e < E ? run : 0;
