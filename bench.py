@@ -256,7 +256,11 @@ class Step:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the timed region runs."""
+    """SM clock and throttle reasons around and during the timed region: NVML reads from a background
+    thread, one when sampling starts, then every 50 ms, and one more when the region ends (so even a
+    region of a few tens of milliseconds is bracketed); `nvidia-smi -lms 200` where NVML cannot be
+    used. Polling NVML every few milliseconds slowed the measured step by 10 %, so the period stays
+    long."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -266,18 +270,88 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = None
+        self.nvml = None
+        self.thread = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(getattr(torch.cuda.get_device_properties(self.index), "uuid", "") or "")
+        for u in (uuid, "GPU-" + uuid):
+            try:
+                if u and u != "GPU-":
+                    return pynvml, pynvml.nvmlDeviceGetHandleByUUID(u)
+            except pynvml.NVMLError:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
 
     def start(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+            self.nvml = (nv, h, nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            nv, h, _ = self.nvml
+            self.rows, self.stop_evt = [], threading.Event()
+
+            def run():
+                while True:
+                    try:
+                        self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                          nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                    except nv.NVMLError:
+                        break
+                    if self.stop_evt.wait(0.05):
+                        break
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            t0 = time.time()
+            while not self.rows and self.thread.is_alive() and time.time() - t0 < 2.0:
+                time.sleep(0.001)
+            return
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)  # its start-up, before the timed region
         except (OSError, FileNotFoundError):
             self.proc = None
 
+    @staticmethod
+    def _summary(sm, mx, reasons, n, source):
+        loaded = [v for v in sm if mx and v > 0.3 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": n, "source": source}
+
     def stop(self):
+        if self.nvml is not None:
+            nv, h, mx = self.nvml
+            self.stop_evt.set()
+            self.thread.join(timeout=2)
+            try:  # the region's end
+                self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                  nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except nv.NVMLError:
+                pass
+            rows = list(self.rows)
+            try:
+                nv.nvmlShutdown()
+            except Exception:
+                pass
+            if not rows:
+                return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["no samples"], "source": "nvml"}
+            bits = (("hw_slowdown", nv.nvmlClocksEventReasonHwSlowdown),
+                    ("hw_thermal_slowdown", nv.nvmlClocksEventReasonHwThermalSlowdown),
+                    ("sw_thermal_slowdown", nv.nvmlClocksEventReasonSwThermalSlowdown),
+                    ("sw_power_cap", nv.nvmlClocksEventReasonSwPowerCap))
+            reasons = {name for _, r in rows for name, b in bits if r & b}
+            return self._summary([float(c) for c, _ in rows], float(mx), reasons, len(rows),
+                                 "nvml at start, every 50 ms and at the end")
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -307,10 +381,7 @@ class ClockSampler:
                               ("sw_thermal_slowdown", 7), ("sw_power_cap", 8)):
                 if r[col].lower().startswith("active"):
                     reasons.add(name)
-        loaded = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(rows)}
+        return self._summary(sm, max(mx) if mx else None, reasons, len(rows), "nvidia-smi every 200 ms")
 
 
 class ExpertSample:
@@ -469,7 +540,6 @@ def gemm_peak(args):
     torch.cuda.synchronize()
     clocks = ClockSampler(0)
     clocks.start()
-    time.sleep(0.3)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(20):
@@ -591,7 +661,6 @@ def main():
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.3)
     n0 = L.launch_count()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record()

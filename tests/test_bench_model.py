@@ -57,3 +57,53 @@ def test_mxfp8_activations_leave_their_producers_quantised():
     assert ops["gemm_fwd1_swiglu_quant"][0] == q(R * d) + q(E * 2 * F * d) + R * 2 * F * 2 + 2 * q(R * F)
     assert ops["combine_bwd_quant"][0] == (T * d + R * d) * 2 + T * k * 8 + R * 4 + 2 * q(R * d)
     assert ops["gemm_dgrad2_swiglu_quant"][0] == q(R * d) + q(E * d * F) + R * 2 * F * 2 + 2 * q(R * 2 * F)
+
+
+class _FakeNvml:
+    """Enough of NVML for the bench's clock sampler: a fixed max clock, a clock sequence and the
+    throttle-reason bits (the values NVML defines)."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonSwPowerCap = 0x4
+
+    class NVMLError(Exception):
+        pass
+
+    def __init__(self, clocks, reasons):
+        self.clocks, self.reasons, self.i = clocks, reasons, 0
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        self.i += 1
+        return self.clocks[self.i % len(self.clocks)]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.reasons
+
+    def nvmlShutdown(self):
+        pass
+
+
+def test_clock_sampler_reads_clocks_and_reasons_from_nvml():
+    import time
+    fake = _FakeNvml([1965, 1950, 120], 0x4 | 0x1)  # sw_power_cap, plus an idle bit that is not reported
+    cs = bench.ClockSampler(0)
+    cs._nvml_handle = lambda: (fake, object())
+    cs.start()
+    time.sleep(0.12)
+    out = cs.stop()
+    assert out["samples"] >= 3 and out["source"].startswith("nvml")
+    assert out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["sw_power_cap"]
+    # the idle 120 MHz samples are dropped before the median
+    assert out["sm_mhz"] in (1950.0, 1957.5, 1965.0)
+    fake2 = _FakeNvml([1965], 0x0)
+    cs2 = bench.ClockSampler(0)
+    cs2._nvml_handle = lambda: (fake2, object())
+    cs2.start()
+    time.sleep(0.02)
+    assert cs2.stop()["reasons"] == []
