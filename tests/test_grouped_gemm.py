@@ -17,6 +17,10 @@ SHAPES = {
     # with an empty second half, single-row and empty experts all occur
     "ragged_pairs": (512, 256, 256, 8, 2, [0, 1, 31, 33, 129, 200, 300, 330]),
     "edges": (400, 192, 384, 6, 2, [32, 127, 128, 0, 400, 113]),
+    # fwd2 / dgrad1 on CTA pairs with 256-column n-blocks: d = 768 gives three of them, d = 320 a
+    # second one with 64 valid columns (an expert holding every token, one holding none)
+    "pairs_n768": (512, 768, 256, 8, 2, [0, 1, 31, 33, 129, 200, 300, 330]),
+    "pairs_n320": (384, 320, 128, 4, 2, [100, 0, 284, 384]),
     "one_expert": (300, 128, 128, 4, 1, [300, 0, 0, 0]),
     "wide": (2048, 2048, 1024, 16, 4, None),
 }
