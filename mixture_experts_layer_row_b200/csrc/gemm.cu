@@ -82,13 +82,13 @@ struct Cfg {
   // MXFP8 tiles of 256 columns, whose per-stage scale columns leave no room for a second
   static constexpr int NACC = (MX && BN == 256) ? 1 : 2;
   static_assert(!epi_quant(EPI) || (MX && !PAIR), "quantising epilogues are MXFP8-only");
-  // staging boxes per epilogue warp: SwiGLU forward h13 gate + up + a (quantising: gate + up; a's codes
-  // go straight to global memory); SwiGLU backward dh13 gate + up (quantising: none, dh13's codes go
+  // staging boxes per epilogue warp: SwiGLU forward h13 gate + up (a, or a's codes when quantising,
+  // goes straight from registers to global memory); SwiGLU backward dh13 gate + up (quantising: none, dh13's codes go
   // straight to global memory); plain stores round robin over NBUF boxes. With one accumulator the
   // MMA waits for the epilogue: the short-contraction wgrad tiles take two boxes (the epilogue hands
   // the accumulator back sooner) at the price of a pipeline stage; long-contraction tiles keep the
   // deeper ring and one box.
-  static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 3
+  static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 2
                               : (EPI == EPI_SWIGLU_FWD_Q) ? 2
                               : (EPI == EPI_SWIGLU_BWD_Q) ? 0
                               : (EPI == EPI_SWIGLU_BWD) ? 2
@@ -256,6 +256,23 @@ __device__ __forceinline__ void stage_row32(uint8_t* box, int lane, int ch0, con
   }
 }
 
+// Store 32 fp32 values of this thread's row to global memory as OES-byte elements (16-byte stores).
+template <int OES>
+__device__ __forceinline__ void store_row32_global(uint8_t* dst, const float* v) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  if constexpr (OES == 2) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      d[q] = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                        pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      d[q] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                        __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+  }
+}
+
 // Store 32 one-byte codes (8 words, column order) of this thread's row: one whole, aligned 32-byte
 // sector of the [rows, cols] code array (the chunk's first column is a multiple of 32).
 __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t (&c)[8]) {
@@ -306,7 +323,6 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmC,
-                        const __grid_constant__ CUtensorMap tmC2,
                         const __grid_constant__ CUtensorMap tmX1,
                         const __grid_constant__ CUtensorMap tmX2, const GemmParams p) {
   // tmX1 / tmX2: pair tail tiles -- 64-row boxes of A / of B (SwiGLU forward)
@@ -357,7 +373,6 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     prefetch_tensormap(&tmC);
-    if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmC2);
     if constexpr (PAIR && MODE == GROUP_M) {
       prefetch_tensormap(&tmA64);
       if constexpr (EPI == EPI_SWIGLU_FWD) prefetch_tensormap(&tmB64);
@@ -768,7 +783,6 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
           tmem_ld_32x32b_x32(t_row + UP, ua);
           uint8_t* bg = wstg;
           uint8_t* bu = wstg + 4096;
-          uint8_t* ba = wstg + 8192;  // a (bf16; not used by the quantising variant)
           uint32_t srow = 0;           // row-block scale bytes of four consecutive chunks
 #pragma unroll
           for (int j = 0; j < NCH; ++j) {
@@ -810,7 +824,11 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
               store_codes32(p.q_qc + off, cc);
               p.q_sc[tiled_sf_offset(col0 + j * 32 + lane, qrb, p.q_kb_col)] = scol;
             } else {
-              stage_row32<C::OES>(ba, lane, ch0, a);
+              // a straight from registers (the row's 32 values are 64 or 128 contiguous bytes): the
+              // epilogue has time to spare behind the MMAs, and the box it no longer stages leaves
+              // room for a sixth pipeline stage
+              store_row32_global<C::OES>(static_cast<uint8_t*>(p.C2) +
+                                             ((size_t)(c1 + lane) * p.ldc2 + col0 + j * 32) * C::OES, a);
             }
             if (j % CPB == CPB - 1 || j == NCH - 1) {
               const int c = col0 + (j / CPB) * C::OEPR;
@@ -818,7 +836,6 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
                 box_store(&tmC, bg, lane, c, c1);
                 box_store(&tmC, bu, lane, p.F + c, c1);
               }
-              if constexpr (EPI == EPI_SWIGLU_FWD) box_store(&tmC2, ba, lane, c, c1);
             }
             if constexpr (EPI == EPI_SWIGLU_FWD_Q) {
               if ((j & 3) == 3) {  // the row's 4 scale bytes of 128 columns
@@ -1113,12 +1130,14 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
       return MOE_ERR_CUDA;
   }
   // outputs: 32-row x 128-byte boxes stored from the epilogue's swizzled staging
-  CUtensorMap tc, tc2;
+  CUtensorMap tc;
   const int64_t out_rows =
       (MODE == GROUP_K) ? (int64_t)k_groups(p) * (p.c_group_rows ? p.c_group_rows : p.M) : A.rows;
   const int64_t out_cols = (epi_swiglu_fwd(EPI) || epi_swiglu_bwd(EPI)) ? 2 * (int64_t)p.F : p.N;
-  if (EPI == EPI_SWIGLU_FWD && !make_tmap(&tc2, p.C2, C::OES, out_rows, p.F, p.ldc2, C::OEPR, 32, 2))
-    return MOE_ERR_CUDA;
+  // SwiGLU forward: a [rows, F] is stored from registers with 16-byte stores
+  if (EPI == EPI_SWIGLU_FWD &&
+      (!p.C2 || (reinterpret_cast<uintptr_t>(p.C2) & 15) || (p.ldc2 * C::OES) % 16 != 0))
+    return MOE_ERR_INVALID_ARG;
   // quantising epilogues: the codes [rows, F] (a) or [rows, 2F] (dh13) are stored from registers
   if (epi_quant(EPI) && (!p.q_qr || !p.q_qc || !p.q_sr || !p.q_sc)) return MOE_ERR_INVALID_ARG;
   if (p.C) {
@@ -1126,11 +1145,10 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
   } else if (EPI == EPI_SWIGLU_BWD_Q) {
     tc = ta;  // dh13 leaves as codes only: tc is never used
   } else if (EPI == EPI_SWIGLU_FWD) {
-    tc = tc2;  // SwiGLU forward without h13: only a is stored, tc is never used
+    tc = ta;  // SwiGLU forward without h13: only a is stored, tc is never used
   } else {
     return MOE_ERR_INVALID_ARG;
   }
-  if (EPI != EPI_SWIGLU_FWD) tc2 = tc;
   // pair tail tiles (M = 128 over the pair): 64-row boxes of A, and of B for the SwiGLU forward,
   // whose tail tile loads 64 gate + 64 up rows per CTA
   CUtensorMap ta64 = ta, tb64 = tb;
@@ -1171,11 +1189,11 @@ int launch_impl(const GemmOperand& A, const GemmOperand& B, const GemmParams& p,
     if (cap > 0 && cap < pairs) pairs = cap;
     cfg.gridDim = dim3((unsigned)(2 * pairs));
     cfg.numAttrs = 2;  // cluster shape + programmatic dependent launch
-    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, tc2, ta64, tb64, q) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, ta64, tb64, q) != cudaSuccess) return MOE_ERR_CUDA;
   } else {
     int64_t grid = sm_count();
     if (cap > 0 && cap < grid) grid = cap;
-    MOE_LAUNCH(launch_pdl(kern, (unsigned)grid, C::THREADS, C::SMEM_BYTES, s, ta, tb, tc, tc2, ta64, tb64, q));
+    MOE_LAUNCH(launch_pdl(kern, (unsigned)grid, C::THREADS, C::SMEM_BYTES, s, ta, tb, tc, ta64, tb64, q));
   }
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
