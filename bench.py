@@ -64,6 +64,7 @@ MEASURED_TRAFFIC = {
     # e128_bf16, ncu capture of the full-size launch of the current kernel
     # (dram__bytes_read.sum + dram__bytes_write.sum)
     ("e128_bf16", "gemm_wgrad1"): 286.59e6 + 1.0129e9,
+    ("e128_bf16", "gemm_fwd1_swiglu"): 1.23e9 + 198.25e6,
 }
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal
 

@@ -71,10 +71,16 @@ struct Cfg {
   static constexpr bool MX = (ES == 1);      // MXFP8 block-scaled (E4M3 operands, UE8M0 scales)
   static_assert(!(PAIR && MX), "block-scaled MMAs run on single CTAs");
   // epilogue warps: four (one per TMEM lane quadrant), or eight (two per quadrant, each taking half
-  // of the accumulator columns) where the MMA waits for the epilogue on every tile: MXFP8 wgrad tiles,
-  // with one accumulator and a contraction of a few stages. The stores a warp keeps in flight bound
-  // how fast it drains the accumulator.
+  // of the accumulator columns) for the MXFP8 wgrad tiles: one accumulator (below) and a contraction of
+  // a few stages, so the accumulator must come back quickly.
   static constexpr int EPW = (ES == 1 && BN == 256 && MODE == GROUP_K && !PAIR && EPI == EPI_STORE) ? 8 : 4;
+  // The same tiles hold one accumulator (below). There each thread reads its 128 accumulator columns
+  // into registers and hands the accumulator back before it converts and stores them, so the next
+  // tile's MMAs overlap the stores. The stores go through a 2 KB transpose buffer per warp (plain
+  // shared-memory stores and loads, whole 64-byte row segments to global memory) instead of TMA
+  // staging boxes, which leaves room for a fourth pipeline stage: a tile's contraction (512 routed
+  // rows at the MXFP8 shapes) is then loaded while the previous tile computes.
+  static constexpr bool EARLY = EPW == 8;
   static constexpr int THREADS = 64 + 32 * EPW;  // producer, MMA issuer, epilogue
   static constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : (MX ? 2 : ES);  // output element size
   static constexpr int OEPR = 128 / OES;     // output columns per staged box
@@ -83,17 +89,19 @@ struct Cfg {
   static constexpr int NACC = (MX && BN == 256) ? 1 : 2;
   static_assert(!epi_quant(EPI) || (MX && !PAIR), "quantising epilogues are MXFP8-only");
   // staging boxes per epilogue warp: SwiGLU forward h13 gate + up (a, or a's codes when quantising,
-  // goes straight from registers to global memory); SwiGLU backward dh13 gate + up (quantising: none, dh13's codes go
-  // straight to global memory); plain stores round robin over NBUF boxes. With one accumulator the
-  // MMA waits for the epilogue: the short-contraction wgrad tiles take two boxes (the epilogue hands
-  // the accumulator back sooner) at the price of a pipeline stage; long-contraction tiles keep the
-  // deeper ring and one box.
+  // goes straight from registers to global memory); SwiGLU backward dh13 gate + up (quantising: none,
+  // dh13's codes go straight to global memory); plain stores round robin over NBUF boxes, one where
+  // a single accumulator makes the MMA wait for the epilogue (a deeper ring pays more there than a
+  // second box).
+  // The early-release wgrad epilogue uses no boxes (its transpose buffers are sized below).
   static constexpr int NBUF = (EPI == EPI_SWIGLU_FWD) ? 2
                               : (EPI == EPI_SWIGLU_FWD_Q) ? 2
                               : (EPI == EPI_SWIGLU_BWD_Q) ? 0
                               : (EPI == EPI_SWIGLU_BWD) ? 2
-                              : (NACC == 1 ? (MODE == GROUP_K ? 2 : 1) : 2);
-  static constexpr int STAGING_BYTES = EPW * NBUF * 4096;
+                              : (NACC == 1 ? 1 : 2);
+  static constexpr int STAGING_BYTES = EARLY ? EPW * 2048 : EPW * NBUF * 4096;
+  static_assert(!EARLY || (NACC == 1 && OES == 2 && EPI == EPI_STORE), "early release: bf16 stores");
+  static_assert(STAGING_BYTES % (EPW * 1024) == 0, "per-warp staging: whole, 1 KB aligned slices");
   // MXFP8: per stage, one 512-byte scale chunk per 128 rows of A and of B (TMEM: 4 columns each)
   static constexpr int SF_BYTES = MX ? 512 + (BN / 128) * 512 : 0;
   static constexpr int SF_COLS = MX ? 4 + 4 * (BN / 128) : 0;
@@ -735,7 +743,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
     const int q = warp & 3;               // TMEM lane quadrant this warp may access
     const int ew = warp - 2;              // epilogue warp index
     const int chalf = ew >> 2;            // eight epilogue warps: the accumulator column half
-    uint8_t* wstg = stg + (size_t)ew * C::NBUF * 4096;
+    uint8_t* wstg = stg + (size_t)ew * (C::STAGING_BYTES / C::EPW);  // this warp's staging
     int nb = 0;                           // next staging box (round robin)
     int local = 0;
     TileInfo nxt;  // the next tile's entry is fetched a tile ahead
@@ -982,7 +990,51 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
             }
           }
         };
-        if (active) {
+        if constexpr (C::EARLY) {
+          constexpr int NCH = BN / 32 / (C::EPW / 4);  // this warp's 32-column chunks
+          const bool acc = nst > 0 && active;
+          uint32_t r[NCH][32];
+          if (acc) {
+#pragma unroll
+            for (int j = 0; j < NCH; ++j) tmem_ld_32x32b_x32(t_row + j * 32, r[j]);
+            tmem_ld_wait_regs(r[0]);
+#pragma unroll
+            for (int j = 1; j < NCH; ++j) tmem_regs_after(r[j]);
+          }
+          tc_fence_before();
+          mbar_arrive(&tempty[buf]);  // the accumulator is free; the values are in registers
+          if (active) {
+            const int col0 = ti.n0 + whalf * (NCH * 32);
+            uint8_t* out = static_cast<uint8_t*>(p.C);
+            // 32 rows x 64 bytes; row r's 16-byte chunk q sits at chunk q ^ ((r >> 1) & 3), so both
+            // the row-wise writes and the transposed reads below touch every bank once per 128 bytes
+            uint8_t* tb = wstg;
+#pragma unroll
+            for (int j = 0; j < NCH; ++j) {
+              const int col = col0 + j * 32;
+              if (col >= p.N) continue;  // warp-uniform
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] = acc ? __uint_as_float(r[j][8 * q + i]) : 0.f;
+                st_shared_v4(tb + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4),
+                             make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                                        pack_bf16(v[6], v[7])));
+              }
+              __syncwarp();
+              // each store instruction writes 8 whole 64-byte row segments: row 8i + lane/4,
+              // 16-byte part lane%4
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int rr = 8 * i + (lane >> 2), sg = lane & 3;
+                const uint4 w = ld_shared_v4(tb + rr * 64 + ((sg ^ ((rr >> 1) & 3)) << 4));
+                *reinterpret_cast<uint4*>(out + ((size_t)(c1 + rr) * p.ldc + col) * 2 + sg * 16) = w;
+              }
+              __syncwarp();
+            }
+          }
+        } else if (active) {
           if (half) store(std::integral_constant<int, BN / 2 / 32>{});
           else store(std::integral_constant<int, BN / 32 / (C::EPW / 4)>{});
         }
@@ -992,7 +1044,7 @@ __global__ void __launch_bounds__(Cfg<ES, A_MN, B_MN, BN, EPI, MODE, PAIR>::THRE
         // the leader's MMA thread waits for every epilogue warp of both CTAs of the pair
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty_lead + 8u * (uint32_t)buf);
-      } else {
+      } else if constexpr (!C::EARLY) {
         mbar_arrive(&tempty[buf]);
       }
     }
