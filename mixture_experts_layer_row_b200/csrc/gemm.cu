@@ -71,15 +71,14 @@ struct Cfg {
   static constexpr bool MX = (ES == 1);      // MXFP8 block-scaled (E4M3 operands, UE8M0 scales)
   static_assert(!(PAIR && MX), "block-scaled MMAs run on single CTAs");
   // epilogue warps: four (one per TMEM lane quadrant), or eight (two per quadrant, each taking half
-  // of the accumulator columns) for the MXFP8 wgrad tiles: one accumulator (below) and a contraction of
-  // a few stages, so the accumulator must come back quickly.
-  static constexpr int EPW = (ES == 1 && BN == 256 && MODE == GROUP_K && !PAIR && EPI == EPI_STORE) ? 8 : 4;
-  // The same tiles hold one accumulator (below). There each thread reads its 128 accumulator columns
-  // into registers and hands the accumulator back before it converts and stores them, so the next
-  // tile's MMAs overlap the stores. The stores go through a 2 KB transpose buffer per warp (plain
+  // of the accumulator columns) for the MXFP8 plain-store tiles of 256 columns (fwd2, dgrad1, wgrads),
+  // which hold one accumulator (below). There each thread reads its 128 accumulator columns into
+  // registers and hands the accumulator back before it converts and stores them, so the next tile's
+  // MMAs overlap the stores. The stores go through a 2 KB transpose buffer per warp (plain
   // shared-memory stores and loads, whole 64-byte row segments to global memory) instead of TMA
-  // staging boxes, which leaves room for a fourth pipeline stage: a tile's contraction (512 routed
-  // rows at the MXFP8 shapes) is then loaded while the previous tile computes.
+  // staging boxes; for the wgrads that leaves room for a fourth pipeline stage, so a tile's short
+  // contraction (512 routed rows at the MXFP8 shapes) is loaded while the previous tile computes.
+  static constexpr int EPW = (ES == 1 && BN == 256 && !PAIR && EPI == EPI_STORE) ? 8 : 4;
   static constexpr bool EARLY = EPW == 8;
   static constexpr int THREADS = 64 + 32 * EPW;  // producer, MMA issuer, epilogue
   static constexpr int OES = (EPI == EPI_STORE_F32_BIAS) ? 4 : (MX ? 2 : ES);  // output element size
