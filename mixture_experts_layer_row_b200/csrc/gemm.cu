@@ -4,15 +4,19 @@
 // parallelism completely synchronisation-free", unite.ai "Parallelismo, precisione e tecniche di
 // memoria").
 //
-// Structure (one persistent CTA per SM, or CTA pair per two SMs; 192 threads each):
+// Structure (one persistent CTA per SM, or CTA pair per two SMs; 192 threads each, 320 with eight
+// epilogue warps):
 //   warp 0      TMA producer: one elected thread streams A/B tiles into a STAGES-deep shared-memory
 //               ring (128-byte swizzle), completion counted on a "full" mbarrier per stage;
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN, fp32 accumulate) into
 //               one of NACC TMEM accumulators and frees each ring stage with tcgen05.commit;
 //   warps 2..5  epilogue: tcgen05.ld the finished accumulator (one row per thread), apply the fused
 //               op (store, SwiGLU forward, SwiGLU backward, fp32 + bias) and store to global memory
-//               with TMA, while the MMA thread already fills the other accumulator (NACC = 2; the
-//               256-column MXFP8 tiles have one, their scale columns filling the rest of TMEM).
+//               (TMA stores of staged boxes; the SwiGLU forward's a and the quantised codes straight
+//               from registers), while the MMA thread already fills the other accumulator (NACC = 2).
+//               The 256-column MXFP8 tiles have one accumulator, their scale columns filling the rest
+//               of TMEM; for the plain stores of those tiles eight epilogue warps (2..9) copy it into
+//               registers and hand it back before converting and storing.
 // The tile schedule is built on the device from the routing metadata (counts, padded offsets): the
 // host never learns the group sizes. Two grouping modes:
 //   GROUP_M  ragged rows per expert (forward and dgrad): tiles (expert, n-block, m-block), m fastest
