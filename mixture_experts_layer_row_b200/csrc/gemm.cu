@@ -127,6 +127,12 @@ struct Cfg {
   static constexpr size_t SMEM_BYTES =
       kCtrlBytes + 1024 /*alignment slack*/ + (size_t)STAGES * (STAGE_BYTES + SF_BYTES) +
       STAGING_BYTES;
+  static_assert(SMEM_BYTES <= (size_t)kSmemBudget, "over the opt-in shared memory per CTA");
+  static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0,
+                "stage operands start on 1 KB boundaries (128-byte swizzle atoms)");
+  static_assert(SF_BYTES % 16 == 0, "scale chunks are bulk-copied in 16-byte units");
+  static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0,
+                "TMEM is allocated in powers of two from 32 to 512 columns");
 };
 
 // One tile of the device schedule. lo / hi are the group's row range as read from the routing
